@@ -1,0 +1,196 @@
+"""fine_grained_fp8_x128_b200: fine-grained FP8 training matmuls on B200.
+
+Python binding of the C ABI in include/fp8q.h (libfp8q.so, built in-tree by
+``build.py``).  Argument marshalling only: every step runs in the library's
+sm_100a kernels, on the caller's current CUDA stream.  There is no CPU path;
+if the shared library is missing, importing this package raises.
+
+Each function has the C entry point's name and takes torch CUDA tensors for the
+device buffers (torch is used only for memory and streams).  Sizes and leading
+dimensions are taken from the tensors' shapes and row strides.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libfp8q.so is not built ({LIB_PATH}); run `python -m fine_grained_fp8_x128_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+FP8Q_OK = 0
+FP8Q_ERR_INVALID_ARG = 1
+FP8Q_ERR_ALIGNMENT = 2
+FP8Q_ERR_UNSUPPORTED = 3
+FP8Q_ERR_CUDA = 4
+FP8Q_ERR_TIMEOUT = 5
+FP8Q_SFB_BLOCK128 = 0
+FP8Q_SFB_ROW = 1
+FP8Q_OUT_BF16 = 0
+FP8Q_OUT_F32 = 1
+
+EXPORTS = (
+    "fp8q_version", "fp8q_status_string", "fp8q_device_status",
+    "fp8q_quant_act_1x128", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
+    "fp8q_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled",
+    "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
+)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int64
+_lib.fp8q_version.restype = ctypes.c_int
+_lib.fp8q_status_string.argtypes = [ctypes.c_int]
+_lib.fp8q_status_string.restype = ctypes.c_char_p
+_lib.fp8q_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int)]
+_lib.fp8q_quant_act_1x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_128x1.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_w_128x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_gemm_blockscaled.argtypes = [_P, _I, _P, _I, _P, _I, _P, _I, ctypes.c_int, _P, _I, ctypes.c_int,
+                                       _I, _I, _I, _P]
+_lib.fp8q_grouped_gemm_blockscaled.argtypes = [_P, _I, _P, _I, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P]
+_lib.fp8q_debug_cast_e4m3_bits.argtypes = [ctypes.c_uint32, _I, _P, _P]
+_lib.fp8q_debug_wait_timeout.argtypes = [_I, _P]
+for _n in EXPORTS[2:]:
+    getattr(_lib, _n).restype = ctypes.c_int
+
+
+class FP8QError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: {fp8q_status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def fp8q_version() -> int:
+    return _lib.fp8q_version()
+
+
+def fp8q_status_string(status: int) -> str:
+    return _lib.fp8q_status_string(int(status)).decode()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _ld(t):
+    """Row stride (elements) of a 2D tensor whose last dimension is contiguous."""
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2D tensor with a contiguous last dimension")
+    return t.stride(0)
+
+
+def _check(rc: int, call: str):
+    if rc != FP8Q_OK:
+        raise FP8QError(rc, call)
+
+
+def fp8q_device_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word (0 = clean)."""
+    code = ctypes.c_int(0)
+    rc = _lib.fp8q_device_status(_stream(stream), ctypes.byref(code))
+    if rc not in (FP8Q_OK, FP8Q_ERR_TIMEOUT):
+        raise FP8QError(rc, "fp8q_device_status")
+    return code.value
+
+
+def fp8q_quant_act_1x128(x, q, sf, stream=None):
+    """x bf16 [M][K] -> q uint8 [M][K], sf float32 [K/128][ld_sf >= M] (sf[kb][m])."""
+    M, K = x.shape
+    _check(_lib.fp8q_quant_act_1x128(_ptr(x), M, K, _ld(x), _ptr(q), _ld(q), _ptr(sf), _ld(sf) if sf.dim() == 2 else M,
+                                     _stream(stream)), "fp8q_quant_act_1x128")
+
+
+def fp8q_quant_act_128x1(x, qt, sf, stream=None):
+    """x bf16 [T][C] -> qt uint8 [C][T], sf float32 [T/128][ld_sf >= C]."""
+    T, C = x.shape
+    _check(_lib.fp8q_quant_act_128x1(_ptr(x), T, C, _ld(x), _ptr(qt), _ld(qt), _ptr(sf), _ld(sf), _stream(stream)),
+           "fp8q_quant_act_128x1")
+
+
+def fp8q_quant_w_128x128(w, q, sf, qt=None, sft=None, stream=None):
+    """w bf16 [N][K] -> q [N][K], sf [N/128][K/128]; optional qt [K][N], sft [K/128][N/128]."""
+    N, K = w.shape
+    _check(_lib.fp8q_quant_w_128x128(_ptr(w), N, K, _ld(w), _ptr(q), _ld(q), _ptr(sf), _ld(sf),
+                                     _ptr(qt), _ld(qt) if qt is not None else 0,
+                                     _ptr(sft), _ld(sft) if sft is not None else 0, _stream(stream)),
+           "fp8q_quant_w_128x128")
+
+
+def fp8q_gemm_blockscaled(a, sfa, b, sfb, sfb_mode, d, stream=None):
+    """d[M][N] = block-scaled a[M][K] . b[N][K]^T; d is bf16 or float32."""
+    M, K = a.shape
+    N = b.shape[0]
+    dt = FP8Q_OUT_F32 if d.dtype == torch.float32 else FP8Q_OUT_BF16
+    _check(_lib.fp8q_gemm_blockscaled(_ptr(a), _ld(a), _ptr(sfa), _ld(sfa), _ptr(b), _ld(b), _ptr(sfb), _ld(sfb),
+                                      int(sfb_mode), _ptr(d), _ld(d), dt, M, N, K, _stream(stream)),
+           "fp8q_gemm_blockscaled")
+
+
+def fp8q_grouped_gemm_blockscaled(a, sfa, w, sfw, group_offsets, d, stream=None):
+    """Per-expert block-scaled GEMM; w [G][N][K], sfw [G][N/128][K/128], offsets int32 [G+1] on device."""
+    M_total, K = a.shape
+    G, N, _ = w.shape
+    _check(_lib.fp8q_grouped_gemm_blockscaled(_ptr(a), _ld(a), _ptr(sfa), _ld(sfa), _ptr(w), _ptr(sfw),
+                                              _ptr(group_offsets), G, M_total, _ptr(d), _ld(d), N, K,
+                                              _stream(stream)), "fp8q_grouped_gemm_blockscaled")
+
+
+def fp8q_debug_cast_e4m3_bits(start: int, count: int, out, stream=None):
+    _check(_lib.fp8q_debug_cast_e4m3_bits(ctypes.c_uint32(start & 0xFFFFFFFF), count, _ptr(out), _stream(stream)),
+           "fp8q_debug_cast_e4m3_bits")
+
+
+def fp8q_debug_wait_timeout(budget_cycles: int, stream=None):
+    _check(_lib.fp8q_debug_wait_timeout(int(budget_cycles), _stream(stream)), "fp8q_debug_wait_timeout")
+
+
+# ---------------------------------------------------------------- allocation helpers
+def sf_ld(rows: int) -> int:
+    """Leading dimension used for [K/128][ld] scale arrays (rows rounded up to 4)."""
+    return (rows + 3) // 4 * 4
+
+
+def quant_act_1x128(x, stream=None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=x.device)
+    fp8q_quant_act_1x128(x, q, sf, stream)
+    return q, sf
+
+
+def quant_act_128x1(x, stream=None):
+    T, C = x.shape
+    qt = torch.empty((C, T), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((T // 128, sf_ld(C)), dtype=torch.float32, device=x.device)
+    fp8q_quant_act_128x1(x, qt, sf, stream)
+    return qt, sf
+
+
+def quant_w_128x128(w, transposed: bool = False, stream=None):
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    sf = torch.empty((N // 128, K // 128), dtype=torch.float32, device=w.device)
+    qt = sft = None
+    if transposed:
+        qt = torch.empty((K, N), dtype=torch.uint8, device=w.device)
+        sft = torch.empty((K // 128, N // 128), dtype=torch.float32, device=w.device)
+    fp8q_quant_w_128x128(w, q, sf, qt, sft, stream)
+    return (q, sf, qt, sft) if transposed else (q, sf)

@@ -1,0 +1,324 @@
+// fp8q: the C ABI declared in include/fp8q.h.  Host-side argument checks,
+// TMA descriptor construction and kernel launches; every kernel lives in the
+// headers included below (one translation unit, so the device status word is a
+// single module variable).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fp8q.h"
+#include "device_common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  bool gemm_attr[2][2][2] = {};   // [grouped][row mode][f32 out]
+  bool q2_attr = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+fp8q_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FP8Q_ERR_CUDA;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return FP8Q_ERR_UNSUPPORTED;   // sm_100a code only
+    d.ready = true;
+  }
+  *out = &d;
+  return FP8Q_OK;
+}
+
+fp8q_status encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return FP8Q_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = g_encode;
+  return FP8Q_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fp8q_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+int64_t grid_for(int64_t items, int sm_count, int per_sm) {
+  int64_t g = static_cast<int64_t>(sm_count) * per_sm;
+  if (items < g) g = items;
+  return g < 1 ? 1 : g;
+}
+
+// K-major E4M3 operand [rows][ld] viewed as a 2D tensor {K, rows}; box
+// {128 bytes, box_rows} with the 128-byte swizzle the UMMA descriptors expect.
+fp8q_status make_tmap(CUtensorMap* map, const void* base, int64_t K, int64_t rows, int64_t ld, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  fp8q_status st = encoder(&enc);
+  if (st != FP8Q_OK) return st;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+template <bool G, int MODE, bool F32>
+fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const fp8q::GemmArgs& args,
+                        int grid, cudaStream_t stream) {
+  const uint32_t smem = (G ? fp8q::GemmSmemLayout::bytes_grouped : fp8q::GemmSmemLayout::bytes_dense) + 1024;
+  auto kern = fp8q::gemm_blockscaled_kernel<G, MODE, F32>;
+  bool& attr = dev->gemm_attr[G ? 1 : 0][MODE == FP8Q_SFB_ROW ? 1 : 0][F32 ? 1 : 0];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    attr = true;
+  }
+  kern<<<grid, fp8q::kGemmThreads, smem, stream>>>(ta, tb, args);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8q_version(void) { return 100; }
+
+const char* fp8q_status_string(fp8q_status s) {
+  switch (s) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_INVALID_ARG: return "invalid argument";
+    case FP8Q_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case FP8Q_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case FP8Q_ERR_CUDA: return "CUDA error";
+    case FP8Q_ERR_TIMEOUT: return "device-side bounded wait gave up";
+    default: return "unknown status";
+  }
+}
+
+fp8q_status fp8q_device_status(void* stream, int* out_code) {
+  if (out_code == nullptr) return FP8Q_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int word = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, fp8q::g_status, sizeof(word), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(fp8q::g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  *out_code = static_cast<int>(word);
+  return word == 0 ? FP8Q_OK : FP8Q_ERR_TIMEOUT;
+}
+
+fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
+                                 float* sf, int64_t ld_sf, void* stream) {
+  if (M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  const int64_t grid = grid_for(items, dev->sm_count, 8);
+  fp8q::quant_act_1x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_act_128x1(const void* x, int64_t T, int64_t C, int64_t ldx, void* qt, int64_t ldqt,
+                                 float* sf, int64_t ld_sf, void* stream) {
+  if (T < 0 || C < 0 || T % 128 != 0 || C % 8 != 0 || ldx < C || ldqt < T || ld_sf < C) return FP8Q_ERR_INVALID_ARG;
+  if (T == 0 || C == 0) return FP8Q_OK;
+  if (x == nullptr || qt == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(qt, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldqt % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!dev->q2_attr) {
+      if (cudaFuncSetAttribute(fp8q::quant_act_128x1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fp8q::kQTSmem) != cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      dev->q2_attr = true;
+    }
+  }
+  const int64_t items = (T / 128) * ((C + fp8q::kQTCols - 1) / fp8q::kQTCols);
+  const int64_t grid = grid_for(items, dev->sm_count, 3);
+  fp8q::quant_act_128x1_kernel<<<static_cast<unsigned>(grid), fp8q::kQTThreads, fp8q::kQTSmem,
+                                 static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(x), T, C, ldx,
+                                                                      static_cast<uint8_t*>(qt), ldqt, sf, ld_sf);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_w_128x128(const void* w, int64_t N, int64_t K, int64_t ldw, void* q, int64_t ldq, float* sf,
+                                 int64_t ld_sf, void* qt, int64_t ldqt, float* sft, int64_t ld_sft, void* stream) {
+  if (N < 0 || K < 0 || N % 128 != 0 || K % 128 != 0 || ldw < K || ldq < K || ld_sf < K / 128)
+    return FP8Q_ERR_INVALID_ARG;
+  if (qt != nullptr && ldqt < N) return FP8Q_ERR_INVALID_ARG;
+  if (sft != nullptr && ld_sft < N / 128) return FP8Q_ERR_INVALID_ARG;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (w == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(sf, 4) || ldw % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  if (qt != nullptr && (!aligned(qt, 16) || ldqt % 16 != 0)) return FP8Q_ERR_ALIGNMENT;
+  if (sft != nullptr && !aligned(sft, 4)) return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t NB = N / 128, KB = K / 128;
+  const int64_t grid = grid_for(NB * KB, dev->sm_count, 8);
+  fp8q::quant_w_128x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQWThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w), NB, KB, ldw, static_cast<uint8_t*>(q), ldq, sf, ld_sf,
+      static_cast<uint8_t*>(qt), ldqt, sft, ld_sft);
+  return launch_status();
+}
+
+fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* b,
+                                  int64_t ldb, const float* sfb, int64_t ld_sfb, int sfb_mode, void* d, int64_t ldd,
+                                  int d_dtype, int64_t M, int64_t N, int64_t K, void* stream) {
+  const int64_t kIntMax = 0x7FFFFFFF;
+  if (M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M > kIntMax || N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  if (lda < K || ldb < K || ldd < N || ld_sfa < M) return FP8Q_ERR_INVALID_ARG;
+  if (sfb_mode != FP8Q_SFB_BLOCK128 && sfb_mode != FP8Q_SFB_ROW) return FP8Q_ERR_INVALID_ARG;
+  if (d_dtype != FP8Q_OUT_BF16 && d_dtype != FP8Q_OUT_F32) return FP8Q_ERR_INVALID_ARG;
+  if (sfb_mode == FP8Q_SFB_BLOCK128 && ld_sfb < K / 128) return FP8Q_ERR_INVALID_ARG;
+  if (sfb_mode == FP8Q_SFB_ROW && ld_sfb < N) return FP8Q_ERR_INVALID_ARG;
+  if (a == nullptr || b == nullptr || sfa == nullptr || sfb == nullptr || d == nullptr) return FP8Q_ERR_INVALID_ARG;
+  const int64_t esz = d_dtype == FP8Q_OUT_F32 ? 4 : 2;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfb, 4) ||
+      lda % 16 != 0 || ldb % 16 != 0 || (ldd * esz) % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  if (sfb_mode == FP8Q_SFB_ROW && (!aligned(sfb, 16) || ld_sfb % 4 != 0)) return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, b, K, N, ldb, fp8q::BN)) != FP8Q_OK) return st;
+  fp8q::GemmArgs args{};
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfb;
+  args.ld_sfb = ld_sfb;
+  args.d = d;
+  args.ldd = ldd;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
+  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
+  args.num_m_tiles = static_cast<int>((M + fp8q::BM - 1) / fp8q::BM);
+  args.group_offsets = nullptr;
+  args.G = 1;
+  const int64_t tiles = static_cast<int64_t>(args.num_m_tiles) * args.num_n_tiles;
+  if (tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (sfb_mode == FP8Q_SFB_BLOCK128) {
+    return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, grid, s)
+                                   : launch_gemm<false, FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, grid, s);
+  }
+  return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_ROW, true>(dev, ta, tb, args, grid, s)
+                                 : launch_gemm<false, FP8Q_SFB_ROW, false>(dev, ta, tb, args, grid, s);
+}
+
+fp8q_status fp8q_grouped_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* w,
+                                          const float* sfw, const int32_t* group_offsets, int64_t G, int64_t M_total,
+                                          void* d, int64_t ldd, int64_t N, int64_t K, void* stream) {
+  const int64_t kIntMax = 0x7FFFFFFF;
+  if (G < 1 || M_total < 0 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (G > fp8q::kMaxGroups || M_total > kIntMax || G * N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  if (lda < K || ldd < N || ld_sfa < M_total) return FP8Q_ERR_INVALID_ARG;
+  if (M_total == 0) return FP8Q_OK;
+  if (a == nullptr || w == nullptr || sfa == nullptr || sfw == nullptr || group_offsets == nullptr || d == nullptr)
+    return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(w, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfw, 4) ||
+      !aligned(group_offsets, 4) || lda % 16 != 0 || (ldd * 2) % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = make_tmap(&ta, a, K, M_total, lda, fp8q::BM)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, w, K, G * N, K, fp8q::BN)) != FP8Q_OK) return st;
+  fp8q::GemmArgs args{};
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfw;
+  args.ld_sfb = K / 128;
+  args.d = d;
+  args.ldd = ldd;
+  args.M = static_cast<int>(M_total);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
+  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
+  args.num_m_tiles = 0;
+  args.group_offsets = group_offsets;
+  args.G = static_cast<int>(G);
+  // upper bound on the device-side tile count: every expert wastes at most one partial m-tile
+  const int64_t bound = ((M_total + fp8q::BM - 1) / fp8q::BM + G) * args.num_n_tiles;
+  if (bound > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(bound < dev->sm_count ? bound : dev->sm_count);
+  return launch_gemm<true, FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, grid, static_cast<cudaStream_t>(stream));
+}
+
+fp8q_status fp8q_debug_cast_e4m3_bits(uint32_t start, int64_t count, void* out, void* stream) {
+  if (count < 0 || count > (int64_t(1) << 32)) return FP8Q_ERR_INVALID_ARG;
+  if (count == 0) return FP8Q_OK;
+  if (out == nullptr) return FP8Q_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t pairs = (count + 1) / 2;
+  const int64_t grid = grid_for((pairs + 255) / 256, dev->sm_count, 16);
+  fp8q::cast_e4m3_bits_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      start, count, static_cast<uint8_t*>(out));
+  return launch_status();
+}
+
+fp8q_status fp8q_debug_wait_timeout(int64_t budget_cycles, void* stream) {
+  if (budget_cycles < 1 || budget_cycles > (int64_t(1) << 34)) return FP8Q_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  fp8q::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<long long>(budget_cycles));
+  return launch_status();
+}
+
+}  // extern "C"

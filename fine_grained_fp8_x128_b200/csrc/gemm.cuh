@@ -1,0 +1,401 @@
+// Block-scaled FP8 GEMM for sm_100a: TMA -> shared memory ring -> tcgen05.mma
+// (kind::f8f6f4, E4M3 x E4M3 -> FP32 in tensor memory) -> per-128-K-chunk
+// promotion into FP32 registers on the CUDA cores -> BF16/FP32 store.
+//
+//   D[m,n] = sum_kb sa[m,kb] * sb(n,kb) * P_kb[m,n],
+//   P_kb   = sum over the 128 K of chunk kb of A[m,k] * B[n,k]   (tensor cores)
+//
+// "FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 3
+// "Decoupled Accumulation in Tensor Core GEMMs": FP8 products on the tensor
+// cores, FP32 accumulation, scales s_A * s_B applied in FP32; "Introduction to
+// LLM Quantization", "Fine-grained Quantization" Step 4 (rescale on the CUDA
+// cores) and "3. Increasing accumulation Quantization" (promotion at an
+// interval N_C, here 128 = one scale chunk).
+//
+// Scale factors are FP32 amax/448 values, not powers of two, so the hardware
+// block-scaled MMA (UE8M0 scales) cannot apply them; every chunk gets its own
+// TMEM accumulator and the scale multiply happens in the TMEM -> register path.
+//
+// CTA organisation (one persistent CTA per SM, 384 threads):
+//   warps 0-7  : promotion + epilogue.  Warp w reads TMEM lanes 32*(w%4).. (its
+//                rows) and columns 128*(w/4).. (its half of the 256-wide tile);
+//                each thread keeps 128 FP32 accumulators of one output row.
+//   warp 8     : TMA producer (one lane).
+//   warp 9     : MMA issuer (one lane); also owns the TMEM allocation.
+//   warps 10-11: idle (they complete the third warpgroup for setmaxnreg).
+// Pipelines:
+//   smem ring  : kStages x (A 128x128 + B 256x128 E4M3), full/empty mbarriers.
+//   TMEM       : 2 chunk accumulators of 128 lanes x 256 FP32 columns (all 512
+//                columns): the MMAs of chunk c+1 overlap the promotion of c.
+//   row scales : (FP8Q_SFB_ROW only) a ring of per-chunk B scale vectors.
+// Every wait is bounded (see mbar_wait) and reports through the status word.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace fp8q {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int kStages = 4;
+constexpr int kSbRing = 8;
+constexpr int kGemmThreads = 384;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kABytes = BM * BK;               // 16 KB
+constexpr uint32_t kBBytes = BN * BK;               // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes; // 48 KB
+constexpr uint32_t kSbBytes = BN * 4;               // 1 KB
+constexpr int kMaxGroups = 2048;
+constexpr int kGroupM = 16;                          // L2 swizzle: m-tiles per group
+
+struct GemmSmemLayout {
+  // offsets from the 1024-aligned base
+  static constexpr uint32_t stages = 0;
+  static constexpr uint32_t sb_ring = stages + kStages * kStageBytes;
+  static constexpr uint32_t bars = sb_ring + kSbRing * kSbBytes;
+  // barriers: full[S], empty[S], tfull[2], tempty[2], sbfull[R], sbempty[R]
+  static constexpr uint32_t nbars = 2 * kStages + 4 + 2 * kSbRing;
+  static constexpr uint32_t misc = bars + nbars * 8;           // tmem base, abort flag
+  static constexpr uint32_t prefix = misc + 16;                // grouped: tile prefix [G+1]
+  static constexpr uint32_t offs = prefix + (kMaxGroups + 1) * 4;  // grouped: clamped offsets [G+1]
+  static constexpr uint32_t bytes_dense = prefix;
+  static constexpr uint32_t bytes_grouped = offs + (kMaxGroups + 1) * 4;
+};
+
+struct GemmArgs {
+  const float* sfa;
+  int64_t ld_sfa;
+  const float* sfb;      // dense: per sfb_mode; grouped: sfw [G][N/128][K/128]
+  int64_t ld_sfb;
+  void* d;
+  int64_t ldd;
+  int M;                 // dense: rows of A; grouped: M_total
+  int N;
+  int K;
+  int num_n_tiles;
+  int num_k_chunks;
+  int num_m_tiles;       // dense only
+  const int32_t* group_offsets;  // grouped only
+  int G;
+};
+
+// Which output tile a linear tile id denotes.
+struct TileCoord {
+  int a_row0;     // first row of A (TMA y coordinate)
+  int row_end;    // one past the last valid output row
+  int n0;         // first output column
+  int b_row0;     // first row of B in its tensor map (grouped: g*N + n0)
+  int group;      // expert (grouped) or 0
+};
+
+template <bool kGrouped>
+__device__ __forceinline__ TileCoord tile_coord(int t, const GemmArgs& p, const int* prefix,
+                                                const int* offs) {
+  TileCoord c;
+  if (!kGrouped) {
+    const int per_group = kGroupM * p.num_n_tiles;
+    const int grp = t / per_group;
+    const int first_m = grp * kGroupM;
+    const int gm = min(kGroupM, p.num_m_tiles - first_m);
+    const int within = t - grp * per_group;
+    const int mt = first_m + within % gm;
+    const int nt = within / gm;
+    c.a_row0 = mt * BM;
+    c.row_end = min(p.M, c.a_row0 + BM);
+    c.n0 = nt * BN;
+    c.b_row0 = c.n0;
+    c.group = 0;
+  } else {
+    // largest g with prefix[g] <= t (empty experts share a prefix and are skipped)
+    int lo = 0, hi = p.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    const int local = t - prefix[g];
+    const int rows = offs[g + 1] - offs[g];
+    const int mtiles = (rows + BM - 1) / BM;
+    const int mt = local % mtiles;
+    const int nt = local / mtiles;
+    c.a_row0 = offs[g] + mt * BM;
+    c.row_end = min(offs[g + 1], c.a_row0 + BM);
+    c.n0 = nt * BN;
+    c.b_row0 = g * p.N + c.n0;
+    c.group = g;
+  }
+  return c;
+}
+
+__device__ __forceinline__ void setmaxnreg_inc232() { asm volatile("setmaxnreg.inc.sync.aligned.u32 232;"); }
+__device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;"); }
+
+}  // namespace fp8q
+
+namespace fp8q {
+
+// Multiply 32 chunk partials by one scale and add them to the accumulators.
+__device__ __forceinline__ void promote32(float* acc, const uint32_t (&v)[32], float scale) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(v[j]), scale, acc[j]);
+}
+
+// Per-column scales (FP8Q_SFB_ROW): acc[j] += v[j] * (sa * sb[j]).
+__device__ __forceinline__ void promote32_rows(float* acc, const uint32_t (&v)[32], float sa,
+                                               const float* sb) {
+  const float4* s4 = reinterpret_cast<const float4*>(sb);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 s = s4[q];
+    acc[4 * q + 0] = fmaf(__uint_as_float(v[4 * q + 0]), sa * s.x, acc[4 * q + 0]);
+    acc[4 * q + 1] = fmaf(__uint_as_float(v[4 * q + 1]), sa * s.y, acc[4 * q + 1]);
+    acc[4 * q + 2] = fmaf(__uint_as_float(v[4 * q + 2]), sa * s.z, acc[4 * q + 2]);
+    acc[4 * q + 3] = fmaf(__uint_as_float(v[4 * q + 3]), sa * s.w, acc[4 * q + 3]);
+  }
+}
+
+template <bool kGrouped, int kSfbMode, bool kOutF32>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                        const GemmArgs p) {
+  extern __shared__ uint8_t gemm_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmemLayout::bars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* sbfull = tempty + 2;
+  uint64_t* sbempty = sbfull + kSbRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GemmSmemLayout::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + GemmSmemLayout::misc + 4);
+  int* prefix = reinterpret_cast<int*>(smem + GemmSmemLayout::prefix);
+  int* offs = reinterpret_cast<int*>(smem + GemmSmemLayout::offs);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nk = p.num_k_chunks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kEpiWarps); }
+    for (int r = 0; r < kSbRing; ++r) { mbar_init(&sbfull[r], 1); mbar_init(&sbempty[r], kEpiWarps); }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8 && lane == 0) { prefetch_tmap(&tmap_a); prefetch_tmap(&tmap_b); }
+  if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  if (kGrouped && warp == 0) {
+    // Clamp the device-side offsets into [0, M_total], force them nondecreasing
+    // (warp max-scan), then the exclusive prefix of each expert's tile count.
+    bool bad = false;
+    int carry = 0;
+    for (int g0 = 0; g0 <= p.G; g0 += 32) {
+      const int g = g0 + lane;
+      int o = 0;
+      if (g <= p.G) {
+        const int raw = p.group_offsets[g];
+        o = min(max(raw, 0), p.M);
+        bad |= (o != raw);
+      }
+      int m = o;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, m, d);
+        if (lane >= d) m = max(m, v);
+      }
+      m = max(m, carry);
+      if (g <= p.G) { bad |= (m != o); offs[g] = m; }
+      carry = __shfl_sync(0xFFFFFFFFu, m, 31);
+    }
+    __syncwarp();
+    if (lane == 0) bad |= (offs[0] != 0) || (offs[p.G] != p.M);
+    int tcarry = 0;
+    for (int g0 = 0; g0 < p.G; g0 += 32) {
+      const int g = g0 + lane;
+      const int tg = (g < p.G) ? ((offs[g + 1] - offs[g] + BM - 1) / BM) * p.num_n_tiles : 0;
+      int s = tg;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, s, d);
+        if (lane >= d) s += v;
+      }
+      if (g < p.G) prefix[g] = tcarry + s - tg;
+      tcarry += __shfl_sync(0xFFFFFFFFu, s, 31);
+    }
+    if (lane == 0) prefix[p.G] = tcarry;
+    bad = __any_sync(0xFFFFFFFFu, bad);
+    if (bad && lane == 0 && blockIdx.x == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_GROUP_OFFSETS);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = kGrouped ? prefix[p.G] : p.num_m_tiles * p.num_n_tiles;
+
+  if (warp >= kEpiWarps) {
+    setmaxnreg_dec40();
+    if (warp == 8) {
+      // ---------------- TMA producer ----------------
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+        const TileCoord c = tile_coord<kGrouped>(t, p, prefix, offs);
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!warp_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+          if (kSfbMode == FP8Q_SFB_ROW) {
+            const int r = it % kSbRing;
+            if (!warp_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+            if (lane == 0) {
+              const uint32_t nbytes = static_cast<uint32_t>(min(BN, p.N - c.n0)) * 4u;
+              mbar_arrive_expect_tx(&sbfull[r], nbytes);
+              bulk_load(smem + GemmSmemLayout::sb_ring + r * kSbBytes,
+                        p.sfb + static_cast<int64_t>(kc) * p.ld_sfb + c.n0, nbytes, &sbfull[r]);
+            }
+          }
+          if (lane == 0) {
+            uint8_t* st = smem + GemmSmemLayout::stages + s * kStageBytes;
+            mbar_arrive_expect_tx(&full[s], kStageBytes);
+            tma_load_2d_nohint(st, &tmap_a, &full[s], kc * BK, c.a_row0);
+            tma_load_2d_nohint(st + kABytes, &tmap_b, &full[s], kc * BK, c.b_row0);
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok) {
+        // error path: let the copies already in flight land before the CTA exits
+        for (int j = max(0, it - kStages); j < it; ++j)
+          warp_wait(&full[j % kStages], (j / kStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+      }
+    } else if (warp == 9) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t idesc = umma_idesc_e4m3_f32(BM, BN);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          const int b = it & 1;
+          const uint32_t bph = (it >> 1) & 1;
+          if (!warp_wait(&tempty[b], bph ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY)) { ok = false; break; }
+          if (!warp_wait(&full[s], ph, abort_flag, WAIT_MMA_FULL)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(smem + GemmSmemLayout::stages + s * kStageBytes);
+            const uint32_t b_addr = a_addr + kABytes;
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k)
+              umma_f8f6f4(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
+                          k > 0 ? 1u : 0u);
+            umma_commit(&empty[s]);
+            umma_commit(&tfull[b]);
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok && it > 0) {
+        // error path: the last issued MMAs must finish reading shared memory
+        const int j = it - 1;
+        warp_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+      }
+    }
+  } else {
+    // ---------------- promotion + epilogue (warps 0-7) ----------------
+    setmaxnreg_inc232();
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int r_in_tile = quad * 32 + lane;
+    const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
+    const int nb_per_group = p.N / 128;
+    float acc[128];
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+      const TileCoord c = tile_coord<kGrouped>(t, p, prefix, offs);
+      const int row = c.a_row0 + r_in_tile;
+      const bool vrow = row < c.row_end;
+      const int ncol0 = c.n0 + half * 128;
+      const bool vcol = ncol0 < p.N;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      for (int kc = 0; kc < nk; ++kc, ++it) {
+        const int b = it & 1;
+        const uint32_t bph = (it >> 1) & 1;
+        const float sa = vrow ? __ldg(p.sfa + static_cast<int64_t>(kc) * p.ld_sfa + row) : 0.0f;
+        float sbk = 0.0f;
+        if (kSfbMode == FP8Q_SFB_BLOCK128 && vcol) {
+          if (kGrouped)
+            sbk = __ldg(p.sfb + (static_cast<int64_t>(c.group) * nb_per_group + ncol0 / 128) * nk + kc);
+          else
+            sbk = __ldg(p.sfb + static_cast<int64_t>(ncol0 / 128) * p.ld_sfb + kc);
+        }
+        if (!warp_wait(&tfull[b], bph, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
+        const float* sbv = nullptr;
+        int r = 0;
+        if (kSfbMode == FP8Q_SFB_ROW) {
+          r = it % kSbRing;
+          if (!warp_wait(&sbfull[r], (it / kSbRing) & 1, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
+          sbv = reinterpret_cast<const float*>(smem + GemmSmemLayout::sb_ring + r * kSbBytes) + half * 128;
+        }
+        tc_fence_after();
+        const float scale = sa * sbk;
+        const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(taddr, v0);
+        tmem_ld_wait_tied(v0);
+        tmem_ld_32x32b_x32(taddr + 32, v1);
+        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc, v0, sa, sbv); else promote32(acc, v0, scale);
+        tmem_ld_wait_tied(v1);
+        tmem_ld_32x32b_x32(taddr + 64, v0);
+        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc + 32, v1, sa, sbv + 32); else promote32(acc + 32, v1, scale);
+        tmem_ld_wait_tied(v0);
+        tmem_ld_32x32b_x32(taddr + 96, v1);
+        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc + 64, v0, sa, sbv + 64); else promote32(acc + 64, v0, scale);
+        tmem_ld_wait_tied(v1);
+        // every TMEM read of this buffer has completed: hand it back to the MMA warp
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc + 96, v1, sa, sbv + 96); else promote32(acc + 96, v1, scale);
+        if (kSfbMode == FP8Q_SFB_ROW) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sbempty[r]);
+        }
+      }
+      if (!ok) break;
+      if (vrow && vcol) {
+        if (kOutF32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * i + 2 * j], acc[8 * i + 2 * j + 1]);
+              w[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace fp8q

@@ -1,0 +1,267 @@
+// Online quantizers: 1x128 activation tiles, 128x1 transposed tiles, 128x128
+// weight blocks.  All three are HBM-bound streaming kernels: 16-byte coalesced
+// loads, a register/shuffle amax per tile, the scale s = amax/448 and the
+// saturating E4M3 cast fused into one store pass.
+//
+// Passages: "Fine-Grained FP8 Quantization in DeepSeek", sections 2-3;
+// "FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 1 (eq. s_W,
+// eq. W_FP8); "Introduction to LLM Quantization", "5) Online Quantization".
+#pragma once
+
+#include "device_common.cuh"
+
+namespace fp8q {
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float amax_word(float m, uint32_t w) {
+  return fmaxf(m, fmaxf(fabsf(bf16lo(w)), fabsf(bf16hi(w))));
+}
+
+// Two BF16 values (one word) -> two E4M3 codes (low byte first).
+__device__ __forceinline__ uint32_t quant_word(uint32_t w, float r, float s) {
+  return cvt_e4m3x2(scaled_for_cast(bf16lo(w), r, s), scaled_for_cast(bf16hi(w), r, s));
+}
+
+// ---------------------------------------------------------------------------
+// 1x128 tiles.  8 consecutive lanes own one tile (16 elements each, two
+// 16-byte loads).  A 256-thread block covers 32 tiles: rows r0..r0+31 of one
+// 128-column chunk kb, so the 32 scales it writes, sf[kb*ld_sf + r0 ..], are
+// one contiguous 128-byte line.
+// ---------------------------------------------------------------------------
+constexpr int kQ1Threads = 256;
+constexpr int kQ1Rows = 32;
+
+__global__ void __launch_bounds__(kQ1Threads)
+quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
+                       uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf) {
+  const int tid = threadIdx.x;
+  const int sub = tid & 7;           // 16-element slice within the tile
+  const int tile = tid >> 3;         // 0..31: row within the block's 32 rows
+  const int64_t row_blocks = (M + kQ1Rows - 1) / kQ1Rows;
+  const int64_t items = row_blocks * KB;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int64_t rb = it / KB;
+    const int64_t kb = it - rb * KB;
+    const int64_t row = rb * kQ1Rows + tile;
+    const bool active = row < M;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+    const int64_t col = kb * 128 + sub * 16;
+    if (active) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + row * ldx + col);
+      v0 = __ldg(src);
+      v1 = __ldg(src + 1);
+    }
+    float m = 0.0f;
+    m = amax_word(m, v0.x); m = amax_word(m, v0.y); m = amax_word(m, v0.z); m = amax_word(m, v0.w);
+    m = amax_word(m, v1.x); m = amax_word(m, v1.y); m = amax_word(m, v1.z); m = amax_word(m, v1.w);
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+    const float s = tile_scale(m);
+    const float r = __frcp_rn(s);
+    if (active) {
+      uint4 o;
+      o.x = quant_word(v0.x, r, s) | (quant_word(v0.y, r, s) << 16);
+      o.y = quant_word(v0.z, r, s) | (quant_word(v0.w, r, s) << 16);
+      o.z = quant_word(v1.x, r, s) | (quant_word(v1.y, r, s) << 16);
+      o.w = quant_word(v1.z, r, s) | (quant_word(v1.w, r, s) << 16);
+      *reinterpret_cast<uint4*>(q + row * ldq + col) = o;
+      if (sub == 0) sf[kb * ld_sf + row] = s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 128x1 tiles along the token dimension, written transposed.  A block stages a
+// 128-token x 256-channel BF16 tile (64 KB) in shared memory with cp.async;
+// thread j then owns channels 2j and 2j+1: one bank-conflict-free 32-bit
+// shared load per token gives both, the amax is a register reduction, and the
+// 128 codes of each channel leave as eight 16-byte stores of the row qt[c].
+// ---------------------------------------------------------------------------
+constexpr int kQTThreads = 128;
+constexpr int kQTCols = 256;
+constexpr int kQTSmem = 128 * kQTCols * 2;   // 65536
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kQTThreads)
+quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C, int64_t ldx,
+                       uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sf, int64_t ld_sf) {
+  extern __shared__ __align__(128) uint8_t q2_smem[];
+  uint32_t* tile = reinterpret_cast<uint32_t*>(q2_smem);   // [128 tokens][128 words]
+  const int tid = threadIdx.x;
+  const int64_t col_blocks = (C + kQTCols - 1) / kQTCols;
+  const int64_t items = (T / 128) * col_blocks;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int64_t tb = it / col_blocks;
+    const int64_t c0 = (it - tb * col_blocks) * kQTCols;
+    const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;   // multiple of 8
+    const int chunks_per_row = static_cast<int>(ncols / 8);          // 16-byte chunks
+    // stage: 128 rows x ncols channels
+    for (int i = tid; i < 128 * (kQTCols / 8); i += kQTThreads) {
+      const int rr = i / (kQTCols / 8);
+      const int cc = i % (kQTCols / 8);
+      if (cc < chunks_per_row)
+        cp_async16(&tile[rr * (kQTCols / 2) + cc * 4], x + (tb * 128 + rr) * ldx + c0 + cc * 8);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    const int64_t ca = c0 + 2 * tid;          // this thread's channels ca, ca + 1
+    if (ca < C) {
+      float ma = 0.0f, mb = 0.0f;
+#pragma unroll 16
+      for (int t = 0; t < 128; ++t) {
+        const uint32_t w = tile[t * (kQTCols / 2) + tid];
+        ma = fmaxf(ma, fabsf(bf16lo(w)));
+        mb = fmaxf(mb, fabsf(bf16hi(w)));
+      }
+      const float sa = tile_scale(ma), sb = tile_scale(mb);
+      const float ra = __frcp_rn(sa), rb = __frcp_rn(sb);
+      uint8_t* qa = qt + ca * ldqt + tb * 128;
+      uint8_t* qb = qa + ldqt;
+#pragma unroll 1
+      for (int t0 = 0; t0 < 128; t0 += 16) {
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t a4 = 0, b4 = 0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int t = t0 + 4 * j + 2 * h;
+            const uint32_t w0 = tile[t * (kQTCols / 2) + tid];
+            const uint32_t w1 = tile[(t + 1) * (kQTCols / 2) + tid];
+            a4 |= cvt_e4m3x2(scaled_for_cast(bf16lo(w0), ra, sa), scaled_for_cast(bf16lo(w1), ra, sa)) << (16 * h);
+            b4 |= cvt_e4m3x2(scaled_for_cast(bf16hi(w0), rb, sb), scaled_for_cast(bf16hi(w1), rb, sb)) << (16 * h);
+          }
+          oa[j] = a4;
+          ob[j] = b4;
+        }
+        *reinterpret_cast<uint4*>(qa + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *reinterpret_cast<uint4*>(qb + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+      }
+      sf[tb * ld_sf + ca] = sa;
+      sf[tb * ld_sf + ca + 1] = sb;
+    }
+    __syncthreads();   // the tile buffer is reused by the next item
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 128x128 weight blocks, with the optional transposed copy for Dgrad.  One
+// 256-thread block per weight block; thread t owns the 8x8 sub-block at rows
+// 8*(t/16).., columns 8*(t%16)..: eight 16-byte row loads (16 lanes cover one
+// 256-byte row), block amax via shuffles and shared memory, eight 8-byte Q
+// stores, and, for Q^T, an in-register 8x8 byte transpose (byte permutes)
+// followed by eight 8-byte stores of the transposed rows.
+// ---------------------------------------------------------------------------
+constexpr int kQWThreads = 256;
+
+// 4x4 byte transpose: in a[i] = row i (byte j = column j); out c[j] = column j.
+__device__ __forceinline__ void transpose4x4(const uint32_t a0, const uint32_t a1, const uint32_t a2,
+                                             const uint32_t a3, uint32_t (&c)[4]) {
+  const uint32_t t0 = __byte_perm(a0, a1, 0x5140);   // a0.b0 a1.b0 a0.b1 a1.b1
+  const uint32_t t1 = __byte_perm(a0, a1, 0x7362);   // a0.b2 a1.b2 a0.b3 a1.b3
+  const uint32_t t2 = __byte_perm(a2, a3, 0x5140);
+  const uint32_t t3 = __byte_perm(a2, a3, 0x7362);
+  c[0] = __byte_perm(t0, t2, 0x5410);
+  c[1] = __byte_perm(t0, t2, 0x7632);
+  c[2] = __byte_perm(t1, t3, 0x5410);
+  c[3] = __byte_perm(t1, t3, 0x7632);
+}
+
+__global__ void __launch_bounds__(kQWThreads)
+quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t KB, int64_t ldw,
+                       uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
+                       uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sft, int64_t ld_sft) {
+  __shared__ float warp_max[kQWThreads / 32];
+  const int tid = threadIdx.x;
+  const int a = tid >> 4;        // rows 8a .. 8a+7
+  const int b = tid & 15;        // cols 8b .. 8b+7
+  const int64_t items = NB * KB;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int64_t nb = it / KB;
+    const int64_t kb = it - nb * KB;
+    const int64_t n0 = nb * 128, k0 = kb * 128;
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = __ldg(reinterpret_cast<const uint4*>(w + (n0 + 8 * a + i) * ldw + k0 + 8 * b));
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      m = amax_word(m, v[i].x); m = amax_word(m, v[i].y);
+      m = amax_word(m, v[i].z); m = amax_word(m, v[i].w);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((tid & 31) == 0) warp_max[tid >> 5] = m;
+    __syncthreads();
+    m = warp_max[0];
+#pragma unroll
+    for (int i = 1; i < kQWThreads / 32; ++i) m = fmaxf(m, warp_max[i]);
+    const float s = tile_scale(m);
+    const float r = __frcp_rn(s);
+    uint32_t lo[8], hi[8];   // row i: bytes of columns 0-3 (lo) and 4-7 (hi)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      lo[i] = quant_word(v[i].x, r, s) | (quant_word(v[i].y, r, s) << 16);
+      hi[i] = quant_word(v[i].z, r, s) | (quant_word(v[i].w, r, s) << 16);
+      *reinterpret_cast<uint2*>(q + (n0 + 8 * a + i) * ldq + k0 + 8 * b) = make_uint2(lo[i], hi[i]);
+    }
+    if (qt != nullptr) {
+      uint32_t c00[4], c01[4], c10[4], c11[4];   // c<rowhalf><colhalf>
+      transpose4x4(lo[0], lo[1], lo[2], lo[3], c00);
+      transpose4x4(hi[0], hi[1], hi[2], hi[3], c01);
+      transpose4x4(lo[4], lo[5], lo[6], lo[7], c10);
+      transpose4x4(hi[4], hi[5], hi[6], hi[7], c11);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        *reinterpret_cast<uint2*>(qt + (k0 + 8 * b + j) * ldqt + n0 + 8 * a) = make_uint2(c00[j], c10[j]);
+        *reinterpret_cast<uint2*>(qt + (k0 + 8 * b + 4 + j) * ldqt + n0 + 8 * a) = make_uint2(c01[j], c11[j]);
+      }
+    }
+    if (tid == 0) {
+      sf[nb * ld_sf + kb] = s;
+      if (sft != nullptr) sft[kb * ld_sft + nb] = s;
+    }
+    __syncthreads();   // warp_max is reused by the next block
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostics: the E4M3 cast over consecutive FP32 bit patterns.
+// ---------------------------------------------------------------------------
+__global__ void cast_e4m3_bits_kernel(uint32_t start, int64_t count, uint8_t* __restrict__ out) {
+  const int64_t pairs = (count + 1) / 2;
+  for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p < pairs;
+       p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t b0 = start + static_cast<uint32_t>(2 * p);
+    const uint32_t code = cvt_e4m3x2(__uint_as_float(b0), __uint_as_float(b0 + 1u));
+    out[2 * p] = static_cast<uint8_t>(code & 0xFF);
+    if (2 * p + 1 < count) out[2 * p + 1] = static_cast<uint8_t>(code >> 8);
+  }
+}
+
+// One block waits on a barrier that nothing completes; the bounded wait gives
+// up after `budget` clocks and records FP8Q_ERR_TIMEOUT.
+__global__ void wait_timeout_kernel(long long budget) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, WAIT_DEBUG, budget);
+  __syncthreads();
+}
+
+}  // namespace fp8q

@@ -1,0 +1,209 @@
+/*
+ * fp8q -- fine-grained FP8 training matmuls for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every entry point takes plain pointers and sizes; no C++ or torch
+ * types cross this boundary.  Page citations name the page title and section:
+ *   "Fine-Grained FP8 Quantization in DeepSeek"                  (shivam2003.com)
+ *   "FP8 Mixed Precision: DeepSeek-V3 Training Architecture"      (aifetchly)
+ *   "Introduction to LLM Quantization"                            (medium)
+ *   "Online Quantization During Training"                         (shivam2003.com)
+ *
+ * Conventions shared by every call:
+ *  - Pointers named x, w, q, qt, sf, a, b, d, group_offsets are DEVICE memory
+ *    owned by the caller.  The library never frees or retains them.
+ *  - Sizes and leading dimensions (ld*) are element counts (int64_t).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Kernels are enqueued asynchronously on it; the call returns after host
+ *    validation and launch.
+ *  - Return value: FP8Q_OK or an error code.  Invalid arguments are reported
+ *    synchronously and nothing is launched.  Nothing throws across the ABI.
+ *  - Outputs are written entirely (no accumulation into an existing output).
+ *    Inputs and outputs must not overlap.
+ *  - Inputs are finite BF16 values; behaviour for Inf/NaN inputs is unspecified.
+ *  - The library allocates no per-call memory and no workspace.
+ *  - E4M3 is the OCP "E4M3FN" encoding (bias 7, max 448, no infinities).
+ *    The cast is round-to-nearest-even with saturation to +-448.
+ *  - Tile scale: s = max(fl32(amax / 448), fl32(1e-12)), IEEE FP32 division;
+ *    q = e4m3(fl32(x / s)), IEEE FP32 division.  s is stored (dequantised
+ *    value = decode(q) * s).
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int fp8q_status;
+
+enum {
+  FP8Q_OK = 0,
+  FP8Q_ERR_INVALID_ARG = 1,  /* a size, leading dimension or mode is invalid    */
+  FP8Q_ERR_ALIGNMENT = 2,    /* a pointer or leading dimension is misaligned    */
+  FP8Q_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement     */
+  FP8Q_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed     */
+  FP8Q_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (device status) */
+};
+
+/* Scale layouts for operand B of fp8q_gemm_blockscaled. */
+enum {
+  FP8Q_SFB_BLOCK128 = 0, /* 128x128 weight blocks: sfb[(n/128) * ld_sfb + kb], ld_sfb >= K/128 */
+  FP8Q_SFB_ROW = 1       /* one scale per row and K chunk: sfb[kb * ld_sfb + n], ld_sfb >= N */
+};
+
+/* Output element types of the GEMMs. */
+enum {
+  FP8Q_OUT_BF16 = 0, /* round-to-nearest-even BF16 */
+  FP8Q_OUT_F32 = 1   /* FP32 */
+};
+
+/* Library version (major*10000 + minor*100 + patch). */
+int fp8q_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fp8q_status_string(fp8q_status s);
+
+/*
+ * Synchronise `stream`, then read and clear this device's sticky device-side
+ * status word.  *out_code receives the raw word: 0 when no kernel reported a
+ * problem; otherwise bits 0-7 hold an FP8Q_ERR_* code and bits 8-31 say which
+ * wait gave up.  Returns FP8Q_OK, FP8Q_ERR_TIMEOUT when the word was non-zero,
+ * or FP8Q_ERR_CUDA.
+ */
+fp8q_status fp8q_device_status(void* stream, int* out_code);
+
+/*
+ * Online 1x128 activation quantization.
+ * "Fine-Grained FP8 Quantization in DeepSeek", section 2 "Activations use 1x128
+ * tiles"; "FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 1
+ * "Fine-Grained Tile and Block-Wise Scaling" (eq. s = max|tile|/448, eq. W_FP8);
+ * "Introduction to LLM Quantization", "5) Online Quantization".
+ *
+ *   x  : BF16 [M][ldx], row-major (token m, channel k).
+ *   q  : E4M3 bytes [M][ldq]; q[m*ldq + k].
+ *   sf : FP32 scales, logical [M][K/128], stored K-chunk-major:
+ *        sf[(k/128) * ld_sf + m] (the layout the GEMM reads for operand A).
+ * Requirements: M >= 0, K % 128 == 0, ldx >= K, ldq >= K, ld_sf >= M;
+ * x and q 16-byte aligned, ldx % 8 == 0, ldq % 16 == 0; sf 4-byte aligned
+ * (else FP8Q_ERR_ALIGNMENT).  M == 0 or K == 0 launches nothing.
+ */
+fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                 void* q, int64_t ldq, float* sf, int64_t ld_sf,
+                                 void* stream);
+
+/*
+ * Online 128x1 quantization along the token dimension, written transposed:
+ * the layout both Wgrad operands need (dL/dW = x^T (dL/dz), "Introduction to
+ * LLM Quantization", "3) Backward propagation"; "Fine-Grained FP8 Quantization
+ * in DeepSeek", section 4: transpose layout).  Same tile rule as above with
+ * tiles of 128 consecutive tokens of one channel.
+ *
+ *   x  : BF16 [T][ldx] (token t, channel c).
+ *   qt : E4M3 [C][ldqt]; qt[c*ldqt + t].
+ *   sf : FP32 [T/128][ld_sf]; sf[(t/128) * ld_sf + c]  (operand-A layout for
+ *        a GEMM whose rows are channels and whose K is tokens).
+ * Requirements: T % 128 == 0, C >= 0, C % 8 == 0, ldx >= C, ldqt >= T,
+ * ld_sf >= C; x, qt 16-byte aligned, ldx % 8 == 0, ldqt % 16 == 0.
+ */
+fp8q_status fp8q_quant_act_128x1(const void* x, int64_t T, int64_t C, int64_t ldx,
+                                 void* qt, int64_t ldqt, float* sf, int64_t ld_sf,
+                                 void* stream);
+
+/*
+ * 128x128 weight block quantization ("Fine-Grained FP8 Quantization in
+ * DeepSeek", section 3 "Weights use 128x128 blocks"; "FP8 Mixed Precision",
+ * eq. s_W = max|W_block| / 448).  Run once per optimizer step; the result is
+ * reused by forward and backward ("Online Quantization During Training",
+ * section 3 "Weights occupy a middle ground").
+ *
+ *   w   : BF16 [N][ldw] (output feature n, input feature k).
+ *   q   : E4M3 [N][ldq].            sf : FP32 [N/128][ld_sf], sf[nb*ld_sf + kb].
+ *   qt  : optional E4M3 W^T [K][ldqt] (NULL to skip) -- operand B of Dgrad.
+ *   sft : optional FP32 [K/128][ld_sft] transposed scale grid (NULL to skip).
+ * The block scale is invariant under transposition, so qt/sft are exactly the
+ * quantization of W^T.
+ * Requirements: N % 128 == 0, K % 128 == 0, ldw >= K, ldq >= K,
+ * ld_sf >= K/128, (qt: ldqt >= N, ldqt % 16 == 0), (sft: ld_sft >= N/128);
+ * w, q, qt 16-byte aligned, ldw % 8 == 0, ldq % 16 == 0.
+ */
+fp8q_status fp8q_quant_w_128x128(const void* w, int64_t N, int64_t K, int64_t ldw,
+                                 void* q, int64_t ldq, float* sf, int64_t ld_sf,
+                                 void* qt, int64_t ldqt, float* sft, int64_t ld_sft,
+                                 void* stream);
+
+/*
+ * Block-scaled FP8 GEMM with FP32 promotion at every 128-wide K chunk:
+ *   D[m,n] = sum_kb  sa[m,kb] * sb(n,kb) * ( sum_{k in chunk kb} A[m,k] * B[n,k] )
+ * "FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 3
+ * "Decoupled Accumulation in Tensor Core GEMMs" (eq. C_ij, per K chunk);
+ * "Introduction to LLM Quantization", "Fine-grained Quantization" Steps 1-4 and
+ * "3. Increasing accumulation Quantization".  The chunk products run on the
+ * tensor cores; the scale multiply and FP32 accumulation run on the CUDA cores.
+ *
+ *   a   : E4M3 [M][lda], K-major.   sfa : FP32 sfa[kb * ld_sfa + m], ld_sfa >= M.
+ *   b   : E4M3 [N][ldb], K-major.   sfb : per sfb_mode (FP8Q_SFB_BLOCK128 for a
+ *         128x128-block weight -- Fprop, Dgrad with b = W^T; FP8Q_SFB_ROW for
+ *         per-row 128x1 tiles -- Wgrad).
+ *   d   : [M][ldd] of d_dtype (FP8Q_OUT_BF16 or FP8Q_OUT_F32).
+ * Requirements: M >= 1, N % 128 == 0, N >= 128, K % 128 == 0, K >= 128,
+ * lda >= K, ldb >= K, ldd >= N; a, b 16-byte aligned, lda % 16 == 0,
+ * ldb % 16 == 0; d 16-byte aligned and ldd * sizeof(elem) % 16 == 0.
+ * The result is deterministic for fixed inputs.
+ */
+fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                  const void* b, int64_t ldb, const float* sfb, int64_t ld_sfb,
+                                  int sfb_mode, void* d, int64_t ldd, int d_dtype,
+                                  int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Grouped (MoE expert) block-scaled FP8 GEMM.  For each expert g, rows
+ * [off[g], off[g+1]) of the expert-packed activations are multiplied by that
+ * expert's 128x128-block weight, with the semantics of fp8q_gemm_blockscaled
+ * (FP8Q_SFB_BLOCK128, BF16 out).  The per-expert sizes are read on the device
+ * only: the host needs M_total (tokens * top_k) and nothing else, so no host
+ * synchronisation is needed.  MoE context: "FP8 Mixed Precision: DeepSeek-V3
+ * Training Architecture", sections 2 "The MoE Inter-Node All-to-All
+ * Communication Wall" and 4 "Low-Precision Systems Co-Design".
+ *
+ *   a   : E4M3 [M_total][lda]; sfa[kb * ld_sfa + m], ld_sfa >= M_total.
+ *   w   : E4M3 [G][N][K] (expert-major, rows K-major, packed).
+ *   sfw : FP32 [G][N/128][K/128] packed.
+ *   group_offsets : device int32 [G+1], nondecreasing, off[0] = 0,
+ *         off[G] = M_total.  Offsets outside [0, M_total] are clamped and the
+ *         device status word records FP8Q_ERR_INVALID_ARG.
+ *   d   : BF16 [M_total][ldd].
+ * Requirements: G >= 1, M_total >= 0, N % 128 == 0, K % 128 == 0, lda >= K,
+ * ldd >= N; alignment as for fp8q_gemm_blockscaled.
+ */
+fp8q_status fp8q_grouped_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                          const void* w, const float* sfw,
+                                          const int32_t* group_offsets, int64_t G, int64_t M_total,
+                                          void* d, int64_t ldd, int64_t N, int64_t K,
+                                          void* stream);
+
+/* ---- diagnostics (used by the test suite; not on the hot path) ---------- */
+
+/*
+ * Cast the `count` FP32 values whose bit patterns are start, start+1, ...
+ * (wrapping modulo 2^32) with the same E4M3 conversion the quantizers use,
+ * writing one byte each to out[0..count).  Lets a test compare the device cast
+ * with an independent encoder over every FP32 input.  count <= 2^32.
+ */
+fp8q_status fp8q_debug_cast_e4m3_bits(uint32_t start, int64_t count, void* out, void* stream);
+
+/*
+ * Launch one block that waits on a barrier no thread ever completes, with a
+ * wait budget of `budget_cycles` SM clocks (1 <= budget <= 2^34).  The wait
+ * gives up, records FP8Q_ERR_TIMEOUT in the device status word and the kernel
+ * returns; fp8q_device_status() then reports it.  Exercises the same bounded
+ * wait every pipeline wait in the library uses, without hanging the device.
+ */
+fp8q_status fp8q_debug_wait_timeout(int64_t budget_cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

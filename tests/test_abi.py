@@ -1,0 +1,122 @@
+"""The C-ABI boundary on the host (no GPU needed): the library loads, exports
+every entry point include/fp8q.h declares, and rejects invalid arguments with
+the documented status codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from common import load_fp8q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+FAKE = 1 << 20        # 16-byte aligned fake device address (never dereferenced)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8q_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def fp8q():
+    return load_fp8q()
+
+
+def test_header_declares_the_five_entry_points():
+    syms = declared_symbols()
+    for name in ("fp8q_quant_act_1x128", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
+                 "fp8q_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(fp8q):
+    lib = ctypes.CDLL(fp8q.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(fp8q.EXPORTS) == set(declared_symbols())
+
+
+def test_version_and_status_strings(fp8q):
+    assert fp8q.fp8q_version() >= 100
+    for code in range(6):
+        assert fp8q.fp8q_status_string(code)
+    assert fp8q.fp8q_status_string(99) == "unknown status"
+
+
+def test_quant_act_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+    assert L.fp8q_quant_act_1x128(FAKE, 4, 100, 100, FAKE, 112, FAKE, 4, None) == INV    # K % 128
+    assert L.fp8q_quant_act_1x128(FAKE, 4, 128, 64, FAKE, 128, FAKE, 4, None) == INV     # ldx < K
+    assert L.fp8q_quant_act_1x128(FAKE, 4, 128, 128, FAKE, 128, FAKE, 3, None) == INV    # ld_sf < M
+    assert L.fp8q_quant_act_1x128(FAKE, -1, 128, 128, FAKE, 128, FAKE, 4, None) == INV
+    assert L.fp8q_quant_act_1x128(FAKE + 8, 4, 128, 128, FAKE, 128, FAKE, 4, None) == ALN
+    assert L.fp8q_quant_act_1x128(FAKE, 4, 128, 132, FAKE, 128, FAKE, 4, None) == ALN    # ldx % 8
+    assert L.fp8q_quant_act_1x128(FAKE, 4, 128, 128, FAKE, 136, FAKE, 4, None) == ALN    # ldq % 16
+    assert L.fp8q_quant_act_1x128(None, 4, 128, 128, FAKE, 128, FAKE, 4, None) == INV
+    assert L.fp8q_quant_act_1x128(None, 0, 128, 128, None, 128, None, 0, None) == 0     # empty: nothing launched
+    assert L.fp8q_quant_act_128x1(FAKE, 100, 8, 8, FAKE, 128, FAKE, 8, None) == INV      # T % 128
+    assert L.fp8q_quant_act_128x1(FAKE, 128, 12, 16, FAKE, 128, FAKE, 12, None) == INV   # C % 8
+    assert L.fp8q_quant_act_128x1(FAKE, 128, 8, 8, FAKE, 120, FAKE, 8, None) == INV      # ldqt < T
+    assert L.fp8q_quant_act_128x1(FAKE, 128, 8, 8, FAKE + 4, 128, FAKE, 8, None) == ALN
+    assert L.fp8q_quant_act_128x1(None, 0, 8, 8, None, 0, None, 8, None) == 0
+
+
+def test_quant_w_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+    assert L.fp8q_quant_w_128x128(FAKE, 100, 128, 128, FAKE, 128, FAKE, 1, None, 0, None, 0, None) == INV
+    assert L.fp8q_quant_w_128x128(FAKE, 128, 256, 256, FAKE, 256, FAKE, 1, None, 0, None, 0, None) == INV  # ld_sf
+    assert L.fp8q_quant_w_128x128(FAKE, 128, 128, 128, FAKE, 128, FAKE, 1, FAKE, 64, None, 0, None) == INV  # ldqt
+    assert L.fp8q_quant_w_128x128(FAKE, 128, 128, 128, FAKE, 128, FAKE, 1, FAKE + 1, 128, None, 0, None) == ALN
+    assert L.fp8q_quant_w_128x128(FAKE, 256, 128, 128, FAKE, 128, FAKE, 1, None, 0, FAKE, 1, None) == INV  # ld_sft
+
+
+def test_gemm_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+    BLK, ROW, BF, F32 = 0, 1, 0, 1
+
+    def g(M=8, N=256, K=256, lda=256, ldb=256, ld_sfa=8, ld_sfb=2, mode=BLK, ldd=256, dt=BF,
+          a=FAKE, b=FAKE, d=FAKE, sfa=FAKE, sfb=FAKE):
+        return L.fp8q_gemm_blockscaled(a, lda, sfa, ld_sfa, b, ldb, sfb, ld_sfb, mode, d, ldd, dt, M, N, K, None)
+
+    assert g(M=0) == INV
+    assert g(N=192) == INV and g(K=100) == INV and g(N=0) == INV and g(K=0) == INV
+    assert g(lda=128) == INV and g(ldb=128) == INV and g(ldd=128) == INV and g(ld_sfa=4) == INV
+    assert g(mode=2) == INV and g(dt=7) == INV
+    assert g(ld_sfb=1) == INV                      # block mode needs ld_sfb >= K/128
+    assert g(mode=ROW, ld_sfb=128) == INV          # row mode needs ld_sfb >= N
+    assert g(a=FAKE + 8) == ALN and g(b=FAKE + 8) == ALN and g(d=FAKE + 8) == ALN
+    assert g(lda=264) == ALN and g(ldb=264) == ALN
+    assert g(ldd=260) == ALN                       # 260 bf16 = 520 bytes, not a multiple of 16
+    assert g(mode=ROW, ld_sfb=258) == ALN          # row-mode scales are bulk-copied: ld % 4
+    assert g(sfa=FAKE + 2) == ALN
+    assert g(a=None) == INV
+
+
+def test_grouped_validation(fp8q):
+    L = fp8q.lib()
+    INV, UNS = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_UNSUPPORTED
+
+    def gg(G=4, Mt=64, N=256, K=256, lda=256, ld_sfa=64, ldd=256):
+        return L.fp8q_grouped_gemm_blockscaled(FAKE, lda, FAKE, ld_sfa, FAKE, FAKE, FAKE, G, Mt, FAKE, ldd, N, K, None)
+
+    assert gg(G=0) == INV and gg(Mt=-1) == INV and gg(N=200) == INV and gg(K=64) == INV
+    assert gg(G=4096) == UNS
+    assert gg(ld_sfa=32) == INV and gg(lda=128) == INV and gg(ldd=128) == INV
+    assert gg(Mt=0, ld_sfa=0) == 0                # no rows: nothing launched
+
+
+def test_debug_entry_validation(fp8q):
+    L = fp8q.lib()
+    INV = fp8q.FP8Q_ERR_INVALID_ARG
+    assert L.fp8q_debug_cast_e4m3_bits(0, -1, FAKE, None) == INV
+    assert L.fp8q_debug_cast_e4m3_bits(0, (1 << 32) + 1, FAKE, None) == INV
+    assert L.fp8q_debug_cast_e4m3_bits(0, 0, None, None) == 0
+    assert L.fp8q_debug_wait_timeout(0, None) == INV
+    assert L.fp8q_debug_wait_timeout((1 << 34) + 1, None) == INV

@@ -188,3 +188,18 @@ def ragged_offsets(counts) -> np.ndarray:
     off = np.zeros(counts.size + 1, np.int64)
     off[1:] = np.cumsum(counts)
     return off
+
+
+def expert_weights_device(G: int, N: int, K: int, seed: int = 0, sigma: float = 0.02,
+                          tid: int = TID_EXPERT_UP, device="cuda"):
+    """BF16 [G][N][K] ~N(0, sigma^2) drawn on the device with torch's seeded
+    generator (one generator per (seed, tid), experts drawn in order), for
+    sizes too large to draw on the host.  A test that needs some experts on the
+    host copies those bytes back."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed((seed << 20) + tid)
+    out = torch.empty((G, N, K), dtype=torch.bfloat16, device=device)
+    for g in range(G):
+        out[g] = (torch.randn((N, K), generator=gen, device=device, dtype=torch.float32) * sigma).to(torch.bfloat16)
+    return out
