@@ -1,0 +1,616 @@
+"""Benchmark: one training step of the fine-grained FP8 hot path on B200.
+
+A step is one pass of every hot-path operation over one batch of synthetic,
+seeded, outlier-injected input:
+  dense linear layer, 8192 tokens x 7168 -> 18432 (forward and backward):
+    quant_w_128x128(W, with W^T)           weights re-quantized once per step
+    quant_act_1x128(X)  -> Fprop  Y  = X W^T          (BF16 out)
+    quant_act_1x128(dY) -> Dgrad  dX = dY W           (BF16 out)
+    quant_act_128x1(dY), quant_act_128x1(X) -> Wgrad dW = dY^T X   (FP32 out)
+  MoE layer, 4096 tokens, top-8 of 256 experts (Zipf 1.1), hidden 7168, expert 2048:
+    quant_act_1x128(X packed) -> grouped up-projection (BF16 out)
+    quant_act_1x128(H)        -> grouped down-projection (BF16 out)
+Expert weights are resident FP8 (quantized once at set-up); the dense weight is
+re-quantized inside every step.
+
+value = GEMM FLOPs of the step / step time (TFLOP/s, whole job over all ranks).
+With --gpus N (torchrun), every rank runs the same step on its own seeded batch
+(weak scaling, no data-path collective); time = max over ranks.
+
+--impl reference times the CPU oracle (the plain C++ statement of the method)
+on a bounded sample of the same step; it is the deliberately slow baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOP/s & % FP8 peak; quantizer GB/s & % HBM BW (1 B200)"
+UNIT = "TFLOP/s"
+
+# dense layer and MoE shapes
+TOK, HID, OUT = 8192, 7168, 18432
+MOE_TOK, MOE_E, MOE_K, MOE_FF = 4096, 256, 8, 2048
+
+# fallbacks when MEASURED_PEAKS.json is absent (earlier measurement on this machine)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0          # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
+
+
+def gemm_flops():
+    f = {
+        "fprop": 2.0 * TOK * OUT * HID,
+        "dgrad": 2.0 * TOK * HID * OUT,
+        "wgrad": 2.0 * OUT * HID * TOK,
+        "moe_up": 2.0 * MOE_TOK * MOE_K * MOE_FF * HID,
+        "moe_down": 2.0 * MOE_TOK * MOE_K * HID * MOE_FF,
+    }
+    return f
+
+
+def quant_bytes():
+    """Algorithmic bytes of each quantizer launch: read BF16 + write E4M3 + write FP32 scales."""
+    def act(m, k):
+        return m * k * 2 + m * k + (m * k // 128) * 4
+    return {
+        "quant_w": OUT * HID * 2 + 2 * OUT * HID + 2 * (OUT // 128) * (HID // 128) * 4,
+        "quant_x": act(TOK, HID),
+        "quant_dy": act(TOK, OUT),
+        "quant_dy_t": act(TOK, OUT),
+        "quant_x_t": act(TOK, HID),
+        "quant_moe_x": act(MOE_TOK * MOE_K, HID),
+        "quant_moe_h": act(MOE_TOK * MOE_K, MOE_FF),
+    }
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), src="measured")
+    except Exception:
+        return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sus=1400.0, src="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fine_grained_fp8_x128_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (profiles/dram_traffic.txt: `key bytes srchash`)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = kernel_source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel_key and parts[2] == cur:
+            return float(parts[1])
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[int(str(device).split(":")[1])])
+        else:
+            dist.barrier()
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): seed = rank."""
+    return int(rank)
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+class CpuSample:
+    """A bounded sample of the step for the oracle: R full output rows of every
+    GEMM of the step, with every quantization those rows need (the dense weight
+    and W^T in full, X^T in full for Wgrad, the owning experts' weights)."""
+
+    def __init__(self, rows: int, seed: int):
+        self.R = rows
+        self.seed = seed
+        self.x_rows = W.activations_with_outliers(rows, HID, seed=seed + 100)
+        self.w = W.weights(OUT, HID, seed=seed)
+        self.wt = np.ascontiguousarray(self.w.T)
+        self.dy_rows = W.grad_with_outlier_tokens(rows, OUT, seed=seed + 100)
+        self.x_full = W.activations_with_outliers(TOK, HID, seed=seed)
+        self.dy_cols = W.grad_with_outlier_tokens(TOK, 128, seed=seed + 200)[:, :rows].copy() \
+            if rows <= 128 else W.grad_with_outlier_tokens(TOK, rows, seed=seed + 200)
+        route = W.moe_routing(seed=seed)
+        pick = np.random.default_rng(seed).choice(int(route.offsets[-1]), size=rows, replace=False)
+        exp_of_row = np.searchsorted(route.offsets, pick, side="right") - 1
+        self.experts = np.unique(exp_of_row)
+        self.moe_x = W.activations_with_outliers(rows, HID, seed=seed + 300)
+        self.moe_h = W.normal_bf16(rows, MOE_FF, 1.0, seed=seed, tid=W.TID_H)
+        self.exp_local = np.searchsorted(self.experts, exp_of_row)
+        self.w_up = W.expert_weights(len(self.experts), MOE_FF, HID, seed=seed, tid=W.TID_EXPERT_UP,
+                                     experts=self.experts)
+        self.w_dn = W.expert_weights(len(self.experts), HID, MOE_FF, seed=seed, tid=W.TID_EXPERT_DN,
+                                     experts=self.experts)
+        # rows sorted by expert so each expert owns a contiguous range
+        order = np.argsort(self.exp_local, kind="stable")
+        self.moe_x, self.moe_h, self.exp_local = self.moe_x[order], self.moe_h[order], self.exp_local[order]
+        self.moe_off = W.ragged_offsets(np.bincount(self.exp_local, minlength=len(self.experts)))
+
+    def flops(self):
+        R = self.R
+        return 2.0 * R * (OUT * HID + HID * OUT + HID * TOK + MOE_FF * HID + HID * MOE_FF)
+
+    def description(self):
+        return (f"{self.R} full output rows of each of the 5 GEMMs of the step (Fprop, Dgrad, Wgrad, MoE up, "
+                f"MoE down) with the quantizations they need (W and W^T 18432x7168 in full, X^T 8192x7168 in "
+                f"full for Wgrad, {len(self.experts)} experts' up/down weights)")
+
+    def run(self):
+        import oracle
+        R = self.R
+        qx, sx = oracle.quant_act_1x128(self.x_rows)
+        qw, sw = oracle.quant_w_128x128(self.w)
+        oracle.gemm_sampled(qx, sx, qw, sw, oracle.SFB_BLOCK128)
+        qdy, sdy = oracle.quant_act_1x128(self.dy_rows)
+        qwt, swt = oracle.quant_w_128x128(self.wt)
+        oracle.gemm_sampled(qdy, sdy, qwt, swt, oracle.SFB_BLOCK128)
+        qdyt, sdyt = oracle.quant_act_128x1(self.dy_cols)
+        qxt, sxt = oracle.quant_act_128x1(self.x_full)
+        oracle.gemm_sampled(qdyt, np.ascontiguousarray(sdyt.T), qxt, np.ascontiguousarray(sxt.T), oracle.SFB_ROW)
+        qa, sa = oracle.quant_act_1x128(self.moe_x)
+        G = len(self.experts)
+        wq = np.empty((G, MOE_FF, HID), np.uint8); ws = np.empty((G, MOE_FF // 128, HID // 128), np.float32)
+        for g in range(G):
+            wq[g], ws[g] = oracle.quant_w_128x128(self.w_up[g])
+        oracle.grouped_gemm_sampled(qa, sa, wq, ws, self.moe_off)
+        qh, sh = oracle.quant_act_1x128(self.moe_h)
+        wq = np.empty((G, HID, MOE_FF), np.uint8); ws = np.empty((G, HID // 128, MOE_FF // 128), np.float32)
+        for g in range(G):
+            wq[g], ws[g] = oracle.quant_w_128x128(self.w_dn[g])
+        oracle.grouped_gemm_sampled(qh, sh, wq, ws, self.moe_off)
+        return R
+
+
+def time_cpu_sample(sample: CpuSample):
+    import oracle
+    oracle.reset_threads_used()
+    t0 = time.perf_counter()
+    sample.run()
+    dt = time.perf_counter() - t0
+    return {"value": sample.flops() / dt / 1e12, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+            "sample": sample.description(), "seconds": dt, "host_threads": oracle.host_threads()}
+
+
+# ----------------------------------------------------------------------------- the device step
+class DeviceStep:
+    """All buffers of one step, resident on the device; step() launches the 12
+    kernels of the hot path on the current stream."""
+
+    KERNELS = ("quant_w", "quant_x", "fprop", "quant_dy", "dgrad", "quant_dy_t", "quant_x_t", "wgrad",
+               "quant_moe_x", "moe_up", "quant_moe_h", "moe_down")
+
+    def __init__(self, fp8q, seed: int, device):
+        import torch
+        self.fp8q = fp8q
+        self.dev = device
+        bf = torch.bfloat16
+        u8 = torch.uint8
+        f32 = torch.float32
+        ld = fp8q.sf_ld
+
+        def dev_bf16(bits):
+            return torch.from_numpy(bits.view(np.int16)).to(device).view(bf)
+
+        # host inputs of the step (pinned) and their device copies
+        self.h_x = torch.from_numpy(W.activations_with_outliers(TOK, HID, seed=seed).view(np.int16)).view(bf).pin_memory()
+        self.h_dy = torch.from_numpy(W.grad_with_outlier_tokens(TOK, OUT, seed=seed).view(np.int16)).view(bf).pin_memory()
+        route = W.moe_routing(tokens=MOE_TOK, experts=MOE_E, top_k=MOE_K, seed=seed)
+        self.mt = int(route.offsets[-1])
+        xt = W.activations_with_outliers(MOE_TOK, HID, seed=seed, tid=W.TID_MISC)
+        self.h_xp = torch.from_numpy(np.ascontiguousarray(xt[route.token_of_row]).view(np.int16)).view(bf).pin_memory()
+        self.h_off = torch.from_numpy(route.offsets.astype(np.int32)).pin_memory()
+        self.w = dev_bf16(W.weights(OUT, HID, seed=seed))                      # model state, resident
+        self.x = torch.empty((TOK, HID), dtype=bf, device=device)
+        self.dy = torch.empty((TOK, OUT), dtype=bf, device=device)
+        self.xp = torch.empty((self.mt, HID), dtype=bf, device=device)
+        self.off = torch.empty((MOE_E + 1,), dtype=torch.int32, device=device)
+        self.upload()
+        # quantized operands and outputs
+        self.wq = torch.empty((OUT, HID), dtype=u8, device=device)
+        self.sw = torch.empty((OUT // 128, HID // 128), dtype=f32, device=device)
+        self.wqt = torch.empty((HID, OUT), dtype=u8, device=device)
+        self.swt = torch.empty((HID // 128, OUT // 128), dtype=f32, device=device)
+        self.xq = torch.empty((TOK, HID), dtype=u8, device=device)
+        self.sx = torch.empty((HID // 128, ld(TOK)), dtype=f32, device=device)
+        self.y = torch.empty((TOK, OUT), dtype=bf, device=device)
+        self.dyq = torch.empty((TOK, OUT), dtype=u8, device=device)
+        self.sdy = torch.empty((OUT // 128, ld(TOK)), dtype=f32, device=device)
+        self.dx = torch.empty((TOK, HID), dtype=bf, device=device)
+        self.dyqt = torch.empty((OUT, TOK), dtype=u8, device=device)
+        self.sdyt = torch.empty((TOK // 128, ld(OUT)), dtype=f32, device=device)
+        self.xqt = torch.empty((HID, TOK), dtype=u8, device=device)
+        self.sxt = torch.empty((TOK // 128, ld(HID)), dtype=f32, device=device)
+        self.dw = torch.empty((OUT, HID), dtype=f32, device=device)
+        # MoE: resident FP8 expert weights, quantized once here with the library
+        self.wup_q = torch.empty((MOE_E, MOE_FF, HID), dtype=u8, device=device)
+        self.wup_s = torch.empty((MOE_E, MOE_FF // 128, HID // 128), dtype=f32, device=device)
+        self.wdn_q = torch.empty((MOE_E, HID, MOE_FF), dtype=u8, device=device)
+        self.wdn_s = torch.empty((MOE_E, HID // 128, MOE_FF // 128), dtype=f32, device=device)
+        for (q, s, n, k, tid) in ((self.wup_q, self.wup_s, MOE_FF, HID, W.TID_EXPERT_UP),
+                                  (self.wdn_q, self.wdn_s, HID, MOE_FF, W.TID_EXPERT_DN)):
+            wb = W.expert_weights_device(MOE_E, n, k, seed=seed, tid=tid, device=device)
+            for g in range(MOE_E):
+                fp8q.fp8q_quant_w_128x128(wb[g], q[g], s[g])
+            del wb
+        self.xpq = torch.empty((self.mt, HID), dtype=u8, device=device)
+        self.sxp = torch.empty((HID // 128, ld(self.mt)), dtype=f32, device=device)
+        self.h = torch.empty((self.mt, MOE_FF), dtype=bf, device=device)
+        self.hq = torch.empty((self.mt, MOE_FF), dtype=u8, device=device)
+        self.sh = torch.empty((MOE_FF // 128, ld(self.mt)), dtype=f32, device=device)
+        self.out = torch.empty((self.mt, HID), dtype=bf, device=device)
+        # pinned host outputs for the end-to-end leg
+        self.h_y = torch.empty_like(self.y, device="cpu").pin_memory()
+        self.h_dx = torch.empty_like(self.dx, device="cpu").pin_memory()
+        self.h_dw = torch.empty_like(self.dw, device="cpu").pin_memory()
+        self.h_out = torch.empty_like(self.out, device="cpu").pin_memory()
+        torch.cuda.synchronize()
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_dy, self.h_xp, self.h_off))
+
+    def d2h_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.h_y, self.h_dx, self.h_dw, self.h_out))
+
+    def upload(self):
+        self.x.copy_(self.h_x, non_blocking=True)
+        self.dy.copy_(self.h_dy, non_blocking=True)
+        self.xp.copy_(self.h_xp, non_blocking=True)
+        self.off.copy_(self.h_off, non_blocking=True)
+
+    def download(self):
+        self.h_y.copy_(self.y, non_blocking=True)
+        self.h_dx.copy_(self.dx, non_blocking=True)
+        self.h_dw.copy_(self.dw, non_blocking=True)
+        self.h_out.copy_(self.out, non_blocking=True)
+
+    def step(self, events=None):
+        """Launch the 12 kernels; if `events` is a list, append (name, start, end) CUDA events."""
+        import torch
+        f = self.fp8q
+        ops = (
+            ("quant_w", lambda: f.fp8q_quant_w_128x128(self.w, self.wq, self.sw, self.wqt, self.swt)),
+            ("quant_x", lambda: f.fp8q_quant_act_1x128(self.x, self.xq, self.sx)),
+            ("fprop", lambda: f.fp8q_gemm_blockscaled(self.xq, self.sx, self.wq, self.sw, f.FP8Q_SFB_BLOCK128, self.y)),
+            ("quant_dy", lambda: f.fp8q_quant_act_1x128(self.dy, self.dyq, self.sdy)),
+            ("dgrad", lambda: f.fp8q_gemm_blockscaled(self.dyq, self.sdy, self.wqt, self.swt, f.FP8Q_SFB_BLOCK128,
+                                                      self.dx)),
+            ("quant_dy_t", lambda: f.fp8q_quant_act_128x1(self.dy, self.dyqt, self.sdyt)),
+            ("quant_x_t", lambda: f.fp8q_quant_act_128x1(self.x, self.xqt, self.sxt)),
+            ("wgrad", lambda: f.fp8q_gemm_blockscaled(self.dyqt, self.sdyt, self.xqt, self.sxt, f.FP8Q_SFB_ROW,
+                                                      self.dw)),
+            ("quant_moe_x", lambda: f.fp8q_quant_act_1x128(self.xp, self.xpq, self.sxp)),
+            ("moe_up", lambda: f.fp8q_grouped_gemm_blockscaled(self.xpq, self.sxp, self.wup_q, self.wup_s, self.off,
+                                                               self.h)),
+            ("quant_moe_h", lambda: f.fp8q_quant_act_1x128(self.h, self.hq, self.sh)),
+            ("moe_down", lambda: f.fp8q_grouped_gemm_blockscaled(self.hq, self.sh, self.wdn_q, self.wdn_s, self.off,
+                                                                 self.out)),
+        )
+        for name, fn in ops:
+            if events is None:
+                fn()
+            else:
+                s = torch.cuda.Event(enable_timing=True)
+                e = torch.cuda.Event(enable_timing=True)
+                s.record()
+                fn()
+                e.record()
+                events.append((name, s, e))
+        return len(ops)
+
+
+# ----------------------------------------------------------------------------- reporting
+def config_block(world):
+    return {
+        "workload": ("one training step of a 8192-token linear layer 7168->18432 (weight quant with W^T, "
+                     "Fprop, Dgrad, Wgrad with 1x128 / 128x1 / 128x128 quantization) plus a 4096-token MoE "
+                     "layer (top-8 of 256 experts, Zipf 1.1, 8 empty; grouped up 7168->2048 and down 2048->7168)"),
+        "tokens": TOK, "hidden": HID, "out_features": OUT,
+        "moe_tokens": MOE_TOK, "experts": MOE_E, "top_k": MOE_K, "expert_ffn": MOE_FF,
+        "tile": "1x128 activations, 128x1 (Wgrad), 128x128 weights; promotion every 128 of K",
+        "l2": "inputs larger than L2: every step streams > 9 GB (7.5 GB of FP8 expert weights alone)",
+        "ranks": world,
+    }
+
+
+def kernel_stats(events, K):
+    import collections
+    tot = collections.defaultdict(float)
+    cnt = collections.defaultdict(int)
+    for name, s, e in events:
+        tot[name] += s.elapsed_time(e) * 1e-3
+        cnt[name] += 1
+    return {n: (tot[n] / cnt[n], tot[n]) for n in tot}
+
+
+def build_breakdown(stats, pk, moe_w_bytes, moe_other_bytes):
+    fl = gemm_flops()
+    qb = quant_bytes()
+    fp8_peak = pk["bf16_sus"] * FP8_OVER_BF16
+    out = {}
+    for name, (avg, total) in stats.items():
+        ent = {"avg_us": round(avg * 1e6, 2), "share": None}
+        if name in qb:
+            gbs = qb[name] / avg / 1e9
+            ent.update(bytes=qb[name], gbps=round(gbs, 1), frac_hbm=round(gbs / pk["hbm"], 3))
+        if name in fl:
+            tf = fl[name] / avg / 1e12
+            ent.update(flops=fl[name], tflops=round(tf, 1), frac_fp8=round(tf / fp8_peak, 3))
+            if name.startswith("moe"):
+                b = moe_w_bytes + moe_other_bytes[name]
+                ent.update(bytes=b, gbps=round(b / avg / 1e9, 1), frac_hbm=round(b / avg / 1e9 / pk["hbm"], 3))
+        out[name] = ent
+    grand = sum(t for _, t in stats.values())
+    for name, (avg, total) in stats.items():
+        out[name]["share"] = round(total / grand, 4)
+    return out
+
+
+def roofline_for(name, stats, pk, breakdown):
+    avg, _ = stats[name]
+    ent = breakdown[name]
+    if name.startswith("moe") or name.startswith("quant"):
+        achieved = ent["bytes"] / avg / 1e9
+        peak = pk["hbm"]
+        bound, unit = "hbm", "GB/s"
+    else:
+        achieved = ent["flops"] / avg / 1e12
+        peak = pk["bf16_sus"] * FP8_OVER_BF16
+        bound, unit = "tensor", "TFLOP/s"
+    return {"kernel": name, "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": recorded_traffic(name),
+            "peak_source": (f"{pk['src']} MEASURED_PEAKS.json: HBM copy GB/s" if bound == "hbm" else
+                            f"{pk['src']} MEASURED_PEAKS.json sustained BF16 TFLOP/s x 2 (nominal FP8:BF16 ratio)")}
+
+
+def run_fp8q(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    init_dist(world, "nccl")
+    if rank == 0:
+        from fine_grained_fp8_x128_b200 import build as _b
+        _b.build()
+    barrier(world, device)
+    import fine_grained_fp8_x128_b200 as fp8q
+
+    pk = peaks()
+    st = DeviceStep(fp8q, rank_seed(rank), device)
+    flops_step = sum(gemm_flops().values())
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize()
+    code = fp8q.fp8q_device_status()
+    if code != 0:
+        raise RuntimeError(f"device status 0x{code:x} after warm-up")
+
+    # ---- device-resident timed region
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    clocks = ClockSampler(uuid)
+    clocks.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+    barrier(world, device)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    events = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    t0.record()
+    for _ in range(args.steps):
+        launches += st.step(events)
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world, device)
+    elapsed = t0.elapsed_time(t1) * 1e-3
+    t_max = max_over_ranks(elapsed, world, device)
+    value = world * flops_step * args.steps / t_max / 1e12
+    stats = kernel_stats(events, args.steps)
+
+    # ---- end-to-end: host inputs in, host outputs back, through the public API
+    barrier(world, device)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        st.upload()
+        st.step()
+        st.download()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_t = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world, device)
+    e2e_value = world * flops_step * args.steps / e2e_t / 1e12
+    code = fp8q.fp8q_device_status()
+    if code != 0:
+        raise RuntimeError(f"device status 0x{code:x} after the timed region")
+
+    nz = int((st.h_off[1:] - st.h_off[:-1] > 0).sum())
+    moe_w = nz * MOE_FF * HID + nz * (MOE_FF // 128) * (HID // 128) * 4
+    mt = st.mt
+    moe_other = {"moe_up": mt * HID + (HID // 128) * mt * 4 + mt * MOE_FF * 2,
+                 "moe_down": mt * MOE_FF + (MOE_FF // 128) * mt * 4 + mt * HID * 2}
+    breakdown = build_breakdown(stats, pk, moe_w, moe_other)
+    dominant = max(stats, key=lambda n: stats[n][1])
+    roof = roofline_for(dominant, stats, pk, breakdown)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_cpu_sample(CpuSample(args.cpu_rows, seed=0))
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_max / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
+            "config": config_block(world),
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": st.h2d_bytes(),
+                    "d2h_bytes_per_step": st.d2h_bytes()},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "breakdown": breakdown,
+            "impl": "fp8q",
+        }
+        print(json.dumps(line), flush=True)
+    del st
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    sample = CpuSample(args.ref_rows, seed=0)
+    for _ in range(args.warmup):
+        sample.run()
+    import oracle
+    oracle.reset_threads_used()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sample.run()
+    dt = time.perf_counter() - t0
+    value = sample.flops() * args.steps / dt / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(world), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+                         "sample": "each step: " + sample.description()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("fp8q", "reference"), default="fp8q")
+    ap.add_argument("--cpu-rows", type=int, default=16, help="rows per GEMM in the oracle's CPU-baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=4, help="rows per GEMM per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_fp8q(args)
+
+
+if __name__ == "__main__":
+    main()

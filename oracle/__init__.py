@@ -86,7 +86,12 @@ def _check(rc: int, what: str):
 
 
 def threads_used() -> int:
+    """Most host threads any oracle call used since reset_threads_used()."""
     return _load().orc_threads_used()
+
+
+def reset_threads_used() -> None:
+    _load().orc_reset_threads_used()
 
 
 def host_threads() -> int:

@@ -56,12 +56,13 @@ template <class F>
 void parallel_for(int64_t n, F fn) {
   int nt = host_threads();
   if (n < 2 || nt < 2) {
-    g_threads_used.store(1);
     for (int64_t i = 0; i < n; ++i) fn(i);
     return;
   }
   if (nt > n) nt = static_cast<int>(n);
-  g_threads_used.store(nt);
+  int prev = g_threads_used.load();
+  while (nt > prev && !g_threads_used.compare_exchange_weak(prev, nt)) {
+  }
   std::atomic<int64_t> next{0};
   std::vector<std::thread> pool;
   pool.reserve(nt);
@@ -230,8 +231,9 @@ extern "C" {
 
 int orc_version(void) { return 1; }
 
-// Threads used by the most recent multithreaded call (for reporting).
+// Most threads any call used since the last reset (for reporting).
 int orc_threads_used(void) { return g_threads_used.load(); }
+void orc_reset_threads_used(void) { g_threads_used.store(1); }
 int orc_host_threads(void) { return host_threads(); }
 
 // ---- codecs ---------------------------------------------------------------

@@ -44,8 +44,8 @@ def run_gemm(fp8q, qa, sfa, qb, sfb, mode, out_f32=False, lda=None, ldb=None, ld
     ldd = ldd or N
     abuf = np.zeros((M, lda), np.uint8); abuf[:, :K] = qa
     bbuf = np.zeros((N, ldb), np.uint8); bbuf[:, :K] = qb
-    a = to_dev_u8(abuf)
-    b = to_dev_u8(bbuf)
+    a = to_dev_u8(abuf)[:, :K]
+    b = to_dev_u8(bbuf)[:, :K]
     sa = sfa_dev(sfa)
     sb = to_dev_f32(sfb) if mode == BLK else sfa_dev(sfb)
     dt = torch.float32 if out_f32 else torch.bfloat16

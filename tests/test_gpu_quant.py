@@ -36,11 +36,11 @@ def run_q1(fp8q, x_bits, ldx=None, ldq=None, ld_sf=None):
     ldx = ldx or K
     ldq = ldq or K
     ld_sf = ld_sf or M
-    xd = to_dev_bf16(_padded_bf16(x_bits, ldx))
+    xd = to_dev_bf16(_padded_bf16(x_bits, ldx))[:, :K]
     # guard rows before and after every output
     qbuf = torch.full((M + 2, ldq), CANARY, dtype=torch.uint8, device="cuda")
     sfbuf = torch.full((K // 128 + 2, ld_sf), -7.0, dtype=torch.float32, device="cuda")
-    q = qbuf[1:M + 1]
+    q = qbuf[1:M + 1, :K]
     sf = sfbuf[1:K // 128 + 1]
     fp8q.fp8q_quant_act_1x128(xd, q, sf)
     torch.cuda.synchronize()
@@ -116,10 +116,10 @@ def run_qt(fp8q, x_bits, ldx=None, ldqt=None, ld_sf=None):
     ldx = ldx or C
     ldqt = ldqt or T
     ld_sf = ld_sf or C
-    xd = to_dev_bf16(_padded_bf16(x_bits, ldx))
+    xd = to_dev_bf16(_padded_bf16(x_bits, ldx))[:, :C]
     qbuf = torch.full((C + 2, ldqt), CANARY, dtype=torch.uint8, device="cuda")
     sfbuf = torch.full((T // 128 + 2, ld_sf), -7.0, dtype=torch.float32, device="cuda")
-    fp8q.fp8q_quant_act_128x1(xd, qbuf[1:C + 1], sfbuf[1:T // 128 + 1])
+    fp8q.fp8q_quant_act_128x1(xd, qbuf[1:C + 1, :T], sfbuf[1:T // 128 + 1])
     torch.cuda.synchronize()
     assert fp8q.fp8q_device_status() == 0
     qh = qbuf.cpu().numpy()
@@ -169,7 +169,7 @@ def run_qw(fp8q, w_bits, transposed=True, ldw=None):
     import torch
     N, K = w_bits.shape
     ldw = ldw or K
-    wd = to_dev_bf16(_padded_bf16(w_bits, ldw))
+    wd = to_dev_bf16(_padded_bf16(w_bits, ldw))[:, :K]
     q = torch.full((N, K), CANARY, dtype=torch.uint8, device="cuda")
     sf = torch.full((N // 128, K // 128), -7.0, dtype=torch.float32, device="cuda")
     qt = sft = None
