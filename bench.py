@@ -594,6 +594,99 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- single-kernel timing
+SINGLE_KERNELS = ("quant_x", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "moe_up", "moe_down")
+
+
+def run_single(args):
+    """Time one kernel of the step in isolation (for A/B comparisons and ncu
+    captures): --tokens scales the token dimension; weights keep their sizes."""
+    import torch
+    import fine_grained_fp8_x128_b200 as fp8q
+    dev = "cuda:0"
+    torch.cuda.set_device(0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    T = args.tokens
+
+    def randn(*shape, sigma=1.0):
+        return (torch.randn(shape, generator=gen, device=dev) * sigma).to(torch.bfloat16)
+
+    name = args.single
+    ld = fp8q.sf_ld
+    u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+    work = None
+    if name in ("quant_x", "quant_x_t"):
+        x = randn(T, HID)
+        if name == "quant_x":
+            q = torch.empty((T, HID), dtype=u8, device=dev); sf = torch.empty((HID // 128, ld(T)), dtype=f32, device=dev)
+            fn = lambda: fp8q.fp8q_quant_act_1x128(x, q, sf)
+        else:
+            q = torch.empty((HID, T), dtype=u8, device=dev); sf = torch.empty((T // 128, ld(HID)), dtype=f32, device=dev)
+            fn = lambda: fp8q.fp8q_quant_act_128x1(x, q, sf)
+        work = ("bytes", T * HID * 3 + T * HID // 128 * 4)
+    elif name == "quant_w":
+        w = randn(OUT, HID, sigma=0.02)
+        q, sf, qt, sft = fp8q.quant_w_128x128(w, transposed=True)
+        fn = lambda: fp8q.fp8q_quant_w_128x128(w, q, sf, qt, sft)
+        work = ("bytes", OUT * HID * 4 + 2 * (OUT // 128) * (HID // 128) * 4)
+    elif name in ("fprop", "dgrad", "wgrad"):
+        if name == "fprop":
+            M, N, K = T, OUT, HID
+        elif name == "dgrad":
+            M, N, K = T, HID, OUT
+        else:
+            M, N, K = OUT, HID, T
+        qa, sa = fp8q.quant_act_1x128(randn(M, K))
+        if name == "wgrad":
+            qb, sb = fp8q.quant_act_1x128(randn(N, K))
+            d = torch.empty((M, N), dtype=f32, device=dev)
+            mode = fp8q.FP8Q_SFB_ROW
+        else:
+            qb, sb = fp8q.quant_w_128x128(randn(N, K, sigma=0.02))
+            d = torch.empty((M, N), dtype=bf, device=dev)
+            mode = fp8q.FP8Q_SFB_BLOCK128
+        fn = lambda: fp8q.fp8q_gemm_blockscaled(qa, sa, qb, sb, mode, d)
+        work = ("flops", 2.0 * M * N * K)
+    elif name in ("moe_up", "moe_down"):
+        moe_tokens = MOE_TOK if T == TOK else T          # --tokens counts MoE tokens before top-k
+        route = W.moe_routing(tokens=moe_tokens, experts=MOE_E, top_k=MOE_K, seed=0)
+        mt = int(route.offsets[-1])
+        K, N = (HID, MOE_FF) if name == "moe_up" else (MOE_FF, HID)
+        qa, sa = fp8q.quant_act_1x128(randn(mt, K))
+        wq = torch.randint(0, 0x7E, (MOE_E, N, K), generator=gen, device=dev, dtype=torch.int32).to(u8)
+        ws = torch.rand((MOE_E, N // 128, K // 128), generator=gen, device=dev) * 1e-3
+        off = torch.from_numpy(route.offsets.astype(np.int32)).to(dev)
+        d = torch.empty((mt, N), dtype=bf, device=dev)
+        fn = lambda: fp8q.fp8q_grouped_gemm_blockscaled(qa, sa, wq, ws, off, d)
+        work = ("flops", 2.0 * mt * N * K)
+    else:
+        raise SystemExit(f"unknown kernel {name}; choose from {SINGLE_KERNELS}")
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        scrub.zero_()                       # evict the inputs from L2 between launches
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(); fn(); e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e) * 1e-3)
+    code = fp8q.fp8q_device_status()
+    t = float(np.median(times))
+    out = {"kernel": name, "tokens": T, "median_us": round(t * 1e6, 2), "min_us": round(min(times) * 1e6, 2),
+           "status": code}
+    if work[0] == "bytes":
+        out["GBps"] = round(work[1] / t / 1e9, 1)
+    else:
+        out["TFLOPs"] = round(work[1] / t / 1e12, 1)
+    print(json.dumps(out), flush=True)
+    if code != 0:
+        raise SystemExit(1)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -603,10 +696,14 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=16, help="rows per GEMM in the oracle's CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=4, help="rows per GEMM per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single", choices=SINGLE_KERNELS, help="time one kernel alone (not the bench line)")
+    ap.add_argument("--tokens", type=int, default=TOK, help="token count for --single")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.single:
+        run_single(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_fp8q(args)

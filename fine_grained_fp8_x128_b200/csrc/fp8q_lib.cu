@@ -7,26 +7,46 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/fp8q.h"
 #include "device_common.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "quant.cuh"
 
 namespace {
 
 constexpr int kMaxDevices = 64;
 
+std::mutex g_mu;
+
 struct DeviceInfo {
   bool ready = false;
   int sm_count = 0;
   bool gemm_attr[2][2][2] = {};   // [grouped][row mode][f32 out]
   bool q2_attr = false;
+  bool pair_attr[2][2] = {};       // [row mode][f32 out]
+  int pair_clusters[2][2] = {};    // co-resident CTA pairs per kernel instance
+  int q1_per_sm = 0;               // resident blocks per SM of each quantizer
+  int q2_per_sm = 0;
+  int qw_per_sm = 0;
 };
 
-std::mutex g_mu;
+// Resident blocks per SM of a kernel (cached per device); at least 1.
+template <class Kern>
+int blocks_per_sm(int* cache, Kern kern, int threads, size_t smem) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (*cache == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess || n < 1) n = 1;
+    *cache = n;
+  }
+  return *cache;
+}
+
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -107,6 +127,52 @@ fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMa
   return launch_status();
 }
 
+template <int MODE, bool F32>
+fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb,
+                             const fp8q::GemmArgs& args, int64_t pair_tiles, cudaStream_t stream) {
+  const uint32_t smem = fp8q::PairSmemLayout::bytes + 1024;
+  auto kern = fp8q::gemm_pair_kernel<MODE, F32>;
+  const int mi = MODE == FP8Q_SFB_ROW ? 1 : 0, fi = F32 ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(fp8q::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!dev->pair_attr[mi][fi]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      cfg.gridDim = dim3(2 * (dev->sm_count / 2), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = dev->sm_count / 2;
+      dev->pair_clusters[mi][fi] = n;
+      dev->pair_attr[mi][fi] = true;
+    }
+  }
+  const int64_t clusters = pair_tiles < dev->pair_clusters[mi][fi] ? pair_tiles : dev->pair_clusters[mi][fi];
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return launch_status();
+}
+
+// Which dense kernel runs: CTA pairs (256-row tiles) when M >= 256, else one
+// CTA per 128-row tile.  FP8Q_DENSE_KERNEL=single|pair overrides the choice
+// (tests use it to check both kernels on the same shapes).
+bool use_pair_kernel(int64_t M) {
+  const char* e = std::getenv("FP8Q_DENSE_KERNEL");
+  if (e != nullptr && std::strcmp(e, "single") == 0) return false;
+  if (e != nullptr && std::strcmp(e, "pair") == 0) return true;
+  return M >= 256;
+}
+
 }  // namespace
 
 extern "C" {
@@ -151,7 +217,8 @@ fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ld
   if (st != FP8Q_OK) return st;
   const int64_t KB = K / 128;
   const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
-  const int64_t grid = grid_for(items, dev->sm_count, 8);
+  const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
   fp8q::quant_act_1x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf);
   return launch_status();
@@ -177,7 +244,8 @@ fp8q_status fp8q_quant_act_128x1(const void* x, int64_t T, int64_t C, int64_t ld
     }
   }
   const int64_t items = (T / 128) * ((C + fp8q::kQTCols - 1) / fp8q::kQTCols);
-  const int64_t grid = grid_for(items, dev->sm_count, 3);
+  const int per_sm = blocks_per_sm(&dev->q2_per_sm, fp8q::quant_act_128x1_kernel, fp8q::kQTThreads, fp8q::kQTSmem);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
   fp8q::quant_act_128x1_kernel<<<static_cast<unsigned>(grid), fp8q::kQTThreads, fp8q::kQTSmem,
                                  static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(x), T, C, ldx,
                                                                       static_cast<uint8_t*>(qt), ldqt, sf, ld_sf);
@@ -200,7 +268,8 @@ fp8q_status fp8q_quant_w_128x128(const void* w, int64_t N, int64_t K, int64_t ld
   fp8q_status st = device_info(&dev);
   if (st != FP8Q_OK) return st;
   const int64_t NB = N / 128, KB = K / 128;
-  const int64_t grid = grid_for(NB * KB, dev->sm_count, 8);
+  const int per_sm = blocks_per_sm(&dev->qw_per_sm, fp8q::quant_w_128x128_kernel, fp8q::kQWThreads, 0);
+  const int64_t grid = grid_for(NB * KB, dev->sm_count, per_sm);
   fp8q::quant_w_128x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQWThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(w), NB, KB, ldw, static_cast<uint8_t*>(q), ldq, sf, ld_sf,
       static_cast<uint8_t*>(qt), ldqt, sft, ld_sft);
@@ -227,9 +296,10 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   DeviceInfo* dev = nullptr;
   fp8q_status st = device_info(&dev);
   if (st != FP8Q_OK) return st;
+  const bool pair = use_pair_kernel(M);
   CUtensorMap ta, tb;
   if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
-  if ((st = make_tmap(&tb, b, K, N, ldb, fp8q::BN)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, b, K, N, ldb, pair ? fp8q::BN / 2 : fp8q::BN)) != FP8Q_OK) return st;
   fp8q::GemmArgs args{};
   args.sfa = sfa;
   args.ld_sfa = ld_sfa;
@@ -249,6 +319,14 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   if (tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pair) {
+    const int64_t pair_tiles = ((M + 2 * fp8q::BM - 1) / (2 * fp8q::BM)) * args.num_n_tiles;
+    if (sfb_mode == FP8Q_SFB_BLOCK128)
+      return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, pair_tiles, s)
+                                     : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, pair_tiles, s);
+    return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_ROW, true>(dev, ta, tb, args, pair_tiles, s)
+                                   : launch_gemm_pair<FP8Q_SFB_ROW, false>(dev, ta, tb, args, pair_tiles, s);
+  }
   if (sfb_mode == FP8Q_SFB_BLOCK128) {
     return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, grid, s)
                                    : launch_gemm<false, FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, grid, s);

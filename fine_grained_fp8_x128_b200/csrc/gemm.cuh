@@ -135,23 +135,24 @@ __device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.de
 
 namespace fp8q {
 
-// Multiply 32 chunk partials by one scale and add them to the accumulators.
-__device__ __forceinline__ void promote32(float* acc, const uint32_t (&v)[32], float scale) {
+// acc[j] += v[j] * scale for 64 columns (packed FP32 pairs).
+__device__ __forceinline__ void promote64(float* acc, const uint32_t (&v)[64], float scale) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(v[j]), scale, acc[j]);
+  for (int j = 0; j < 64; j += 2)
+    fma2(acc[j], acc[j + 1], __uint_as_float(v[j]), __uint_as_float(v[j + 1]), scale, scale);
 }
 
 // Per-column scales (FP8Q_SFB_ROW): acc[j] += v[j] * (sa * sb[j]).
-__device__ __forceinline__ void promote32_rows(float* acc, const uint32_t (&v)[32], float sa,
-                                               const float* sb) {
+__device__ __forceinline__ void promote64_rows(float* acc, const uint32_t (&v)[64], float sa, const float* sb) {
   const float4* s4 = reinterpret_cast<const float4*>(sb);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
+  for (int q = 0; q < 16; ++q) {
     const float4 s = s4[q];
-    acc[4 * q + 0] = fmaf(__uint_as_float(v[4 * q + 0]), sa * s.x, acc[4 * q + 0]);
-    acc[4 * q + 1] = fmaf(__uint_as_float(v[4 * q + 1]), sa * s.y, acc[4 * q + 1]);
-    acc[4 * q + 2] = fmaf(__uint_as_float(v[4 * q + 2]), sa * s.z, acc[4 * q + 2]);
-    acc[4 * q + 3] = fmaf(__uint_as_float(v[4 * q + 3]), sa * s.w, acc[4 * q + 3]);
+    float c0, c1, c2, c3;
+    mul2(c0, c1, s.x, s.y, sa, sa);
+    mul2(c2, c3, s.z, s.w, sa, sa);
+    fma2(acc[4 * q + 0], acc[4 * q + 1], __uint_as_float(v[4 * q + 0]), __uint_as_float(v[4 * q + 1]), c0, c1);
+    fma2(acc[4 * q + 2], acc[4 * q + 3], __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]), c2, c3);
   }
 }
 
@@ -323,17 +324,26 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
       const bool vcol = ncol0 < p.N;
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      // Scale factors of chunk kc are loaded kScalePrefetch chunks ahead (a
+      // register shift ring) so their L2 latency stays off the promotion path.
+      const float* sa_ptr = p.sfa + row;
+      const float* sb_ptr = kGrouped ? p.sfb + (static_cast<int64_t>(c.group) * nb_per_group + ncol0 / 128) * nk
+                                     : p.sfb + static_cast<int64_t>(ncol0 / 128) * p.ld_sfb;
+      auto load_sa = [&](int k) -> float {
+        return (vrow && k < nk) ? __ldg(sa_ptr + static_cast<int64_t>(k) * p.ld_sfa) : 0.0f;
+      };
+      auto load_sb = [&](int k) -> float {
+        return (kSfbMode == FP8Q_SFB_BLOCK128 && vcol && k < nk) ? __ldg(sb_ptr + k) : 0.0f;
+      };
+      float sa_q0 = load_sa(0), sa_q1 = load_sa(1), sa_q2 = load_sa(2), sa_q3 = load_sa(3);
+      float sb_q0 = load_sb(0), sb_q1 = load_sb(1), sb_q2 = load_sb(2), sb_q3 = load_sb(3);
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int b = it & 1;
         const uint32_t bph = (it >> 1) & 1;
-        const float sa = vrow ? __ldg(p.sfa + static_cast<int64_t>(kc) * p.ld_sfa + row) : 0.0f;
-        float sbk = 0.0f;
-        if (kSfbMode == FP8Q_SFB_BLOCK128 && vcol) {
-          if (kGrouped)
-            sbk = __ldg(p.sfb + (static_cast<int64_t>(c.group) * nb_per_group + ncol0 / 128) * nk + kc);
-          else
-            sbk = __ldg(p.sfb + static_cast<int64_t>(ncol0 / 128) * p.ld_sfb + kc);
-        }
+        const float sa = sa_q0;
+        const float sbk = sb_q0;
+        sa_q0 = sa_q1; sa_q1 = sa_q2; sa_q2 = sa_q3; sa_q3 = load_sa(kc + 4);
+        sb_q0 = sb_q1; sb_q1 = sb_q2; sb_q2 = sb_q3; sb_q3 = load_sb(kc + 4);
         if (!warp_wait(&tfull[b], bph, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
         const float* sbv = nullptr;
         int r = 0;
@@ -345,23 +355,18 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         tc_fence_after();
         const float scale = sa * sbk;
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
-        uint32_t v0[32], v1[32];
-        tmem_ld_32x32b_x32(taddr, v0);
-        tmem_ld_wait_tied(v0);
-        tmem_ld_32x32b_x32(taddr + 32, v1);
-        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc, v0, sa, sbv); else promote32(acc, v0, scale);
-        tmem_ld_wait_tied(v1);
-        tmem_ld_32x32b_x32(taddr + 64, v0);
-        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc + 32, v1, sa, sbv + 32); else promote32(acc + 32, v1, scale);
-        tmem_ld_wait_tied(v0);
-        tmem_ld_32x32b_x32(taddr + 96, v1);
-        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc + 64, v0, sa, sbv + 64); else promote32(acc + 64, v0, scale);
-        tmem_ld_wait_tied(v1);
-        // every TMEM read of this buffer has completed: hand it back to the MMA warp
+        // two 64-column TMEM reads; the buffer goes back to the MMA warp as soon
+        // as the second read has landed, before its FMAs
+        uint32_t v[64];
+        tmem_ld_32x32b_x64(taddr, v);
+        tmem_ld_wait_tied64(v);
+        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc, v, sa, sbv); else promote64(acc, v, scale);
+        tmem_ld_32x32b_x64(taddr + 64, v);
+        tmem_ld_wait_tied64(v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[b]);
-        if (kSfbMode == FP8Q_SFB_ROW) promote32_rows(acc + 96, v1, sa, sbv + 96); else promote32(acc + 96, v1, scale);
+        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
         if (kSfbMode == FP8Q_SFB_ROW) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&sbempty[r]);

@@ -1,0 +1,261 @@
+// Dense block-scaled FP8 GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same arithmetic as gemm.cuh -- D[m,n] = sum_kb sa[m,kb] * sb(n,kb) * P_kb[m,n]
+// with a TMEM accumulator per 128-wide K chunk and FP32 promotion on the CUDA
+// cores ("FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 3;
+// "Introduction to LLM Quantization", "Fine-grained Quantization" Steps 1-4) --
+// but a cluster of two CTAs on two SMs computes one 256 x 256 output tile:
+//   * each CTA loads its own 128 rows of A and its own 128-row half of B
+//     (32 KB per K chunk instead of the 48 KB a lone 128 x 256 CTA needs) with
+//     cta_group::2 TMA loads whose completion is counted on the leader CTA's
+//     barrier -- no multicast loads;
+//   * the leader CTA issues tcgen05.mma.cta_group::2 (M = 256, N = 256), which
+//     reads both CTAs' shared memory and writes each CTA's 128 x 256 FP32 chunk
+//     result into that CTA's TMEM;
+//   * each CTA promotes and stores its own 128 rows, exactly as the single-CTA
+//     kernel does, and hands TMEM buffers back to the leader's MMA warp with a
+//     cluster-scope arrive.
+// Warp roles, TMEM double buffering, scale prefetch and the bounded waits are
+// those of gemm.cuh.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace fp8q {
+
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
+constexpr uint32_t kPairBBytes = 128 * BK;                    // 16 KB (half of the 256-row B tile)
+constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
+constexpr int kPairGroupM = 8;                                // L2 swizzle: 256-row tiles per group
+
+struct PairSmemLayout {
+  static constexpr uint32_t stages = 0;
+  static constexpr uint32_t sb_ring = stages + kPairStages * kPairStageBytes;
+  static constexpr uint32_t bars = sb_ring + kSbRing * kSbBytes;
+  // full[S], empty[S], tfull[2], tempty[2], sbfull[R], sbempty[R]
+  static constexpr uint32_t nbars = 2 * kPairStages + 4 + 2 * kSbRing;
+  static constexpr uint32_t misc = bars + nbars * 8;
+  static constexpr uint32_t bytes = misc + 16;
+};
+
+template <int kSfbMode, bool kOutF32>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const GemmArgs p) {
+  extern __shared__ uint8_t pair_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pair_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PairSmemLayout::bars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kPairStages;
+  uint64_t* tfull = bars + 2 * kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* sbfull = tempty + 2;
+  uint64_t* sbempty = sbfull + kSbRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PairSmemLayout::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PairSmemLayout::misc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nk = p.num_k_chunks;
+  const uint32_t rank = cluster_ctarank();          // 0 = leader
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+  const int num_m_pairs = (p.M + 2 * BM - 1) / (2 * BM);
+  const int total_tiles = num_m_pairs * p.num_n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 2 * kEpiWarps); }
+    for (int r = 0; r < kSbRing; ++r) { mbar_init(&sbfull[r], 1); mbar_init(&sbempty[r], kEpiWarps); }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8 && lane == 0) { prefetch_tmap(&tmap_a); prefetch_tmap(&tmap_b); }
+  if (warp == 9) { tmem_alloc_pair(tmem_slot, 512); tmem_relinquish_pair(); }
+  tc_fence_before();
+  cluster_sync_all();          // both CTAs' barriers exist before any remote signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // pair tile t -> first row of this CTA's half and first column
+  auto tile_rows = [&](int t, int& a_row0, int& n0) {
+    const int per_group = kPairGroupM * p.num_n_tiles;
+    const int grp = t / per_group;
+    const int first_m = grp * kPairGroupM;
+    const int gm = min(kPairGroupM, num_m_pairs - first_m);
+    const int within = t - grp * per_group;
+    const int mt = first_m + within % gm;
+    const int nt = within / gm;
+    a_row0 = mt * 2 * BM + static_cast<int>(rank) * BM;
+    n0 = nt * BN;
+  };
+
+  if (warp >= kEpiWarps) {
+    setmaxnreg_dec40();
+    if (warp == 8) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
+      int it = 0;
+      bool ok = true;
+      for (int t = cluster; ok && t < total_tiles; t += nclusters) {
+        int a_row0, n0;
+        tile_rows(t, a_row0, n0);
+        const int b_row0 = n0 + static_cast<int>(rank) * (BN / 2);
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % kPairStages;
+          const uint32_t ph = (it / kPairStages) & 1;
+          if (!warp_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+          if (kSfbMode == FP8Q_SFB_ROW) {
+            const int r = it % kSbRing;
+            if (!warp_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+            if (lane == 0) {
+              const uint32_t nbytes = static_cast<uint32_t>(min(BN, p.N - n0)) * 4u;
+              mbar_arrive_expect_tx(&sbfull[r], nbytes);
+              bulk_load(smem + PairSmemLayout::sb_ring + r * kSbBytes,
+                        p.sfb + static_cast<int64_t>(kc) * p.ld_sfb + n0, nbytes, &sbfull[r]);
+            }
+          }
+          if (lane == 0) {
+            uint8_t* st = smem + PairSmemLayout::stages + s * kPairStageBytes;
+            const uint32_t leader_full = leader_full0 + static_cast<uint32_t>(s) * 8u;
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);   // both CTAs' bytes
+            tma_load_2d_pair(st, &tmap_a, leader_full, kc * BK, a_row0);
+            tma_load_2d_pair(st + kPairABytes, &tmap_b, leader_full, kc * BK, b_row0);
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int j = max(0, it - kPairStages); j < it; ++j)
+          warp_wait(&full[j % kPairStages], (j / kPairStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+      }
+    } else if (warp == 9 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA only) ----------------
+      const uint32_t idesc = umma_idesc_e4m3_f32(2 * BM, BN);
+      int it = 0;
+      bool ok = true;
+      for (int t = cluster; ok && t < total_tiles; t += nclusters) {
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % kPairStages;
+          const uint32_t ph = (it / kPairStages) & 1;
+          const int b = it & 1;
+          const uint32_t bph = (it >> 1) & 1;
+          if (!warp_wait(&tempty[b], bph ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY)) { ok = false; break; }
+          if (!warp_wait(&full[s], ph, abort_flag, WAIT_MMA_FULL)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(smem + PairSmemLayout::stages + s * kPairStageBytes);
+            const uint32_t b_addr = a_addr + kPairABytes;
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k)
+              umma_f8f6f4_pair(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
+                               k > 0 ? 1u : 0u);
+            umma_commit_pair(&empty[s], 0x3);
+            umma_commit_pair(&tfull[b], 0x3);
+          }
+          __syncwarp();
+        }
+      }
+      if (!ok && it > 0) {
+        const int j = it - 1;
+        warp_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+      }
+    }
+  } else {
+    // ---------------- promotion + epilogue (warps 0-7, both CTAs) ----------------
+    setmaxnreg_inc232();
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int r_in_tile = quad * 32 + lane;
+    const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    float acc[128];
+    int it = 0;
+    bool ok = true;
+    for (int t = cluster; ok && t < total_tiles; t += nclusters) {
+      int a_row0, n0;
+      tile_rows(t, a_row0, n0);
+      const int row = a_row0 + r_in_tile;
+      const bool vrow = row < p.M;
+      const int ncol0 = n0 + half * 128;
+      const bool vcol = ncol0 < p.N;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      const float* sa_ptr = p.sfa + row;
+      const float* sb_ptr = p.sfb + static_cast<int64_t>(ncol0 / 128) * p.ld_sfb;
+      auto load_sa = [&](int k) -> float {
+        return (vrow && k < nk) ? __ldg(sa_ptr + static_cast<int64_t>(k) * p.ld_sfa) : 0.0f;
+      };
+      auto load_sb = [&](int k) -> float {
+        return (kSfbMode == FP8Q_SFB_BLOCK128 && vcol && k < nk) ? __ldg(sb_ptr + k) : 0.0f;
+      };
+      float sa_q0 = load_sa(0), sa_q1 = load_sa(1), sa_q2 = load_sa(2), sa_q3 = load_sa(3);
+      float sb_q0 = load_sb(0), sb_q1 = load_sb(1), sb_q2 = load_sb(2), sb_q3 = load_sb(3);
+      for (int kc = 0; kc < nk; ++kc, ++it) {
+        const int b = it & 1;
+        const uint32_t bph = (it >> 1) & 1;
+        const float sa = sa_q0;
+        const float sbk = sb_q0;
+        sa_q0 = sa_q1; sa_q1 = sa_q2; sa_q2 = sa_q3; sa_q3 = load_sa(kc + 4);
+        sb_q0 = sb_q1; sb_q1 = sb_q2; sb_q2 = sb_q3; sb_q3 = load_sb(kc + 4);
+        if (!warp_wait(&tfull[b], bph, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
+        const float* sbv = nullptr;
+        int r = 0;
+        if (kSfbMode == FP8Q_SFB_ROW) {
+          r = it % kSbRing;
+          if (!warp_wait(&sbfull[r], (it / kSbRing) & 1, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
+          sbv = reinterpret_cast<const float*>(smem + PairSmemLayout::sb_ring + r * kSbBytes) + half * 128;
+        }
+        tc_fence_after();
+        const float scale = sa * sbk;
+        const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
+        uint32_t v[64];
+        tmem_ld_32x32b_x64(taddr, v);
+        tmem_ld_wait_tied64(v);
+        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc, v, sa, sbv); else promote64(acc, v, scale);
+        tmem_ld_32x32b_x64(taddr + 64, v);
+        tmem_ld_wait_tied64(v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(b) * 8u);
+        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
+        if (kSfbMode == FP8Q_SFB_ROW) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sbempty[r]);
+        }
+      }
+      if (!ok) break;
+      if (vrow && vcol) {
+        if (kOutF32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * i + 2 * j], acc[8 * i + 2 * j + 1]);
+              w[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();          // the peer's shared memory and TMEM are no longer in use
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+}  // namespace fp8q

@@ -25,131 +25,193 @@ __device__ __forceinline__ uint32_t quant_word(uint32_t w, float r, float s) {
 }
 
 // ---------------------------------------------------------------------------
-// 1x128 tiles.  8 consecutive lanes own one tile (16 elements each, two
-// 16-byte loads).  A 256-thread block covers 32 tiles: rows r0..r0+31 of one
-// 128-column chunk kb, so the 32 scales it writes, sf[kb*ld_sf + r0 ..], are
-// one contiguous 128-byte line.
+// 1x128 tiles.  4 consecutive lanes own one tile (32 elements each, four
+// 16-byte loads).  Lane `sub` reads bytes 16*sub + 64*i (i = 0..3) of the
+// tile's 256, so each load instruction covers whole 32-byte sectors; its codes
+// leave as four 8-byte stores at the matching offsets.  A 256-thread block
+// covers 64 tiles: rows r0..r0+63 of one 128-column chunk kb, so the 64 scales
+// it writes, sf[kb*ld_sf + r0 ..], are contiguous.  The loads of the block's
+// next grid-stride item are issued before the current item is cast.
 // ---------------------------------------------------------------------------
 constexpr int kQ1Threads = 256;
-constexpr int kQ1Rows = 32;
+constexpr int kQ1Rows = 64;
+
+struct Q1Slice {
+  uint4 v[4];
+};
+
+__device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB,
+                                        int64_t ldx, int64_t it, int tile, int sub) {
+  const int64_t rb = it / KB;
+  const int64_t kb = it - rb * KB;
+  const int64_t row = rb * kQ1Rows + tile;
+  if (row < M) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + row * ldx + kb * 128 + sub * 8);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d.v[i] = __ldcs(src + 4 * i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d.v[i] = make_uint4(0, 0, 0, 0);
+  }
+}
 
 __global__ void __launch_bounds__(kQ1Threads)
 quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
                        uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf) {
   const int tid = threadIdx.x;
-  const int sub = tid & 7;           // 16-element slice within the tile
-  const int tile = tid >> 3;         // 0..31: row within the block's 32 rows
+  const int sub = tid & 3;           // 32-element slice within the tile
+  const int tile = tid >> 2;         // 0..63: row within the block's 64 rows
   const int64_t row_blocks = (M + kQ1Rows - 1) / kQ1Rows;
   const int64_t items = row_blocks * KB;
-  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+  int64_t it = blockIdx.x;
+  if (it >= items) return;
+  Q1Slice cur, nxt;
+  q1_load(cur, x, M, KB, ldx, it, tile, sub);
+  for (; it < items; it += gridDim.x) {
+    const int64_t it_next = it + gridDim.x;
+    if (it_next < items) q1_load(nxt, x, M, KB, ldx, it_next, tile, sub);
     const int64_t rb = it / KB;
     const int64_t kb = it - rb * KB;
     const int64_t row = rb * kQ1Rows + tile;
-    const bool active = row < M;
-    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-    const int64_t col = kb * 128 + sub * 16;
-    if (active) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + row * ldx + col);
-      v0 = __ldg(src);
-      v1 = __ldg(src + 1);
-    }
     float m = 0.0f;
-    m = amax_word(m, v0.x); m = amax_word(m, v0.y); m = amax_word(m, v0.z); m = amax_word(m, v0.w);
-    m = amax_word(m, v1.x); m = amax_word(m, v1.y); m = amax_word(m, v1.z); m = amax_word(m, v1.w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m = amax_word(m, cur.v[i].x); m = amax_word(m, cur.v[i].y);
+      m = amax_word(m, cur.v[i].z); m = amax_word(m, cur.v[i].w);
+    }
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
     const float s = tile_scale(m);
     const float r = __frcp_rn(s);
-    if (active) {
-      uint4 o;
-      o.x = quant_word(v0.x, r, s) | (quant_word(v0.y, r, s) << 16);
-      o.y = quant_word(v0.z, r, s) | (quant_word(v0.w, r, s) << 16);
-      o.z = quant_word(v1.x, r, s) | (quant_word(v1.y, r, s) << 16);
-      o.w = quant_word(v1.z, r, s) | (quant_word(v1.w, r, s) << 16);
-      *reinterpret_cast<uint4*>(q + row * ldq + col) = o;
+    if (row < M) {
+      uint8_t* dst = q + row * ldq + kb * 128 + sub * 8;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint2 o;
+        o.x = quant_word(cur.v[i].x, r, s) | (quant_word(cur.v[i].y, r, s) << 16);
+        o.y = quant_word(cur.v[i].z, r, s) | (quant_word(cur.v[i].w, r, s) << 16);
+        *reinterpret_cast<uint2*>(dst + 32 * i) = o;
+      }
       if (sub == 0) sf[kb * ld_sf + row] = s;
     }
+    cur = nxt;
   }
 }
 
 // ---------------------------------------------------------------------------
-// 128x1 tiles along the token dimension, written transposed.  A block stages a
-// 128-token x 256-channel BF16 tile (64 KB) in shared memory with cp.async;
-// thread j then owns channels 2j and 2j+1: one bank-conflict-free 32-bit
-// shared load per token gives both, the amax is a register reduction, and the
-// 128 codes of each channel leave as eight 16-byte stores of the row qt[c].
+// 128x1 tiles along the token dimension, written transposed.  A 256-thread
+// block stages 128-token x 128-channel BF16 tiles (32 KB) in shared memory
+// with cp.async, double-buffered so the next tile's copy overlaps this one's
+// cast.  Thread t owns the channel pair p = t % 64 for the 32-token
+// quarter r = t / 64: a bank-conflict-free 32-bit shared load per token gives
+// both channels, the four quarters' maxima combine through shared memory, and
+// each thread writes its 32 codes per channel as two 16-byte stores (whole
+// 32-byte sectors of the rows qt[c]).
 // ---------------------------------------------------------------------------
-constexpr int kQTThreads = 128;
-constexpr int kQTCols = 256;
-constexpr int kQTSmem = 128 * kQTCols * 2;   // 65536
+constexpr int kQTThreads = 256;
+constexpr int kQTCols = 128;
+constexpr int kQTTileBytes = 128 * kQTCols * 2;                 // 32 KB staged BF16 tile
+constexpr int kQTSmem = 2 * kQTTileBytes + 4 * kQTCols * 4;     // double buffer + per-quarter maxima
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Stage item `it` (128 tokens x up to 128 channels) into `tile` with cp.async.
+__device__ __forceinline__ void qt_stage(uint32_t* tile, const __nv_bfloat16* __restrict__ x, int64_t C, int64_t ldx,
+                                         int64_t col_blocks, int64_t it, int tid) {
+  const int64_t tb = it / col_blocks;
+  const int64_t c0 = (it - tb * col_blocks) * kQTCols;
+  const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;   // multiple of 8
+  const int chunks_per_row = static_cast<int>(ncols / 8);
+  for (int i = tid; i < 128 * (kQTCols / 8); i += kQTThreads) {
+    const int rr = i / (kQTCols / 8);
+    const int cc = i % (kQTCols / 8);
+    if (cc < chunks_per_row) cp_async16(&tile[rr * (kQTCols / 2) + cc * 4], x + (tb * 128 + rr) * ldx + c0 + cc * 8);
+  }
+  cp_async_commit();
 }
 
 __global__ void __launch_bounds__(kQTThreads)
 quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C, int64_t ldx,
                        uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sf, int64_t ld_sf) {
   extern __shared__ __align__(128) uint8_t q2_smem[];
-  uint32_t* tile = reinterpret_cast<uint32_t*>(q2_smem);   // [128 tokens][128 words]
+  float* qmax = reinterpret_cast<float*>(q2_smem + 2 * kQTTileBytes);   // [4 quarters][128 channels]
   const int tid = threadIdx.x;
+  const int p = tid & 63;          // channel pair
+  const int r = tid >> 6;          // token quarter
+  constexpr int kWords = kQTCols / 2;   // 64 words per staged row
   const int64_t col_blocks = (C + kQTCols - 1) / kQTCols;
   const int64_t items = (T / 128) * col_blocks;
-  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+  int64_t it = blockIdx.x;
+  if (it >= items) return;
+  int buf = 0;
+  qt_stage(reinterpret_cast<uint32_t*>(q2_smem), x, C, ldx, col_blocks, it, tid);
+  for (; it < items; it += gridDim.x, buf ^= 1) {
+    // prefetch the next item into the other buffer while this one is cast
+    const int64_t next = it + gridDim.x;
+    if (next < items) {
+      qt_stage(reinterpret_cast<uint32_t*>(q2_smem + (buf ^ 1) * kQTTileBytes), x, C, ldx, col_blocks, next, tid);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint32_t* tile = reinterpret_cast<const uint32_t*>(q2_smem + buf * kQTTileBytes);
     const int64_t tb = it / col_blocks;
     const int64_t c0 = (it - tb * col_blocks) * kQTCols;
-    const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;   // multiple of 8
-    const int chunks_per_row = static_cast<int>(ncols / 8);          // 16-byte chunks
-    // stage: 128 rows x ncols channels
-    for (int i = tid; i < 128 * (kQTCols / 8); i += kQTThreads) {
-      const int rr = i / (kQTCols / 8);
-      const int cc = i % (kQTCols / 8);
-      if (cc < chunks_per_row)
-        cp_async16(&tile[rr * (kQTCols / 2) + cc * 4], x + (tb * 128 + rr) * ldx + c0 + cc * 8);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    const int64_t ca = c0 + 2 * tid;          // this thread's channels ca, ca + 1
-    if (ca < C) {
-      float ma = 0.0f, mb = 0.0f;
-#pragma unroll 16
-      for (int t = 0; t < 128; ++t) {
-        const uint32_t w = tile[t * (kQTCols / 2) + tid];
+    const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;
+    const bool active = 2 * p < ncols;
+    float ma = 0.0f, mb = 0.0f;
+    if (active) {
+#pragma unroll 8
+      for (int t = 32 * r; t < 32 * r + 32; ++t) {
+        const uint32_t w = tile[t * kWords + p];
         ma = fmaxf(ma, fabsf(bf16lo(w)));
         mb = fmaxf(mb, fabsf(bf16hi(w)));
       }
+    }
+    qmax[r * kQTCols + 2 * p] = ma;
+    qmax[r * kQTCols + 2 * p + 1] = mb;
+    __syncthreads();
+    if (active) {
+      ma = fmaxf(fmaxf(qmax[2 * p], qmax[kQTCols + 2 * p]), fmaxf(qmax[2 * kQTCols + 2 * p], qmax[3 * kQTCols + 2 * p]));
+      mb = fmaxf(fmaxf(qmax[2 * p + 1], qmax[kQTCols + 2 * p + 1]),
+                 fmaxf(qmax[2 * kQTCols + 2 * p + 1], qmax[3 * kQTCols + 2 * p + 1]));
       const float sa = tile_scale(ma), sb = tile_scale(mb);
       const float ra = __frcp_rn(sa), rb = __frcp_rn(sb);
-      uint8_t* qa = qt + ca * ldqt + tb * 128;
+      const int64_t ca = c0 + 2 * p;
+      uint8_t* qa = qt + ca * ldqt + tb * 128 + 32 * r;
       uint8_t* qb = qa + ldqt;
-#pragma unroll 1
-      for (int t0 = 0; t0 < 128; t0 += 16) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         uint32_t oa[4], ob[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t a4 = 0, b4 = 0;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int t = t0 + 4 * j + 2 * h;
-            const uint32_t w0 = tile[t * (kQTCols / 2) + tid];
-            const uint32_t w1 = tile[(t + 1) * (kQTCols / 2) + tid];
-            a4 |= cvt_e4m3x2(scaled_for_cast(bf16lo(w0), ra, sa), scaled_for_cast(bf16lo(w1), ra, sa)) << (16 * h);
-            b4 |= cvt_e4m3x2(scaled_for_cast(bf16hi(w0), rb, sb), scaled_for_cast(bf16hi(w1), rb, sb)) << (16 * h);
+          for (int e = 0; e < 2; ++e) {
+            const int t = 32 * r + 16 * h + 4 * j + 2 * e;
+            const uint32_t w0 = tile[t * kWords + p];
+            const uint32_t w1 = tile[(t + 1) * kWords + p];
+            a4 |= cvt_e4m3x2(scaled_for_cast(bf16lo(w0), ra, sa), scaled_for_cast(bf16lo(w1), ra, sa)) << (16 * e);
+            b4 |= cvt_e4m3x2(scaled_for_cast(bf16hi(w0), rb, sb), scaled_for_cast(bf16hi(w1), rb, sb)) << (16 * e);
           }
           oa[j] = a4;
           ob[j] = b4;
         }
-        *reinterpret_cast<uint4*>(qa + t0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        *reinterpret_cast<uint4*>(qb + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        *reinterpret_cast<uint4*>(qa + 16 * h) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *reinterpret_cast<uint4*>(qb + 16 * h) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
       }
-      sf[tb * ld_sf + ca] = sa;
-      sf[tb * ld_sf + ca + 1] = sb;
+      if (r == 0) {
+        sf[tb * ld_sf + ca] = sa;
+        sf[tb * ld_sf + ca + 1] = sb;
+      }
     }
-    __syncthreads();   // the tile buffer is reused by the next item
+    __syncthreads();   // this buffer is refilled two items later; the maxima are reused next item
   }
 }
 
@@ -176,7 +238,7 @@ __device__ __forceinline__ void transpose4x4(const uint32_t a0, const uint32_t a
   c[3] = __byte_perm(t1, t3, 0x7632);
 }
 
-__global__ void __launch_bounds__(kQWThreads)
+__global__ void __launch_bounds__(kQWThreads, 3)
 quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t KB, int64_t ldw,
                        uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
                        uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sft, int64_t ld_sft) {

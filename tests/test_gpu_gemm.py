@@ -84,15 +84,24 @@ def test_linear_y_wx_worked_example(fp8q):
     check_gemm(y.float().cpu().numpy(), ref, rounded(ref, False))
 
 
+@pytest.fixture(params=["single", "pair"])
+def dense_kernel(request, monkeypatch):
+    """Run a test on the one-CTA kernel and on the CTA-pair kernel."""
+    monkeypatch.setenv("FP8Q_DENSE_KERNEL", request.param)
+    return request.param
+
+
 @pytest.mark.parametrize("M,N,K,mode,f32", [
+    (1, 256, 128, BLK, False),       # one row (a pair tile with 255 empty rows)
     (128, 256, 128, BLK, False),     # one tile, one chunk
     (300, 384, 640, BLK, False),     # ragged M, half N tile, 5 chunks
     (300, 384, 640, BLK, True),
     (257, 512, 1024, ROW, True),     # Wgrad scale mode
     (129, 128, 384, ROW, False),
     (1000, 1280, 768, BLK, False),   # several tiles per CTA pass
+    (2048, 2560, 512, ROW, True),    # more pair tiles than co-resident pairs
 ])
-def test_gemm_parity_small(fp8q, M, N, K, mode, f32):
+def test_gemm_parity_small(fp8q, dense_kernel, M, N, K, mode, f32):
     x = W.activations_with_outliers(M, K, seed=M, channel_frac=2 / K, elem_frac=1e-3)
     qa, sa = oracle.quant_act_1x128(x)
     if mode == BLK:
@@ -104,7 +113,7 @@ def test_gemm_parity_small(fp8q, M, N, K, mode, f32):
     check_gemm(d, ref, rounded(ref, f32))
 
 
-def test_gemm_integer_exact(fp8q):
+def test_gemm_integer_exact(fp8q, dense_kernel):
     """Small-integer codes with power-of-two scales: every partial sum is exact
     in FP32, so the device result must equal the oracle exactly."""
     rng = np.random.default_rng(1)
@@ -119,7 +128,7 @@ def test_gemm_integer_exact(fp8q):
     assert np.array_equal(d, ref)
 
 
-def test_gemm_one_hot_rows(fp8q):
+def test_gemm_one_hot_rows(fp8q, dense_kernel):
     N, K = 256, 256
     qb, sb = oracle.quant_w_128x128(W.weights(N, K, seed=5))
     qa = np.zeros((3, K), np.uint8)
