@@ -17,7 +17,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfp8q.so")
+# FP8Q_LIBRARY may name another build of the same library (A/B timing).
+LIB_PATH = os.environ.get("FP8Q_LIBRARY") or os.path.join(_HERE, "libfp8q.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libfp8q.so is not built ({LIB_PATH}); run `python -m fine_grained_fp8_x128_b200.build`")

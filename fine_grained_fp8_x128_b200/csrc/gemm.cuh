@@ -39,7 +39,10 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
 constexpr int kStages = 4;
-constexpr int kSbRing = 8;
+#ifndef FP8Q_SB_RING
+#define FP8Q_SB_RING 8
+#endif
+constexpr int kSbRing = FP8Q_SB_RING;
 constexpr int kGemmThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = BM * BK;               // 16 KB
@@ -355,19 +358,21 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         tc_fence_after();
         const float scale = sa * sbk;
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
-        // two 64-column TMEM reads; the buffer goes back to the MMA warp as soon
-        // as the second read has landed, before its FMAs
+        // two 64-column TMEM reads (each waited for inside its own asm statement);
+        // the buffer goes back to the MMA warp as soon as the second read has
+        // landed, before its FMAs
         uint32_t v[64];
-        tmem_ld_32x32b_x64(taddr, v);
-        tmem_ld_wait_tied64(v);
+        tmem_ld_32x32b_x64_sync(taddr, v);
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc, v, sa, sbv); else promote64(acc, v, scale);
-        tmem_ld_32x32b_x64(taddr + 64, v);
-        tmem_ld_wait_tied64(v);
+        tmem_ld_32x32b_x64_sync(taddr + 64, v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[b]);
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
         if (kSfbMode == FP8Q_SFB_ROW) {
+          // the ring slot was read with ordinary loads and is refilled by a bulk
+          // copy (async proxy): order the reads before the release across proxies
+          fence_proxy_async_shared();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sbempty[r]);
         }

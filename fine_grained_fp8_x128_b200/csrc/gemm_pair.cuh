@@ -23,7 +23,10 @@
 
 namespace fp8q {
 
-constexpr int kPairStages = 6;
+#ifndef FP8Q_PAIR_STAGES
+#define FP8Q_PAIR_STAGES 6
+#endif
+constexpr int kPairStages = FP8Q_PAIR_STAGES;
 constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
 constexpr uint32_t kPairBBytes = 128 * BK;                    // 16 KB (half of the 256-row B tile)
 constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
@@ -212,16 +215,17 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         const float scale = sa * sbk;
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
         uint32_t v[64];
-        tmem_ld_32x32b_x64(taddr, v);
-        tmem_ld_wait_tied64(v);
+        tmem_ld_32x32b_x64_sync(taddr, v);
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc, v, sa, sbv); else promote64(acc, v, scale);
-        tmem_ld_32x32b_x64(taddr + 64, v);
-        tmem_ld_wait_tied64(v);
+        tmem_ld_32x32b_x64_sync(taddr + 64, v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(b) * 8u);
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
         if (kSfbMode == FP8Q_SFB_ROW) {
+          // the ring slot was read with ordinary loads and is refilled by a bulk
+          // copy (async proxy): order the reads before the release across proxies
+          fence_proxy_async_shared();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sbempty[r]);
         }
