@@ -345,7 +345,7 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 // Arrive on an mbarrier that may live in the peer CTA (shared::cluster address).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // 2D tiled load into this CTA's shared memory whose completion is counted on
 // the pair leader's mbarrier (cta_group::2); no multicast.

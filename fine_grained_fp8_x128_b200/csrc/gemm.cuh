@@ -20,8 +20,8 @@
 //   warps 0-7  : promotion + epilogue.  Warp w reads TMEM lanes 32*(w%4).. (its
 //                rows) and columns 128*(w/4).. (its half of the 256-wide tile);
 //                each thread keeps 128 FP32 accumulators of one output row.
-//   warp 8     : TMA producer (one lane).
-//   warp 9     : MMA issuer (one lane); also owns the TMEM allocation.
+//   warp 8     : TMA producer (lane 0 runs the loop).
+//   warp 9     : MMA issuer (lane 0); owns the TMEM allocation.
 //   warps 10-11: idle (they complete the third warpgroup for setmaxnreg).
 // Pipelines:
 //   smem ring  : kStages x (A 128x128 + B 256x128 E4M3), full/empty mbarriers.
@@ -241,72 +241,71 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
   if (warp >= kEpiWarps) {
     setmaxnreg_dec40();
     if (warp == 8) {
-      // ---------------- TMA producer ----------------
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
-        const TileCoord c = tile_coord<kGrouped>(t, p, prefix, offs);
-        for (int kc = 0; kc < nk; ++kc, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!warp_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
-          if (kSfbMode == FP8Q_SFB_ROW) {
-            const int r = it % kSbRing;
-            if (!warp_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
-            if (lane == 0) {
+      // ---------------- TMA producer (one lane) ----------------
+      if (lane == 0) {
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+          const TileCoord c = tile_coord<kGrouped>(t, p, prefix, offs);
+          for (int kc = 0; kc < nk; ++kc, ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+            if (kSfbMode == FP8Q_SFB_ROW) {
+              const int r = it % kSbRing;
+              if (!mbar_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
               const uint32_t nbytes = static_cast<uint32_t>(min(BN, p.N - c.n0)) * 4u;
               mbar_arrive_expect_tx(&sbfull[r], nbytes);
               bulk_load(smem + GemmSmemLayout::sb_ring + r * kSbBytes,
                         p.sfb + static_cast<int64_t>(kc) * p.ld_sfb + c.n0, nbytes, &sbfull[r]);
             }
-          }
-          if (lane == 0) {
             uint8_t* st = smem + GemmSmemLayout::stages + s * kStageBytes;
             mbar_arrive_expect_tx(&full[s], kStageBytes);
             tma_load_2d_nohint(st, &tmap_a, &full[s], kc * BK, c.a_row0);
             tma_load_2d_nohint(st + kABytes, &tmap_b, &full[s], kc * BK, c.b_row0);
           }
-          __syncwarp();
+        }
+        if (!ok) {
+          // error path: let the copies already in flight land before the CTA exits
+          for (int j = max(0, it - kStages); j < it; ++j)
+            mbar_wait(&full[j % kStages], (j / kStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
         }
       }
-      if (!ok) {
-        // error path: let the copies already in flight land before the CTA exits
-        for (int j = max(0, it - kStages); j < it; ++j)
-          warp_wait(&full[j % kStages], (j / kStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
-      }
+      __syncwarp();
     } else if (warp == 9) {
-      // ---------------- MMA issuer ----------------
-      const uint32_t idesc = umma_idesc_e4m3_f32(BM, BN);
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
-        for (int kc = 0; kc < nk; ++kc, ++it) {
+      // ---------------- MMA issuer (one lane) ----------------
+      if (lane == 0) {
+        const uint32_t idesc = umma_idesc_e4m3_f32(BM, BN);
+        const int total_chunks = ((total_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                                  static_cast<int>(gridDim.x)) * nk;
+        auto ready = [&](int c) -> bool {   // buffer and stage of chunk c are available
+          return mbar_wait(&tempty[c & 1], ((c >> 1) & 1) ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY) &&
+                 mbar_wait(&full[c % kStages], (c / kStages) & 1, abort_flag, WAIT_MMA_FULL);
+        };
+        bool ok = true;
+        int it = 0;
+        for (; ok && it < total_chunks; ++it) {
           const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
           const int b = it & 1;
-          const uint32_t bph = (it >> 1) & 1;
-          if (!warp_wait(&tempty[b], bph ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY)) { ok = false; break; }
-          if (!warp_wait(&full[s], ph, abort_flag, WAIT_MMA_FULL)) { ok = false; break; }
+          if (!ready(it)) { ok = false; break; }
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_addr = smem_u32(smem + GemmSmemLayout::stages + s * kStageBytes);
-            const uint32_t b_addr = a_addr + kABytes;
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+          const uint32_t a_addr = smem_u32(smem + GemmSmemLayout::stages + s * kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
 #pragma unroll
-            for (int k = 0; k < BK / 32; ++k)
-              umma_f8f6f4(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
-                          k > 0 ? 1u : 0u);
-            umma_commit(&empty[s]);
-            umma_commit(&tfull[b]);
-          }
-          __syncwarp();
+          for (int k = 0; k < BK / 32; ++k)
+            umma_f8f6f4(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
+                        k > 0 ? 1u : 0u);
+          umma_commit(&empty[s]);
+          umma_commit(&tfull[b]);
+        }
+        if (!ok && it > 0) {
+          // error path: the last issued MMAs must finish reading shared memory
+          const int j = it - 1;
+          mbar_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
         }
       }
-      if (!ok && it > 0) {
-        // error path: the last issued MMAs must finish reading shared memory
-        const int j = it - 1;
-        warp_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
-      }
+      __syncwarp();
     }
   } else {
     // ---------------- promotion + epilogue (warps 0-7) ----------------

@@ -97,74 +97,73 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   if (warp >= kEpiWarps) {
     setmaxnreg_dec40();
     if (warp == 8) {
-      // ---------------- TMA producer (both CTAs) ----------------
-      const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
-      int it = 0;
-      bool ok = true;
-      for (int t = cluster; ok && t < total_tiles; t += nclusters) {
-        int a_row0, n0;
-        tile_rows(t, a_row0, n0);
-        const int b_row0 = n0 + static_cast<int>(rank) * (BN / 2);
-        for (int kc = 0; kc < nk; ++kc, ++it) {
-          const int s = it % kPairStages;
-          const uint32_t ph = (it / kPairStages) & 1;
-          if (!warp_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
-          if (kSfbMode == FP8Q_SFB_ROW) {
-            const int r = it % kSbRing;
-            if (!warp_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
-            if (lane == 0) {
+      // ---------------- TMA producer (both CTAs, one lane) ----------------
+      if (lane == 0) {
+        const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
+        int it = 0;
+        bool ok = true;
+        for (int t = cluster; ok && t < total_tiles; t += nclusters) {
+          int a_row0, n0;
+          tile_rows(t, a_row0, n0);
+          const int b_row0 = n0 + static_cast<int>(rank) * (BN / 2);
+          for (int kc = 0; kc < nk; ++kc, ++it) {
+            const int s = it % kPairStages;
+            const uint32_t ph = (it / kPairStages) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+            if (kSfbMode == FP8Q_SFB_ROW) {
+              const int r = it % kSbRing;
+              if (!mbar_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
               const uint32_t nbytes = static_cast<uint32_t>(min(BN, p.N - n0)) * 4u;
               mbar_arrive_expect_tx(&sbfull[r], nbytes);
               bulk_load(smem + PairSmemLayout::sb_ring + r * kSbBytes,
                         p.sfb + static_cast<int64_t>(kc) * p.ld_sfb + n0, nbytes, &sbfull[r]);
             }
-          }
-          if (lane == 0) {
             uint8_t* st = smem + PairSmemLayout::stages + s * kPairStageBytes;
             const uint32_t leader_full = leader_full0 + static_cast<uint32_t>(s) * 8u;
             if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);   // both CTAs' bytes
             tma_load_2d_pair(st, &tmap_a, leader_full, kc * BK, a_row0);
             tma_load_2d_pair(st + kPairABytes, &tmap_b, leader_full, kc * BK, b_row0);
           }
-          __syncwarp();
+        }
+        if (!ok && rank == 0) {
+          for (int j = max(0, it - kPairStages); j < it; ++j)
+            mbar_wait(&full[j % kPairStages], (j / kPairStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
         }
       }
-      if (!ok && rank == 0) {
-        for (int j = max(0, it - kPairStages); j < it; ++j)
-          warp_wait(&full[j % kPairStages], (j / kPairStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
-      }
+      __syncwarp();
     } else if (warp == 9 && rank == 0) {
-      // ---------------- MMA issuer (leader CTA only) ----------------
-      const uint32_t idesc = umma_idesc_e4m3_f32(2 * BM, BN);
-      int it = 0;
-      bool ok = true;
-      for (int t = cluster; ok && t < total_tiles; t += nclusters) {
-        for (int kc = 0; kc < nk; ++kc, ++it) {
+      // ---------------- MMA issuer (leader CTA, one lane) ----------------
+      if (lane == 0) {
+        const uint32_t idesc = umma_idesc_e4m3_f32(2 * BM, BN);
+        const int total_chunks =
+            ((total_tiles - cluster + nclusters - 1) / nclusters) * nk;
+        auto ready = [&](int c) -> bool {
+          return mbar_wait(&tempty[c & 1], ((c >> 1) & 1) ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY) &&
+                 mbar_wait(&full[c % kPairStages], (c / kPairStages) & 1, abort_flag, WAIT_MMA_FULL);
+        };
+        bool ok = true;
+        int it = 0;
+        for (; ok && it < total_chunks; ++it) {
           const int s = it % kPairStages;
-          const uint32_t ph = (it / kPairStages) & 1;
           const int b = it & 1;
-          const uint32_t bph = (it >> 1) & 1;
-          if (!warp_wait(&tempty[b], bph ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY)) { ok = false; break; }
-          if (!warp_wait(&full[s], ph, abort_flag, WAIT_MMA_FULL)) { ok = false; break; }
+          if (!ready(it)) { ok = false; break; }
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_addr = smem_u32(smem + PairSmemLayout::stages + s * kPairStageBytes);
-            const uint32_t b_addr = a_addr + kPairABytes;
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+          const uint32_t a_addr = smem_u32(smem + PairSmemLayout::stages + s * kPairStageBytes);
+          const uint32_t b_addr = a_addr + kPairABytes;
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
 #pragma unroll
-            for (int k = 0; k < BK / 32; ++k)
-              umma_f8f6f4_pair(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
-                               k > 0 ? 1u : 0u);
-            umma_commit_pair(&empty[s], 0x3);
-            umma_commit_pair(&tfull[b], 0x3);
-          }
-          __syncwarp();
+          for (int k = 0; k < BK / 32; ++k)
+            umma_f8f6f4_pair(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
+                             k > 0 ? 1u : 0u);
+          umma_commit_pair(&empty[s], 0x3);
+          umma_commit_pair(&tfull[b], 0x3);
+        }
+        if (!ok && it > 0) {
+          const int j = it - 1;
+          mbar_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
         }
       }
-      if (!ok && it > 0) {
-        const int j = it - 1;
-        warp_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
-      }
+      __syncwarp();
     }
   } else {
     // ---------------- promotion + epilogue (warps 0-7, both CTAs) ----------------
