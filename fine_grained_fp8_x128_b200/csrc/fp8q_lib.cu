@@ -111,6 +111,24 @@ fp8q_status make_tmap(CUtensorMap* map, const void* base, int64_t K, int64_t row
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// FP32 matrix [outer][ld] viewed as a 2D tensor {inner, outer}; box
+// {box_inner, 1}, no swizzle.  Used for the per-column B scales of the pair
+// kernel's FP8Q_SFB_ROW mode (rows [K/128], 256 columns per box).
+fp8q_status make_tmap_f32(CUtensorMap* map, const float* base, int64_t inner, int64_t outer, int64_t ld,
+                          uint32_t box_inner) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  fp8q_status st = encoder(&enc);
+  if (st != FP8Q_OK) return st;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4u};
+  cuuint32_t box[2] = {box_inner, 1u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 template <bool G, int MODE, bool F32>
 fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const fp8q::GemmArgs& args,
                         int grid, cudaStream_t stream) {
@@ -128,7 +146,7 @@ fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMa
 }
 
 template <int MODE, bool F32>
-fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb,
+fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsb,
                              const fp8q::GemmArgs& args, int64_t pair_tiles, cudaStream_t stream) {
   const uint32_t smem = fp8q::PairSmemLayout::bytes + 1024;
   auto kern = fp8q::gemm_pair_kernel<MODE, F32>;
@@ -159,17 +177,20 @@ fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUten
   }
   const int64_t clusters = pair_tiles < dev->pair_clusters[mi][fi] ? pair_tiles : dev->pair_clusters[mi][fi];
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
   return launch_status();
 }
 
-// Which dense kernel runs: one CTA per 128 x 256 tile by default (the faster
-// of the two on B200 as measured); FP8Q_DENSE_KERNEL=pair selects the CTA-pair
-// kernel (256 x 256 tiles), =single the default (tests check both).
+// Which dense kernel runs: the CTA-pair kernel (256 x 256 tiles) when A has
+// more than one 128-row tile (the faster of the two on B200, both in short
+// bursts and under the power cap), else the one-CTA kernel (128 x 256 tiles),
+// which wastes no tensor-core rows on a short A.  FP8Q_DENSE_KERNEL=single or
+// =pair forces one of them (the tests run both on every shape).
 bool use_pair_kernel(int64_t M) {
   const char* e = std::getenv("FP8Q_DENSE_KERNEL");
-  if (e != nullptr && std::strcmp(e, "pair") == 0) return M >= 1;
-  return false;
+  if (e != nullptr && std::strcmp(e, "single") == 0) return false;
+  if (e != nullptr && std::strcmp(e, "pair") == 0) return true;
+  return M > fp8q::BM;
 }
 
 }  // namespace
@@ -296,9 +317,14 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   fp8q_status st = device_info(&dev);
   if (st != FP8Q_OK) return st;
   const bool pair = use_pair_kernel(M);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tsb;
   if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
   if ((st = make_tmap(&tb, b, K, N, ldb, pair ? fp8q::BN / 2 : fp8q::BN)) != FP8Q_OK) return st;
+  if (pair && sfb_mode == FP8Q_SFB_ROW) {   // sb[K/128][ld_sfb], 256 columns per load
+    if ((st = make_tmap_f32(&tsb, sfb, N, K / 128, ld_sfb, fp8q::BN)) != FP8Q_OK) return st;
+  } else {
+    tsb = tb;   // not read
+  }
   fp8q::GemmArgs args{};
   args.sfa = sfa;
   args.ld_sfa = ld_sfa;
@@ -321,10 +347,10 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   if (pair) {
     const int64_t pair_tiles = ((M + 2 * fp8q::BM - 1) / (2 * fp8q::BM)) * args.num_n_tiles;
     if (sfb_mode == FP8Q_SFB_BLOCK128)
-      return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, pair_tiles, s)
-                                     : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, pair_tiles, s);
-    return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_ROW, true>(dev, ta, tb, args, pair_tiles, s)
-                                   : launch_gemm_pair<FP8Q_SFB_ROW, false>(dev, ta, tb, args, pair_tiles, s);
+      return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, tsb, args, pair_tiles, s)
+                                     : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, tsb, args, pair_tiles, s);
+    return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_ROW, true>(dev, ta, tb, tsb, args, pair_tiles, s)
+                                   : launch_gemm_pair<FP8Q_SFB_ROW, false>(dev, ta, tb, tsb, args, pair_tiles, s);
   }
   if (sfb_mode == FP8Q_SFB_BLOCK128) {
     return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, grid, s)

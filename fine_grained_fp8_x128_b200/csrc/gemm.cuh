@@ -24,10 +24,18 @@
 //   warp 9     : MMA issuer (lane 0); owns the TMEM allocation.
 //   warps 10-11: idle (they complete the third warpgroup for setmaxnreg).
 // Pipelines:
-//   smem ring  : kStages x (A 128x128 + B 256x128 E4M3), full/empty mbarriers.
+//   smem ring  : kStages x (A 128x128 + B 256x128 E4M3).
 //   TMEM       : 2 chunk accumulators of 128 lanes x 256 FP32 columns (all 512
 //                columns): the MMAs of chunk c+1 overlap the promotion of c.
 //   row scales : (FP8Q_SFB_ROW only) a ring of per-chunk B scale vectors.
+// Two mbarriers per ring stage carry all of it, so the MMA warp does one wait
+// and one commit per chunk (each extra wait or commit between two chunks' MMAs
+// leaves the tensor pipe idle for tens of cycles):
+//   go[s]   (count 1 + 8): chunk c's operands have landed in stage s = c % S
+//           (producer's expect_tx + TMA bytes) AND its TMEM buffer c % 2 is
+//           free (one arrive per epilogue warp when chunk c-2 was read out).
+//   done[s] (count 1): chunk c's MMAs have completed (one tcgen05.commit):
+//           stage s may be refilled and TMEM buffer c % 2 may be read.
 // Every wait is bounded (see mbar_wait) and reports through the status word.
 #pragma once
 
@@ -57,8 +65,8 @@ struct GemmSmemLayout {
   static constexpr uint32_t stages = 0;
   static constexpr uint32_t sb_ring = stages + kStages * kStageBytes;
   static constexpr uint32_t bars = sb_ring + kSbRing * kSbBytes;
-  // barriers: full[S], empty[S], tfull[2], tempty[2], sbfull[R], sbempty[R]
-  static constexpr uint32_t nbars = 2 * kStages + 4 + 2 * kSbRing;
+  // barriers: go[S], done[S], sbfull[R], sbempty[R]
+  static constexpr uint32_t nbars = 2 * kStages + 2 * kSbRing;
   static constexpr uint32_t misc = bars + nbars * 8;           // tmem base, abort flag
   static constexpr uint32_t prefix = misc + 16;                // grouped: tile prefix [G+1]
   static constexpr uint32_t offs = prefix + (kMaxGroups + 1) * 4;  // grouped: clamped offsets [G+1]
@@ -166,11 +174,9 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
   extern __shared__ uint8_t gemm_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmemLayout::bars);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* sbfull = tempty + 2;
+  uint64_t* go = bars;
+  uint64_t* done = bars + kStages;
+  uint64_t* sbfull = bars + 2 * kStages;
   uint64_t* sbempty = sbfull + kSbRing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + GemmSmemLayout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + GemmSmemLayout::misc + 4);
@@ -182,9 +188,10 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
   const int nk = p.num_k_chunks;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kEpiWarps); }
+    for (int s = 0; s < kStages; ++s) { mbar_init(&go[s], 1 + kEpiWarps); mbar_init(&done[s], 1); }
     for (int r = 0; r < kSbRing; ++r) { mbar_init(&sbfull[r], 1); mbar_init(&sbempty[r], kEpiWarps); }
+    // both TMEM buffers start free: the epilogue's share of go[] for chunks 0 and 1
+    for (int w = 0; w < kEpiWarps; ++w) { mbar_arrive(&go[0]); mbar_arrive(&go[1 % kStages]); }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -250,7 +257,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int s = it % kStages;
             const uint32_t ph = (it / kStages) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
+            if (!mbar_wait(&done[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
             if (kSfbMode == FP8Q_SFB_ROW) {
               const int r = it % kSbRing;
               if (!mbar_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
@@ -260,15 +267,17 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
                         p.sfb + static_cast<int64_t>(kc) * p.ld_sfb + c.n0, nbytes, &sbfull[r]);
             }
             uint8_t* st = smem + GemmSmemLayout::stages + s * kStageBytes;
-            mbar_arrive_expect_tx(&full[s], kStageBytes);
-            tma_load_2d_nohint(st, &tmap_a, &full[s], kc * BK, c.a_row0);
-            tma_load_2d_nohint(st + kABytes, &tmap_b, &full[s], kc * BK, c.b_row0);
+            mbar_arrive_expect_tx(&go[s], kStageBytes);
+            tma_load_2d_nohint(st, &tmap_a, &go[s], kc * BK, c.a_row0);
+            tma_load_2d_nohint(st + kABytes, &tmap_b, &go[s], kc * BK, c.b_row0);
           }
         }
         if (!ok) {
-          // error path: let the copies already in flight land before the CTA exits
+          // error path: let the copies already in flight land before the CTA exits.
+          // go[] also waits for epilogue arrivals that may never come, so each
+          // wait is short; the copies themselves land within microseconds.
           for (int j = max(0, it - kStages); j < it; ++j)
-            mbar_wait(&full[j % kStages], (j / kStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+            mbar_wait(&go[j % kStages], (j / kStages) & 1, nullptr, WAIT_DRAIN, 1ll << 22);
         }
       }
       __syncwarp();
@@ -278,16 +287,12 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         const uint32_t idesc = umma_idesc_e4m3_f32(BM, BN);
         const int total_chunks = ((total_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                                   static_cast<int>(gridDim.x)) * nk;
-        auto ready = [&](int c) -> bool {   // buffer and stage of chunk c are available
-          return mbar_wait(&tempty[c & 1], ((c >> 1) & 1) ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY) &&
-                 mbar_wait(&full[c % kStages], (c / kStages) & 1, abort_flag, WAIT_MMA_FULL);
-        };
         bool ok = true;
         int it = 0;
         for (; ok && it < total_chunks; ++it) {
           const int s = it % kStages;
           const int b = it & 1;
-          if (!ready(it)) { ok = false; break; }
+          if (!mbar_wait(&go[s], (it / kStages) & 1, abort_flag, WAIT_MMA_FULL)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + GemmSmemLayout::stages + s * kStageBytes);
           const uint32_t b_addr = a_addr + kABytes;
@@ -296,13 +301,12 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
           for (int k = 0; k < BK / 32; ++k)
             umma_f8f6f4(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
                         k > 0 ? 1u : 0u);
-          umma_commit(&empty[s]);
-          umma_commit(&tfull[b]);
+          umma_commit(&done[s]);
         }
         if (!ok && it > 0) {
           // error path: the last issued MMAs must finish reading shared memory
           const int j = it - 1;
-          mbar_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+          mbar_wait(&done[j % kStages], (j / kStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
         }
       }
       __syncwarp();
@@ -341,12 +345,12 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
       float sb_q0 = load_sb(0), sb_q1 = load_sb(1), sb_q2 = load_sb(2), sb_q3 = load_sb(3);
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int b = it & 1;
-        const uint32_t bph = (it >> 1) & 1;
+        const int s = it % kStages;
         const float sa = sa_q0;
         const float sbk = sb_q0;
         sa_q0 = sa_q1; sa_q1 = sa_q2; sa_q2 = sa_q3; sa_q3 = load_sa(kc + 4);
         sb_q0 = sb_q1; sb_q1 = sb_q2; sb_q2 = sb_q3; sb_q3 = load_sb(kc + 4);
-        if (!warp_wait(&tfull[b], bph, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
+        if (!warp_wait(&done[s], (it / kStages) & 1, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
         const float* sbv = nullptr;
         int r = 0;
         if (kSfbMode == FP8Q_SFB_ROW) {
@@ -366,7 +370,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         tmem_ld_32x32b_x64_sync(taddr + 64, v);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[b]);
+        if (lane == 0) mbar_arrive(&go[(it + 2) % kStages]);   // buffer b is free for chunk it + 2
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
         if (kSfbMode == FP8Q_SFB_ROW) {
           // the ring slot was read with ordinary loads and is refilled by a bulk

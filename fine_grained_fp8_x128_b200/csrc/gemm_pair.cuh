@@ -14,9 +14,19 @@
 //     result into that CTA's TMEM;
 //   * each CTA promotes and stores its own 128 rows, exactly as the single-CTA
 //     kernel does, and hands TMEM buffers back to the leader's MMA warp with a
-//     cluster-scope arrive.
-// Warp roles, TMEM double buffering, scale prefetch and the bounded waits are
-// those of gemm.cuh.
+//     remote arrive on the leader's go[] barrier.
+// Warp roles, TMEM double buffering, the go/done barrier pair per stage (one
+// wait and one commit per chunk in the MMA warp), scale prefetch and the
+// bounded waits are those of gemm.cuh.  Here go[s] lives on the leader and
+// counts the leader's expect_tx, both CTAs' TMA bytes and 16 epilogue warps;
+// done[s] is signalled in both CTAs by one multicast commit.
+// Per-column B scales (FP8Q_SFB_ROW) travel with the operands: each CTA
+// TMA-loads the 256 scales of chunk c into slot c % kPairSbSlots of a ring,
+// counted on go[], so the epilogue reads them after done(c) with no barrier of
+// their own.  The slot is refilled (chunk c + kPairSbSlots) after done(c +
+// kPairSbSlots - S), which needs every epilogue warp's release of chunk
+// c + kPairSbSlots - S - 2 >= c + 1, issued after the warp's last read of slot
+// c; a proxy fence before each release orders those reads before the refill.
 #pragma once
 
 #include "gemm.cuh"
@@ -31,13 +41,15 @@ constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
 constexpr uint32_t kPairBBytes = 128 * BK;                    // 16 KB (half of the 256-row B tile)
 constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
 constexpr int kPairGroupM = 8;                                // L2 swizzle: 256-row tiles per group
+constexpr int kPairSbSlots = 12;                              // per-column scale ring (>= S + 3)
+static_assert(kPairSbSlots >= kPairStages + 3, "a scale slot may be refilled while still being read");
 
 struct PairSmemLayout {
   static constexpr uint32_t stages = 0;
   static constexpr uint32_t sb_ring = stages + kPairStages * kPairStageBytes;
-  static constexpr uint32_t bars = sb_ring + kSbRing * kSbBytes;
-  // full[S], empty[S], tfull[2], tempty[2], sbfull[R], sbempty[R]
-  static constexpr uint32_t nbars = 2 * kPairStages + 4 + 2 * kSbRing;
+  static constexpr uint32_t bars = sb_ring + kPairSbSlots * kSbBytes;
+  // go[S], done[S]
+  static constexpr uint32_t nbars = 2 * kPairStages;
   static constexpr uint32_t misc = bars + nbars * 8;
   static constexpr uint32_t bytes = misc + 16;
 };
@@ -45,16 +57,12 @@ struct PairSmemLayout {
 template <int kSfbMode, bool kOutF32>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                 const GemmArgs p) {
+                 const __grid_constant__ CUtensorMap tmap_sb, const GemmArgs p) {
   extern __shared__ uint8_t pair_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pair_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PairSmemLayout::bars);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kPairStages;
-  uint64_t* tfull = bars + 2 * kPairStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* sbfull = tempty + 2;
-  uint64_t* sbempty = sbfull + kSbRing;
+  uint64_t* go = bars;
+  uint64_t* done = bars + kPairStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PairSmemLayout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PairSmemLayout::misc + 4);
 
@@ -68,13 +76,17 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   const int total_tiles = num_m_pairs * p.num_n_tiles;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPairStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 2 * kEpiWarps); }
-    for (int r = 0; r < kSbRing; ++r) { mbar_init(&sbfull[r], 1); mbar_init(&sbempty[r], kEpiWarps); }
+    for (int s = 0; s < kPairStages; ++s) { mbar_init(&go[s], 1 + 2 * kEpiWarps); mbar_init(&done[s], 1); }
+    // both TMEM buffers start free: the epilogues' share of go[] for chunks 0 and 1
+    for (int w = 0; w < 2 * kEpiWarps; ++w) { mbar_arrive(&go[0]); mbar_arrive(&go[1 % kPairStages]); }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 8 && lane == 0) { prefetch_tmap(&tmap_a); prefetch_tmap(&tmap_b); }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    if (kSfbMode == FP8Q_SFB_ROW) prefetch_tmap(&tmap_sb);
+  }
   if (warp == 9) { tmem_alloc_pair(tmem_slot, 512); tmem_relinquish_pair(); }
   tc_fence_before();
   cluster_sync_all();          // both CTAs' barriers exist before any remote signal
@@ -99,7 +111,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     if (warp == 8) {
       // ---------------- TMA producer (both CTAs, one lane) ----------------
       if (lane == 0) {
-        const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
+        const uint32_t leader_go0 = mapa_shared(smem_u32(&go[0]), 0);
         int it = 0;
         bool ok = true;
         for (int t = cluster; ok && t < total_tiles; t += nclusters) {
@@ -109,25 +121,22 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int s = it % kPairStages;
             const uint32_t ph = (it / kPairStages) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
-            if (kSfbMode == FP8Q_SFB_ROW) {
-              const int r = it % kSbRing;
-              if (!mbar_wait(&sbempty[r], ((it / kSbRing) & 1) ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
-              const uint32_t nbytes = static_cast<uint32_t>(min(BN, p.N - n0)) * 4u;
-              mbar_arrive_expect_tx(&sbfull[r], nbytes);
-              bulk_load(smem + PairSmemLayout::sb_ring + r * kSbBytes,
-                        p.sfb + static_cast<int64_t>(kc) * p.ld_sfb + n0, nbytes, &sbfull[r]);
-            }
+            if (!mbar_wait(&done[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
             uint8_t* st = smem + PairSmemLayout::stages + s * kPairStageBytes;
-            const uint32_t leader_full = leader_full0 + static_cast<uint32_t>(s) * 8u;
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);   // both CTAs' bytes
-            tma_load_2d_pair(st, &tmap_a, leader_full, kc * BK, a_row0);
-            tma_load_2d_pair(st + kPairABytes, &tmap_b, leader_full, kc * BK, b_row0);
+            const uint32_t leader_go = leader_go0 + static_cast<uint32_t>(s) * 8u;
+            if (rank == 0)   // both CTAs' bytes (operands, and per-column scales in FP8Q_SFB_ROW)
+              mbar_arrive_expect_tx(&go[s], 2 * (kPairStageBytes + (kSfbMode == FP8Q_SFB_ROW ? kSbBytes : 0u)));
+            tma_load_2d_pair(st, &tmap_a, leader_go, kc * BK, a_row0);
+            tma_load_2d_pair(st + kPairABytes, &tmap_b, leader_go, kc * BK, b_row0);
+            if (kSfbMode == FP8Q_SFB_ROW)   // sb[kc][n0 .. n0+255] (columns past N read as zero)
+              tma_load_2d_pair(smem + PairSmemLayout::sb_ring + (it % kPairSbSlots) * kSbBytes, &tmap_sb, leader_go,
+                               n0, kc);
           }
         }
         if (!ok && rank == 0) {
+          // short waits: go[] also counts epilogue arrivals that may never come
           for (int j = max(0, it - kPairStages); j < it; ++j)
-            mbar_wait(&full[j % kPairStages], (j / kPairStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+            mbar_wait(&go[j % kPairStages], (j / kPairStages) & 1, nullptr, WAIT_DRAIN, 1ll << 22);
         }
       }
       __syncwarp();
@@ -137,16 +146,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         const uint32_t idesc = umma_idesc_e4m3_f32(2 * BM, BN);
         const int total_chunks =
             ((total_tiles - cluster + nclusters - 1) / nclusters) * nk;
-        auto ready = [&](int c) -> bool {
-          return mbar_wait(&tempty[c & 1], ((c >> 1) & 1) ^ 1, abort_flag, WAIT_MMA_TMEM_EMPTY) &&
-                 mbar_wait(&full[c % kPairStages], (c / kPairStages) & 1, abort_flag, WAIT_MMA_FULL);
-        };
         bool ok = true;
         int it = 0;
         for (; ok && it < total_chunks; ++it) {
           const int s = it % kPairStages;
           const int b = it & 1;
-          if (!ready(it)) { ok = false; break; }
+          if (!mbar_wait(&go[s], (it / kPairStages) & 1, abort_flag, WAIT_MMA_FULL)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + PairSmemLayout::stages + s * kPairStageBytes);
           const uint32_t b_addr = a_addr + kPairABytes;
@@ -155,12 +160,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           for (int k = 0; k < BK / 32; ++k)
             umma_f8f6f4_pair(d_tmem, umma_desc_k_sw128(a_addr + 32 * k), umma_desc_k_sw128(b_addr + 32 * k), idesc,
                              k > 0 ? 1u : 0u);
-          umma_commit_pair(&empty[s], 0x3);
-          umma_commit_pair(&tfull[b], 0x3);
+          umma_commit_pair(&done[s], 0x3);
         }
         if (!ok && it > 0) {
           const int j = it - 1;
-          mbar_wait(&tfull[j & 1], (j >> 1) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
+          mbar_wait(&done[j % kPairStages], (j / kPairStages) & 1, nullptr, WAIT_DRAIN, 1ll << 26);
         }
       }
       __syncwarp();
@@ -172,7 +176,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     const int half = warp >> 2;
     const int r_in_tile = quad * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t leader_go0 = mapa_shared(smem_u32(&go[0]), 0);
     float acc[128];
     int it = 0;
     bool ok = true;
@@ -197,19 +201,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       float sb_q0 = load_sb(0), sb_q1 = load_sb(1), sb_q2 = load_sb(2), sb_q3 = load_sb(3);
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int b = it & 1;
-        const uint32_t bph = (it >> 1) & 1;
+        const int s = it % kPairStages;
         const float sa = sa_q0;
         const float sbk = sb_q0;
         sa_q0 = sa_q1; sa_q1 = sa_q2; sa_q2 = sa_q3; sa_q3 = load_sa(kc + 4);
         sb_q0 = sb_q1; sb_q1 = sb_q2; sb_q2 = sb_q3; sb_q3 = load_sb(kc + 4);
-        if (!warp_wait(&tfull[b], bph, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
+        if (!warp_wait(&done[s], (it / kPairStages) & 1, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
         const float* sbv = nullptr;
-        int r = 0;
-        if (kSfbMode == FP8Q_SFB_ROW) {
-          r = it % kSbRing;
-          if (!warp_wait(&sbfull[r], (it / kSbRing) & 1, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
-          sbv = reinterpret_cast<const float*>(smem + PairSmemLayout::sb_ring + r * kSbBytes) + half * 128;
-        }
+        if (kSfbMode == FP8Q_SFB_ROW)   // landed with the operands (go[] counted its bytes)
+          sbv = reinterpret_cast<const float*>(smem + PairSmemLayout::sb_ring + (it % kPairSbSlots) * kSbBytes) +
+                half * 128;
         tc_fence_after();
         const float scale = sa * sbk;
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
@@ -217,17 +218,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         tmem_ld_32x32b_x64_sync(taddr, v);
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc, v, sa, sbv); else promote64(acc, v, scale);
         tmem_ld_32x32b_x64_sync(taddr + 64, v);
+        // scale slots read so far (ordinary loads) are refilled by TMA (async
+        // proxy) only after releases like this one: order across proxies
+        if (kSfbMode == FP8Q_SFB_ROW) fence_proxy_async_shared();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_tempty0 + static_cast<uint32_t>(b) * 8u);
+        if (lane == 0)   // buffer b is free for chunk it + 2
+          mbar_arrive_cluster(leader_go0 + static_cast<uint32_t>((it + 2) % kPairStages) * 8u);
         if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
-        if (kSfbMode == FP8Q_SFB_ROW) {
-          // the ring slot was read with ordinary loads and is refilled by a bulk
-          // copy (async proxy): order the reads before the release across proxies
-          fence_proxy_async_shared();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sbempty[r]);
-        }
       }
       if (!ok) break;
       if (vrow && vcol) {

@@ -113,13 +113,6 @@ constexpr int kQTCols = 128;
 constexpr int kQTTileBytes = 128 * kQTCols * 2;                 // 32 KB staged BF16 tile
 constexpr int kQTSmem = 2 * kQTTileBytes + 4 * kQTCols * 4;     // double buffer + per-quarter maxima
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 // Stage item `it` (128 tokens x up to 128 channels) into `tile` with cp.async.
 __device__ __forceinline__ void qt_stage(uint32_t* tile, const __nv_bfloat16* __restrict__ x, int64_t C, int64_t ldx,
                                          int64_t col_blocks, int64_t it, int tid) {
