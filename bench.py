@@ -693,7 +693,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("fp8q", "reference"), default="fp8q")
-    ap.add_argument("--cpu-rows", type=int, default=16, help="rows per GEMM in the oracle's CPU-baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=256,
+                    help="rows per GEMM in the oracle's CPU-baseline sample (10-15 s on a 16-core host)")
     ap.add_argument("--ref-rows", type=int, default=4, help="rows per GEMM per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--single", choices=SINGLE_KERNELS, help="time one kernel alone (not the bench line)")

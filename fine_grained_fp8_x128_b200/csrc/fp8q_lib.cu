@@ -186,6 +186,19 @@ fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUten
 // bursts and under the power cap), else the one-CTA kernel (128 x 256 tiles),
 // which wastes no tensor-core rows on a short A.  FP8Q_DENSE_KERNEL=single or
 // =pair forces one of them (the tests run both on every shape).
+// L2 tile order of the pair kernel: tiles run through groups of group_m
+// 256-row tile pairs, m fastest.  Keep whichever operand fits in about 40% of
+// the 126 MB L2 resident and stream the other once: A resident -> one group
+// over all of M; B resident -> groups of one tile pair (all of N sweeps past
+// each 256 rows of A).  Otherwise groups of 8 tile pairs (2048 rows), which
+// measured fewer DRAM bytes on B200 than smaller groups sized to the L2.
+int64_t pair_group_m(int64_t m_pairs, int64_t a_bytes, int64_t b_bytes) {
+  const int64_t kResident = 48ll << 20;
+  if (a_bytes <= kResident) return m_pairs < 1 ? 1 : m_pairs;
+  if (b_bytes <= kResident) return 1;
+  return m_pairs < 8 ? m_pairs : 8;
+}
+
 bool use_pair_kernel(int64_t M) {
   const char* e = std::getenv("FP8Q_DENSE_KERNEL");
   if (e != nullptr && std::strcmp(e, "single") == 0) return false;
@@ -345,7 +358,9 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pair) {
-    const int64_t pair_tiles = ((M + 2 * fp8q::BM - 1) / (2 * fp8q::BM)) * args.num_n_tiles;
+    const int64_t m_pairs = (M + 2 * fp8q::BM - 1) / (2 * fp8q::BM);
+    const int64_t pair_tiles = m_pairs * args.num_n_tiles;
+    args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
     if (sfb_mode == FP8Q_SFB_BLOCK128)
       return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, tsb, args, pair_tiles, s)
                                      : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, tsb, args, pair_tiles, s);

@@ -89,6 +89,7 @@ struct GemmArgs {
   int num_m_tiles;       // dense only
   const int32_t* group_offsets;  // grouped only
   int G;
+  int group_m;           // pair kernel: 256-row tiles per L2 group (tiles run m-fastest within a group)
 };
 
 // Which output tile a linear tile id denotes.

@@ -40,7 +40,6 @@ constexpr int kPairStages = FP8Q_PAIR_STAGES;
 constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
 constexpr uint32_t kPairBBytes = 128 * BK;                    // 16 KB (half of the 256-row B tile)
 constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
-constexpr int kPairGroupM = 8;                                // L2 swizzle: 256-row tiles per group
 constexpr int kPairSbSlots = 12;                              // per-column scale ring (>= S + 3)
 static_assert(kPairSbSlots >= kPairStages + 3, "a scale slot may be refilled while still being read");
 
@@ -95,10 +94,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
 
   // pair tile t -> first row of this CTA's half and first column
   auto tile_rows = [&](int t, int& a_row0, int& n0) {
-    const int per_group = kPairGroupM * p.num_n_tiles;
+    const int per_group = p.group_m * p.num_n_tiles;
     const int grp = t / per_group;
-    const int first_m = grp * kPairGroupM;
-    const int gm = min(kPairGroupM, num_m_pairs - first_m);
+    const int first_m = grp * p.group_m;
+    const int gm = min(p.group_m, num_m_pairs - first_m);
     const int within = t - grp * per_group;
     const int mt = first_m + within % gm;
     const int nt = within / gm;
