@@ -112,16 +112,16 @@ fp8q_status make_tmap(CUtensorMap* map, const void* base, int64_t K, int64_t row
 }
 
 // FP32 matrix [outer][ld] viewed as a 2D tensor {inner, outer}; box
-// {box_inner, 1}, no swizzle.  Used for the per-column B scales of the pair
-// kernel's FP8Q_SFB_ROW mode (rows [K/128], 256 columns per box).
+// {box_inner, box_outer}, no swizzle.  The pair GEMM loads its scale factors
+// with these (ld must be a multiple of 4, the base 16-byte aligned).
 fp8q_status make_tmap_f32(CUtensorMap* map, const float* base, int64_t inner, int64_t outer, int64_t ld,
-                          uint32_t box_inner) {
+                          uint32_t box_inner, uint32_t box_outer) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   fp8q_status st = encoder(&enc);
   if (st != FP8Q_OK) return st;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4u};
-  cuuint32_t box[2] = {box_inner, 1u};
+  cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -146,8 +146,9 @@ fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMa
 }
 
 template <int MODE, bool F32>
-fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsb,
-                             const fp8q::GemmArgs& args, int64_t pair_tiles, cudaStream_t stream) {
+fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                             const CUtensorMap& tsb, const fp8q::GemmArgs& args, int64_t pair_tiles,
+                             cudaStream_t stream) {
   const uint32_t smem = fp8q::PairSmemLayout::bytes + 1024;
   auto kern = fp8q::gemm_pair_kernel<MODE, F32>;
   const int mi = MODE == FP8Q_SFB_ROW ? 1 : 0, fi = F32 ? 1 : 0;
@@ -177,15 +178,10 @@ fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUten
   }
   const int64_t clusters = pair_tiles < dev->pair_clusters[mi][fi] ? pair_tiles : dev->pair_clusters[mi][fi];
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
   return launch_status();
 }
 
-// Which dense kernel runs: the CTA-pair kernel (256 x 256 tiles) when A has
-// more than one 128-row tile (the faster of the two on B200, both in short
-// bursts and under the power cap), else the one-CTA kernel (128 x 256 tiles),
-// which wastes no tensor-core rows on a short A.  FP8Q_DENSE_KERNEL=single or
-// =pair forces one of them (the tests run both on every shape).
 // L2 tile order of the pair kernel: tiles run through groups of group_m
 // 256-row tile pairs, m fastest.  Keep whichever operand fits in about 40% of
 // the 126 MB L2 resident and stream the other once: A resident -> one group
@@ -199,9 +195,17 @@ int64_t pair_group_m(int64_t m_pairs, int64_t a_bytes, int64_t b_bytes) {
   return m_pairs < 8 ? m_pairs : 8;
 }
 
-bool use_pair_kernel(int64_t M) {
+// Which dense kernel runs: the CTA-pair kernel (256 x 256 tiles) when A has
+// more than one 128-row tile (the faster of the two on B200, both in short
+// bursts and under the power cap), else the one-CTA kernel (128 x 256 tiles),
+// which wastes no tensor-core rows on a short A.  The pair kernel TMA-loads
+// the scale factors, so it also needs both scale arrays 16-byte aligned with
+// leading dimensions that are multiples of 4 floats.  FP8Q_DENSE_KERNEL=single
+// or =pair forces one of them where it applies (the tests run both).
+bool use_pair_kernel(int64_t M, const float* sfa, int64_t ld_sfa, const float* sfb, int64_t ld_sfb) {
+  const bool fits = aligned(sfa, 16) && aligned(sfb, 16) && ld_sfa % 4 == 0 && ld_sfb % 4 == 0;
   const char* e = std::getenv("FP8Q_DENSE_KERNEL");
-  if (e != nullptr && std::strcmp(e, "single") == 0) return false;
+  if (!fits || (e != nullptr && std::strcmp(e, "single") == 0)) return false;
   if (e != nullptr && std::strcmp(e, "pair") == 0) return true;
   return M > fp8q::BM;
 }
@@ -329,14 +333,18 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   DeviceInfo* dev = nullptr;
   fp8q_status st = device_info(&dev);
   if (st != FP8Q_OK) return st;
-  const bool pair = use_pair_kernel(M);
-  CUtensorMap ta, tb, tsb;
+  const bool pair = use_pair_kernel(M, sfa, ld_sfa, sfb, ld_sfb);
+  CUtensorMap ta, tb, tsa, tsb;
   if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
   if ((st = make_tmap(&tb, b, K, N, ldb, pair ? fp8q::BN / 2 : fp8q::BN)) != FP8Q_OK) return st;
-  if (pair && sfb_mode == FP8Q_SFB_ROW) {   // sb[K/128][ld_sfb], 256 columns per load
-    if ((st = make_tmap_f32(&tsb, sfb, N, K / 128, ld_sfb, fp8q::BN)) != FP8Q_OK) return st;
-  } else {
-    tsb = tb;   // not read
+  if (pair) {
+    // sa[K/128][ld_sfa]: 128 row scales per load
+    if ((st = make_tmap_f32(&tsa, sfa, M, K / 128, ld_sfa, fp8q::BM, 1)) != FP8Q_OK) return st;
+    // sb: [K/128][ld_sfb] per-column scales, 256 per load; or [N/128][ld_sfb]
+    // block scales, 4 chunks x the tile's 2 column blocks per load
+    st = sfb_mode == FP8Q_SFB_ROW ? make_tmap_f32(&tsb, sfb, N, K / 128, ld_sfb, fp8q::BN, 1)
+                                  : make_tmap_f32(&tsb, sfb, K / 128, N / 128, ld_sfb, 4, 2);
+    if (st != FP8Q_OK) return st;
   }
   fp8q::GemmArgs args{};
   args.sfa = sfa;
@@ -362,10 +370,11 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
     const int64_t pair_tiles = m_pairs * args.num_n_tiles;
     args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
     if (sfb_mode == FP8Q_SFB_BLOCK128)
-      return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, tsb, args, pair_tiles, s)
-                                     : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, tsb, args, pair_tiles, s);
-    return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_ROW, true>(dev, ta, tb, tsb, args, pair_tiles, s)
-                                   : launch_gemm_pair<FP8Q_SFB_ROW, false>(dev, ta, tb, tsb, args, pair_tiles, s);
+      return d_dtype == FP8Q_OUT_F32
+                 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+                 : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, tsa, tsb, args, pair_tiles, s);
+    return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_ROW, true>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+                                   : launch_gemm_pair<FP8Q_SFB_ROW, false>(dev, ta, tb, tsa, tsb, args, pair_tiles, s);
   }
   if (sfb_mode == FP8Q_SFB_BLOCK128) {
     return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, grid, s)

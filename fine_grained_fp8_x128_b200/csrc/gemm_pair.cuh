@@ -16,17 +16,20 @@
 //     kernel does, and hands TMEM buffers back to the leader's MMA warp with a
 //     remote arrive on the leader's go[] barrier.
 // Warp roles, TMEM double buffering, the go/done barrier pair per stage (one
-// wait and one commit per chunk in the MMA warp), scale prefetch and the
-// bounded waits are those of gemm.cuh.  Here go[s] lives on the leader and
-// counts the leader's expect_tx, both CTAs' TMA bytes and 16 epilogue warps;
-// done[s] is signalled in both CTAs by one multicast commit.
-// Per-column B scales (FP8Q_SFB_ROW) travel with the operands: each CTA
-// TMA-loads the 256 scales of chunk c into slot c % kPairSbSlots of a ring,
-// counted on go[], so the epilogue reads them after done(c) with no barrier of
-// their own.  The slot is refilled (chunk c + kPairSbSlots) after done(c +
-// kPairSbSlots - S), which needs every epilogue warp's release of chunk
-// c + kPairSbSlots - S - 2 >= c + 1, issued after the warp's last read of slot
-// c; a proxy fence before each release orders those reads before the refill.
+// wait and one commit per chunk in the MMA warp) and the bounded waits are
+// those of gemm.cuh.  Here go[s] lives on the leader and counts the leader's
+// expect_tx, both CTAs' TMA bytes and 16 epilogue warps; done[s] is signalled
+// in both CTAs by one multicast commit.
+// The scale factors travel with the operands: each CTA TMA-loads chunk c's
+// row scales of its 128 rows and the B scales of the tile (the two 128x128
+// block scales, or the 256 per-column scales in FP8Q_SFB_ROW) into slot
+// c % kPairScaleSlots of a ring, counted on go[], so the epilogue reads them
+// from shared memory after done(c) with no load latency and no barrier of
+// their own.  The slot is refilled (chunk c + kPairScaleSlots) after done(c +
+// kPairScaleSlots - S), which needs every epilogue warp's release of chunk
+// c + kPairScaleSlots - S - 2 >= c + 1, issued after the warp's last read of
+// slot c; a proxy fence before each release orders those reads before the
+// refill.
 #pragma once
 
 #include "gemm.cuh"
@@ -40,13 +43,21 @@ constexpr int kPairStages = FP8Q_PAIR_STAGES;
 constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
 constexpr uint32_t kPairBBytes = 128 * BK;                    // 16 KB (half of the 256-row B tile)
 constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
-constexpr int kPairSbSlots = 12;                              // per-column scale ring (>= S + 3)
-static_assert(kPairSbSlots >= kPairStages + 3, "a scale slot may be refilled while still being read");
+constexpr int kPairScaleSlots = 12;                           // scale ring (>= S + 3)
+static_assert(kPairScaleSlots >= kPairStages + 3, "a scale slot may be refilled while still being read");
+// One slot: B scales at 0 (256 per-column floats, or a 4 x 2 box of block
+// scales: chunks (c & ~3)..+3 of the tile's two 128-column blocks), the 128
+// row scales of this CTA at 1024.
+constexpr uint32_t kPairSlotBytes = 2048;
+constexpr uint32_t kPairSlotSa = 1024;
+constexpr uint32_t kPairSaBytes = 128 * 4;
+template <int kSfbMode>
+__host__ __device__ constexpr uint32_t pair_sb_bytes() { return kSfbMode == FP8Q_SFB_ROW ? BN * 4 : 4 * 2 * 4; }
 
 struct PairSmemLayout {
   static constexpr uint32_t stages = 0;
-  static constexpr uint32_t sb_ring = stages + kPairStages * kPairStageBytes;
-  static constexpr uint32_t bars = sb_ring + kPairSbSlots * kSbBytes;
+  static constexpr uint32_t scales = stages + kPairStages * kPairStageBytes;
+  static constexpr uint32_t bars = scales + kPairScaleSlots * kPairSlotBytes;
   // go[S], done[S]
   static constexpr uint32_t nbars = 2 * kPairStages;
   static constexpr uint32_t misc = bars + nbars * 8;
@@ -56,7 +67,8 @@ struct PairSmemLayout {
 template <int kSfbMode, bool kOutF32>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                 const __grid_constant__ CUtensorMap tmap_sb, const GemmArgs p) {
+                 const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
+                 const GemmArgs p) {
   extern __shared__ uint8_t pair_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pair_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PairSmemLayout::bars);
@@ -84,7 +96,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   if (warp == 8 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
-    if (kSfbMode == FP8Q_SFB_ROW) prefetch_tmap(&tmap_sb);
+    prefetch_tmap(&tmap_sa);
+    prefetch_tmap(&tmap_sb);
   }
   if (warp == 9) { tmem_alloc_pair(tmem_slot, 512); tmem_relinquish_pair(); }
   tc_fence_before();
@@ -123,13 +136,17 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             if (!mbar_wait(&done[s], ph ^ 1, abort_flag, WAIT_PRODUCER_EMPTY)) { ok = false; break; }
             uint8_t* st = smem + PairSmemLayout::stages + s * kPairStageBytes;
             const uint32_t leader_go = leader_go0 + static_cast<uint32_t>(s) * 8u;
-            if (rank == 0)   // both CTAs' bytes (operands, and per-column scales in FP8Q_SFB_ROW)
-              mbar_arrive_expect_tx(&go[s], 2 * (kPairStageBytes + (kSfbMode == FP8Q_SFB_ROW ? kSbBytes : 0u)));
+            uint8_t* slot = smem + PairSmemLayout::scales + (it % kPairScaleSlots) * kPairSlotBytes;
+            if (rank == 0)   // both CTAs' operand and scale bytes
+              mbar_arrive_expect_tx(&go[s], 2 * (kPairStageBytes + kPairSaBytes + pair_sb_bytes<kSfbMode>()));
             tma_load_2d_pair(st, &tmap_a, leader_go, kc * BK, a_row0);
             tma_load_2d_pair(st + kPairABytes, &tmap_b, leader_go, kc * BK, b_row0);
+            // sa[kc][a_row0 .. +127] (rows past M read as zero)
+            tma_load_2d_pair(slot + kPairSlotSa, &tmap_sa, leader_go, a_row0, kc);
             if (kSfbMode == FP8Q_SFB_ROW)   // sb[kc][n0 .. n0+255] (columns past N read as zero)
-              tma_load_2d_pair(smem + PairSmemLayout::sb_ring + (it % kPairSbSlots) * kSbBytes, &tmap_sb, leader_go,
-                               n0, kc);
+              tma_load_2d_pair(slot, &tmap_sb, leader_go, n0, kc);
+            else                            // sb[n0/128 .. +1][(kc & ~3) .. +3]: a 16-byte aligned group
+              tma_load_2d_pair(slot, &tmap_sb, leader_go, kc & ~3, n0 / 128);
           }
         }
         if (!ok && rank == 0) {
@@ -188,28 +205,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       const bool vcol = ncol0 < p.N;
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-      const float* sa_ptr = p.sfa + row;
-      const float* sb_ptr = p.sfb + static_cast<int64_t>(ncol0 / 128) * p.ld_sfb;
-      auto load_sa = [&](int k) -> float {
-        return (vrow && k < nk) ? __ldg(sa_ptr + static_cast<int64_t>(k) * p.ld_sfa) : 0.0f;
-      };
-      auto load_sb = [&](int k) -> float {
-        return (kSfbMode == FP8Q_SFB_BLOCK128 && vcol && k < nk) ? __ldg(sb_ptr + k) : 0.0f;
-      };
-      float sa_q0 = load_sa(0), sa_q1 = load_sa(1), sa_q2 = load_sa(2), sa_q3 = load_sa(3);
-      float sb_q0 = load_sb(0), sb_q1 = load_sb(1), sb_q2 = load_sb(2), sb_q3 = load_sb(3);
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int b = it & 1;
         const int s = it % kPairStages;
-        const float sa = sa_q0;
-        const float sbk = sb_q0;
-        sa_q0 = sa_q1; sa_q1 = sa_q2; sa_q2 = sa_q3; sa_q3 = load_sa(kc + 4);
-        sb_q0 = sb_q1; sb_q1 = sb_q2; sb_q2 = sb_q3; sb_q3 = load_sb(kc + 4);
         if (!warp_wait(&done[s], (it / kPairStages) & 1, abort_flag, WAIT_EPI_TMEM_FULL)) { ok = false; break; }
-        const float* sbv = nullptr;
-        if (kSfbMode == FP8Q_SFB_ROW)   // landed with the operands (go[] counted its bytes)
-          sbv = reinterpret_cast<const float*>(smem + PairSmemLayout::sb_ring + (it % kPairSbSlots) * kSbBytes) +
-                half * 128;
+        // this chunk's scales landed with its operands (go[] counted their bytes)
+        const float* slot = reinterpret_cast<const float*>(smem + PairSmemLayout::scales +
+                                                           (it % kPairScaleSlots) * kPairSlotBytes);
+        const float sa = slot[kPairSlotSa / 4 + r_in_tile];
+        const float* sbv = slot + half * 128;                                  // FP8Q_SFB_ROW
+        const float sbk = kSfbMode == FP8Q_SFB_ROW ? 0.0f : slot[half * 4 + (kc & 3)];
         tc_fence_after();
         const float scale = sa * sbk;
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
@@ -219,7 +224,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         tmem_ld_32x32b_x64_sync(taddr + 64, v);
         // scale slots read so far (ordinary loads) are refilled by TMA (async
         // proxy) only after releases like this one: order across proxies
-        if (kSfbMode == FP8Q_SFB_ROW) fence_proxy_async_shared();
+        fence_proxy_async_shared();
         tc_fence_before();
         __syncwarp();
         if (lane == 0)   // buffer b is free for chunk it + 2

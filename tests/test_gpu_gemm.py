@@ -34,7 +34,17 @@ def sfa_dev(sf_mk, ld=None):
     return to_dev_f32(buf)
 
 
-def run_gemm(fp8q, qa, sfa, qb, sfb, mode, out_f32=False, lda=None, ldb=None, ldd=None):
+def sfb_dev(sfb, pad=True):
+    """Block scales [N/128][K/128] on the device; with pad, the row stride is
+    rounded up to 4 floats (the layout the CTA-pair kernel loads with TMA)."""
+    NB, KB = sfb.shape
+    ld = (KB + 3) // 4 * 4 if pad else KB
+    buf = np.full((NB, ld), np.nan, np.float32)
+    buf[:, :KB] = sfb
+    return to_dev_f32(buf)[:, :KB]
+
+
+def run_gemm(fp8q, qa, sfa, qb, sfb, mode, out_f32=False, lda=None, ldb=None, ldd=None, pad_sfb=True):
     """qa [M][K], sfa [M][K/128]; qb [N][K]; sfb [N/128][K/128] (BLK) or [N][K/128] (ROW)."""
     import torch
     M, K = qa.shape
@@ -47,7 +57,7 @@ def run_gemm(fp8q, qa, sfa, qb, sfb, mode, out_f32=False, lda=None, ldb=None, ld
     a = to_dev_u8(abuf)[:, :K]
     b = to_dev_u8(bbuf)[:, :K]
     sa = sfa_dev(sfa)
-    sb = to_dev_f32(sfb) if mode == BLK else sfa_dev(sfb)
+    sb = sfb_dev(sfb, pad_sfb) if mode == BLK else sfa_dev(sfb)
     dt = torch.float32 if out_f32 else torch.bfloat16
     dbuf = torch.full((M + 2, ldd), -3.0, dtype=dt, device="cuda")
     d = dbuf[1:M + 1, :N]
@@ -111,6 +121,17 @@ def test_gemm_parity_small(fp8q, dense_kernel, M, N, K, mode, f32):
     ref = oracle.gemm_sampled(qa, sa, qb, sb, mode)
     d = run_gemm(fp8q, qa, sa, qb, sb, mode, f32, lda=K + 16, ldb=K + 32, ldd=N + 8)
     check_gemm(d, ref, rounded(ref, f32))
+
+
+def test_gemm_unaligned_scale_layout(fp8q, dense_kernel):
+    """Block scales with a row stride of K/128 = 5 floats: the CTA-pair kernel
+    cannot TMA-load them, so even when forced the one-CTA kernel runs."""
+    M, N, K = 300, 384, 640
+    qa, sa = oracle.quant_act_1x128(W.activations_with_outliers(M, K, seed=7, channel_frac=2 / K, elem_frac=1e-3))
+    qb, sb = oracle.quant_w_128x128(W.weights(N, K, seed=8))
+    ref = oracle.gemm_sampled(qa, sa, qb, sb, BLK)
+    d = run_gemm(fp8q, qa, sa, qb, sb, BLK, pad_sfb=False)
+    check_gemm(d, ref, rounded(ref, False))
 
 
 def test_gemm_integer_exact(fp8q, dense_kernel):
