@@ -82,6 +82,11 @@ def _edge_rows():
     rows.append(t)
     # amax = 448 * 2^-5 -> s = 2^-5: midpoints scaled
     rows.append(t * np.float32(2.0 ** -5))
+    # amax = 1344 -> s = 3 exactly, not a power of two: x = 3*mid (exact in BF16)
+    # divides exactly onto the midpoint, while x * fl32(1/3) lands just off it,
+    # so these ties must come out of the exact (division) path
+    t3 = np.zeros(128, np.float32); t3[0] = 1344.0; t3[1:1 + mids.size] = 3 * mids; t3[20:20 + mids.size] = -3 * mids
+    rows.append(t3)
     # values far below the tile max: subnormal codes
     sub = np.linspace(-2e-4, 2e-4, 128).astype(np.float32); sub[5] = 3.0; rows.append(sub)
     for lane in range(0, 128, 9):
@@ -195,6 +200,22 @@ def test_quant_w_parity(fp8q, N, K, ldw):
     assert np.array_equal(sft, osf.T) and np.array_equal(qt, oq.T)
     q2, sf2 = run_qw(fp8q, w, False)
     assert np.array_equal(q2, oq) and np.array_equal(sf2, osf)
+
+
+def test_quant_w_edge_blocks(fp8q):
+    """The edge tiles (zeros, -0, ties at scales 1, 2^-5 and 3, subnormal
+    landings) laid out as 128x128 weight blocks."""
+    e = _edge_rows()                                   # [rows][128]
+    reps = -(-128 // e.shape[0])
+    blk = np.concatenate([e] * reps, axis=0)[:128]     # one block per edge set
+    w = np.concatenate([blk, e[np.arange(128) % e.shape[0]][:, ::-1]], axis=0)   # two blocks
+    for i, row in enumerate(e[:8]):                    # and blocks whose max is one edge row's
+        b = np.zeros((128, 128), np.uint16); b[5] = row; b[77] = row[::-1]
+        w = np.concatenate([w, b], axis=0)
+    q, sf, qt, sft = run_qw(fp8q, np.ascontiguousarray(w), True)
+    oq, osf = oracle.quant_w_128x128(w)
+    assert np.array_equal(sf, osf) and np.array_equal(q, oq)
+    assert np.array_equal(sft, osf.T) and np.array_equal(qt, oq.T)
 
 
 def test_quant_w_full_weight(fp8q):
