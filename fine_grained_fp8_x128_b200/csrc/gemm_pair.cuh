@@ -64,6 +64,24 @@ struct PairSmemLayout {
   static constexpr uint32_t bytes = misc + 16;
 };
 
+// Per-column scales (FP8Q_SFB_ROW) on the 16x256b fragment of 16 TMEM lanes:
+// acc[4k + 2i + j] += v[4k + 2i + j] * (sa_i * sb[8k + 2c + j]) for the
+// thread's two rows i (scales sa_lo, sa_hi) and column pairs c = lane % 4.
+// Each thread needs 32 column scales, read as 16 8-byte loads that 8 lanes
+// share, instead of the 128 that a 32x32b row would need.
+__device__ __forceinline__ void promote_rows16(float* acc, const uint32_t (&v)[64], float sa_lo, float sa_hi,
+                                               const float* sb_cols) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float2 sb = *reinterpret_cast<const float2*>(sb_cols + 8 * k);
+    float c0, c1, c2, c3;
+    mul2(c0, c1, sb.x, sb.y, sa_lo, sa_lo);
+    mul2(c2, c3, sb.x, sb.y, sa_hi, sa_hi);
+    fma2(acc[4 * k + 0], acc[4 * k + 1], __uint_as_float(v[4 * k + 0]), __uint_as_float(v[4 * k + 1]), c0, c1);
+    fma2(acc[4 * k + 2], acc[4 * k + 3], __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), c2, c3);
+  }
+}
+
 template <int kSfbMode, bool kOutF32>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -212,16 +230,22 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         // this chunk's scales landed with its operands (go[] counted their bytes)
         const float* slot = reinterpret_cast<const float*>(smem + PairSmemLayout::scales +
                                                            (it % kPairScaleSlots) * kPairSlotBytes);
-        const float sa = slot[kPairSlotSa / 4 + r_in_tile];
-        const float* sbv = slot + half * 128;                                  // FP8Q_SFB_ROW
-        const float sbk = kSfbMode == FP8Q_SFB_ROW ? 0.0f : slot[half * 4 + (kc & 3)];
         tc_fence_after();
-        const float scale = sa * sbk;
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
         uint32_t v[64];
-        tmem_ld_32x32b_x64_sync(taddr, v);
-        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc, v, sa, sbv); else promote64(acc, v, scale);
-        tmem_ld_32x32b_x64_sync(taddr + 64, v);
+        if (kSfbMode == FP8Q_SFB_ROW) {
+          // 16x256b fragments: rows 32*quad + {l4, l4+8} (lanes +0), then
+          // {16+l4, 24+l4} (lanes +16); columns 8k + 2*(lane%4) + {0,1}
+          const float* sa_rows = slot + kPairSlotSa / 4 + quad * 32 + (lane >> 2);
+          const float* sb_cols = slot + half * 128 + 2 * (lane & 3);
+          tmem_ld_16x256b_x16_sync(taddr, v);
+          promote_rows16(acc, v, sa_rows[0], sa_rows[8], sb_cols);
+          tmem_ld_16x256b_x16_sync(taddr + (16u << 16), v);
+        } else {
+          tmem_ld_32x32b_x64_sync(taddr, v);
+          promote64(acc, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
+          tmem_ld_32x32b_x64_sync(taddr + 64, v);
+        }
         // scale slots read so far (ordinary loads) are refilled by TMA (async
         // proxy) only after releases like this one: order across proxies
         fence_proxy_async_shared();
@@ -229,10 +253,40 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         __syncwarp();
         if (lane == 0)   // buffer b is free for chunk it + 2
           mbar_arrive_cluster(leader_go0 + static_cast<uint32_t>((it + 2) % kPairStages) * 8u);
-        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
+        if (kSfbMode == FP8Q_SFB_ROW) {
+          const float* sa_rows = slot + kPairSlotSa / 4 + quad * 32 + 16 + (lane >> 2);
+          promote_rows16(acc + 64, v, sa_rows[0], sa_rows[8], slot + half * 128 + 2 * (lane & 3));
+        } else {
+          promote64(acc + 64, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
+        }
       }
       if (!ok) break;
-      if (vrow && vcol) {
+      if (kSfbMode == FP8Q_SFB_ROW) {
+        // 16x256b fragments: acc[64*g + 4k + 2i + j] is row 32*quad + 16g + 8i +
+        // lane/4, column 8k + 2*(lane%4) + j of this half; 4 lanes write one
+        // 32-byte sector of a row per group k
+        if (vcol) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = a_row0 + quad * 32 + 16 * g + 8 * i + (lane >> 2);
+              if (r >= p.M) continue;
+              const int64_t base = static_cast<int64_t>(r) * p.ldd + ncol0 + 2 * (lane & 3);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const float x0 = acc[64 * g + 4 * k + 2 * i], x1 = acc[64 * g + 4 * k + 2 * i + 1];
+                if (kOutF32) {
+                  *reinterpret_cast<float2*>(static_cast<float*>(p.d) + base + 8 * k) = make_float2(x0, x1);
+                } else {
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+                  *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.d) + base + 8 * k) = h;
+                }
+              }
+            }
+          }
+        }
+      } else if (vrow && vcol) {
         if (kOutF32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
 #pragma unroll
