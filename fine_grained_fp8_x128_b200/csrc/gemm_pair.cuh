@@ -64,21 +64,26 @@ struct PairSmemLayout {
   static constexpr uint32_t bytes = misc + 16;
 };
 
-// Per-column scales (FP8Q_SFB_ROW) on the 16x256b fragment of 16 TMEM lanes:
-// acc[4k + 2i + j] += v[4k + 2i + j] * (sa_i * sb[8k + 2c + j]) for the
-// thread's two rows i (scales sa_lo, sa_hi) and column pairs c = lane % 4.
-// Each thread needs 32 column scales, read as 16 8-byte loads that 8 lanes
-// share, instead of the 128 that a 32x32b row would need.
-__device__ __forceinline__ void promote_rows16(float* acc, const uint32_t (&v)[64], float sa_lo, float sa_hi,
+// Per-column scales (FP8Q_SFB_ROW) on 16x256b fragments (tmem_ld_16x256b_x8x2_sync):
+// the thread holds 4 rows x 16 columns; acc[32g + 4k + 2i + j] += v[...] *
+// (sa[2g + i] * sb[8k + 2c + j]) with c = lane % 4.  Each column-scale pair is
+// one 8-byte shared load (shared by 8 lanes) used for all 4 rows, where a
+// 32x32b row fragment would need all 128 column scales in every thread.
+__device__ __forceinline__ void promote_rows16(float* acc, const uint32_t (&v)[64], const float* sa_rows,
                                                const float* sb_cols) {
+  float sa[4];   // rows l4, l4 + 8, l4 + 16, l4 + 24
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
+  for (int q = 0; q < 4; ++q) sa[q] = sa_rows[8 * ((q & 1) + 2 * (q >> 1))];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
     const float2 sb = *reinterpret_cast<const float2*>(sb_cols + 8 * k);
-    float c0, c1, c2, c3;
-    mul2(c0, c1, sb.x, sb.y, sa_lo, sa_lo);
-    mul2(c2, c3, sb.x, sb.y, sa_hi, sa_hi);
-    fma2(acc[4 * k + 0], acc[4 * k + 1], __uint_as_float(v[4 * k + 0]), __uint_as_float(v[4 * k + 1]), c0, c1);
-    fma2(acc[4 * k + 2], acc[4 * k + 3], __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), c2, c3);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {   // q = 2g + i
+      const int x = 32 * (q >> 1) + 4 * k + 2 * (q & 1);
+      float c0, c1;
+      mul2(c0, c1, sb.x, sb.y, sa[q], sa[q]);
+      fma2(acc[x], acc[x + 1], __uint_as_float(v[x]), __uint_as_float(v[x + 1]), c0, c1);
+    }
   }
 }
 
@@ -233,14 +238,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         tc_fence_after();
         const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(b * BN + half * 128);
         uint32_t v[64];
+        // FP8Q_SFB_ROW, 16x256b fragments: rows 32*quad + {l4, l4+8, l4+16, l4+24}
+        // with l4 = lane/4; columns 8k + 2*(lane%4) + {0,1} of each 64-column half
+        const float* sa_rows = slot + kPairSlotSa / 4 + quad * 32 + (lane >> 2);
         if (kSfbMode == FP8Q_SFB_ROW) {
-          // 16x256b fragments: rows 32*quad + {l4, l4+8} (lanes +0), then
-          // {16+l4, 24+l4} (lanes +16); columns 8k + 2*(lane%4) + {0,1}
-          const float* sa_rows = slot + kPairSlotSa / 4 + quad * 32 + (lane >> 2);
-          const float* sb_cols = slot + half * 128 + 2 * (lane & 3);
-          tmem_ld_16x256b_x16_sync(taddr, v);
-          promote_rows16(acc, v, sa_rows[0], sa_rows[8], sb_cols);
-          tmem_ld_16x256b_x16_sync(taddr + (16u << 16), v);
+          tmem_ld_16x256b_x8x2_sync(taddr, v);
+          promote_rows16(acc, v, sa_rows, slot + half * 128 + 2 * (lane & 3));
+          tmem_ld_16x256b_x8x2_sync(taddr + 64, v);
         } else {
           tmem_ld_32x32b_x64_sync(taddr, v);
           promote64(acc, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
@@ -254,17 +258,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         if (lane == 0)   // buffer b is free for chunk it + 2
           mbar_arrive_cluster(leader_go0 + static_cast<uint32_t>((it + 2) % kPairStages) * 8u);
         if (kSfbMode == FP8Q_SFB_ROW) {
-          const float* sa_rows = slot + kPairSlotSa / 4 + quad * 32 + 16 + (lane >> 2);
-          promote_rows16(acc + 64, v, sa_rows[0], sa_rows[8], slot + half * 128 + 2 * (lane & 3));
+          promote_rows16(acc + 64, v, sa_rows, slot + half * 128 + 64 + 2 * (lane & 3));
         } else {
           promote64(acc + 64, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
         }
       }
       if (!ok) break;
       if (kSfbMode == FP8Q_SFB_ROW) {
-        // 16x256b fragments: acc[64*g + 4k + 2i + j] is row 32*quad + 16g + 8i +
-        // lane/4, column 8k + 2*(lane%4) + j of this half; 4 lanes write one
-        // 32-byte sector of a row per group k
+        // 16x256b fragments: acc[64h + 32g + 4k + 2i + j] is row 32*quad + 16g +
+        // 8i + lane/4, column 64h + 8k + 2*(lane%4) + j of this half; 4 lanes
+        // write one 32-byte sector of a row per group k
         if (vcol) {
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
@@ -274,8 +277,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
               if (r >= p.M) continue;
               const int64_t base = static_cast<int64_t>(r) * p.ldd + ncol0 + 2 * (lane & 3);
 #pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const float x0 = acc[64 * g + 4 * k + 2 * i], x1 = acc[64 * g + 4 * k + 2 * i + 1];
+              for (int k = 0; k < 16; ++k) {   // k < 8: first 64 columns, k >= 8: second
+                const int x = 64 * (k >> 3) + 32 * g + 4 * (k & 7) + 2 * i;
+                const float x0 = acc[x], x1 = acc[x + 1];
                 if (kOutF32) {
                   *reinterpret_cast<float2*>(static_cast<float*>(p.d) + base + 8 * k) = make_float2(x0, x1);
                 } else {
