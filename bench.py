@@ -350,7 +350,20 @@ class DeviceStep:
         self.h_dx = torch.empty_like(self.dx, device="cpu").pin_memory()
         self.h_dw = torch.empty_like(self.dw, device="cpu").pin_memory()
         self.h_out = torch.empty_like(self.out, device="cpu").pin_memory()
+        # the end-to-end leg double-buffers the step's inputs and outputs so that
+        # the copies of neighbouring steps overlap this step's kernels
+        self.slots = [self._slot_tensors()]
+        self.slots.append({k: torch.empty_like(v) for k, v in self.slots[0].items()})
         torch.cuda.synchronize()
+
+    _SLOT = ("x", "dy", "xp", "off", "y", "dx", "dw", "out")
+
+    def _slot_tensors(self):
+        return {k: getattr(self, k) for k in self._SLOT}
+
+    def use_slot(self, b):
+        for k, v in self.slots[b].items():
+            setattr(self, k, v)
 
     def h2d_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_dy, self.h_xp, self.h_off))
@@ -515,18 +528,50 @@ def run_fp8q(args):
     value = world * flops_step * args.steps / t_max / 1e12
     stats = kernel_stats(events, args.steps)
 
-    # ---- end-to-end: host inputs in, host outputs back, through the public API
+    # ---- end-to-end: host inputs in, host outputs back, through the public API.
+    # Every step uploads its inputs and downloads its outputs inside the timed
+    # region; with two buffer sets, step i+1's upload and step i-1's download
+    # run on their own streams while step i's kernels run.
     barrier(world, device)
     torch.cuda.synchronize()
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        st.upload()
+    e0.record(comp)
+
+    def upload_into(b, after=None):
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(e0)
+            if after is not None:
+                s_in.wait_event(after)      # the slot's previous step has finished reading it
+            st.use_slot(b)
+            st.upload()
+            in_ready[b].record(s_in)
+
+    upload_into(0)
+    for i in range(args.steps):
+        b = i % 2
+        if i + 1 < args.steps:
+            upload_into(b ^ 1, comp_done[b ^ 1] if i >= 1 else None)
+        comp.wait_event(in_ready[b])
+        if i >= 2:
+            comp.wait_event(out_done[b])    # step i-2's outputs have left this slot
+        st.use_slot(b)
         st.step()
-        st.download()
-    e1.record()
+        comp_done[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            st.download()
+            out_done[b].record(s_out)
+    comp.wait_event(out_done[(args.steps - 1) % 2])
+    if args.steps >= 2:
+        comp.wait_event(out_done[args.steps % 2])
+    e1.record(comp)
     torch.cuda.synchronize()
+    st.use_slot(0)
     e2e_t = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world, device)
     e2e_value = world * flops_step * args.steps / e2e_t / 1e12
     code = fp8q.fp8q_device_status()
