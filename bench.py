@@ -8,8 +8,9 @@ seeded, outlier-injected input:
     quant_act_1x128(dY) -> Dgrad  dX = dY W           (BF16 out)
     quant_act_128x1(dY), quant_act_128x1(X) -> Wgrad dW = dY^T X   (FP32 out)
   MoE layer, 4096 tokens, top-8 of 256 experts (Zipf 1.1), hidden 7168, expert 2048:
-    quant_act_1x128(X packed) -> grouped up-projection (BF16 out)
-    quant_act_1x128(H)        -> grouped down-projection (BF16 out)
+    quant_act_1x128 over the dispatch gather (tokens -> expert rows)
+    grouped up-projection, epilogue emitting H as 1x128 FP8 tiles
+    grouped down-projection (BF16 out)
 Expert weights are resident FP8 (quantized once at set-up); the dense weight is
 re-quantized inside every step.
 
@@ -73,8 +74,9 @@ def quant_bytes():
         "quant_dy": act(TOK, OUT),
         "quant_dy_t": act(TOK, OUT),
         "quant_x_t": act(TOK, HID),
-        "quant_moe_x": act(MOE_TOK * MOE_K, HID),
-        "quant_moe_h": act(MOE_TOK * MOE_K, MOE_FF),
+        # the gather reads each token once from HBM (the 59 MB of tokens stay
+        # in the L2 across their top-k copies) and writes every expert row
+        "quant_moe_x": MOE_TOK * HID * 2 + MOE_TOK * MOE_K * HID + (MOE_TOK * MOE_K * HID // 128) * 4,
     }
 
 
@@ -222,7 +224,6 @@ class CpuSample:
         exp_of_row = np.searchsorted(route.offsets, pick, side="right") - 1
         self.experts = np.unique(exp_of_row)
         self.moe_x = W.activations_with_outliers(rows, HID, seed=seed + 300)
-        self.moe_h = W.normal_bf16(rows, MOE_FF, 1.0, seed=seed, tid=W.TID_H)
         self.exp_local = np.searchsorted(self.experts, exp_of_row)
         self.w_up = W.expert_weights(len(self.experts), MOE_FF, HID, seed=seed, tid=W.TID_EXPERT_UP,
                                      experts=self.experts)
@@ -230,7 +231,7 @@ class CpuSample:
                                      experts=self.experts)
         # rows sorted by expert so each expert owns a contiguous range
         order = np.argsort(self.exp_local, kind="stable")
-        self.moe_x, self.moe_h, self.exp_local = self.moe_x[order], self.moe_h[order], self.exp_local[order]
+        self.moe_x, self.exp_local = self.moe_x[order], self.exp_local[order]
         self.moe_off = W.ragged_offsets(np.bincount(self.exp_local, minlength=len(self.experts)))
 
     def flops(self):
@@ -240,7 +241,8 @@ class CpuSample:
     def description(self):
         return (f"{self.R} full output rows of each of the 5 GEMMs of the step (Fprop, Dgrad, Wgrad, MoE up, "
                 f"MoE down) with the quantizations they need (W and W^T 18432x7168 in full, X^T 8192x7168 in "
-                f"full for Wgrad, {len(self.experts)} experts' up/down weights)")
+                f"full for Wgrad, {len(self.experts)} experts' up/down weights, the up projection's BF16 rows "
+                f"re-quantized 1x128 as the down projection's input)")
 
     def run(self):
         import oracle
@@ -259,8 +261,8 @@ class CpuSample:
         wq = np.empty((G, MOE_FF, HID), np.uint8); ws = np.empty((G, MOE_FF // 128, HID // 128), np.float32)
         for g in range(G):
             wq[g], ws[g] = oracle.quant_w_128x128(self.w_up[g])
-        oracle.grouped_gemm_sampled(qa, sa, wq, ws, self.moe_off)
-        qh, sh = oracle.quant_act_1x128(self.moe_h)
+        h = oracle.grouped_gemm_sampled(qa, sa, wq, ws, self.moe_off)
+        qh, sh = oracle.quant_act_1x128(W.f32_to_bf16_bits(oracle.round_bf16(h).astype(np.float32)))
         wq = np.empty((G, HID, MOE_FF), np.uint8); ws = np.empty((G, HID // 128, MOE_FF // 128), np.float32)
         for g in range(G):
             wq[g], ws[g] = oracle.quant_w_128x128(self.w_dn[g])
@@ -280,11 +282,11 @@ def time_cpu_sample(sample: CpuSample):
 
 # ----------------------------------------------------------------------------- the device step
 class DeviceStep:
-    """All buffers of one step, resident on the device; step() launches the 12
+    """All buffers of one step, resident on the device; step() launches the 11
     kernels of the hot path on the current stream."""
 
     KERNELS = ("quant_w", "quant_x", "fprop", "quant_dy", "dgrad", "quant_dy_t", "quant_x_t", "wgrad",
-               "quant_moe_x", "moe_up", "quant_moe_h", "moe_down")
+               "quant_moe_x", "moe_up", "moe_down")
 
     def __init__(self, fp8q, seed: int, device):
         import torch
@@ -304,12 +306,14 @@ class DeviceStep:
         route = W.moe_routing(tokens=MOE_TOK, experts=MOE_E, top_k=MOE_K, seed=seed)
         self.mt = int(route.offsets[-1])
         xt = W.activations_with_outliers(MOE_TOK, HID, seed=seed, tid=W.TID_MISC)
-        self.h_xp = torch.from_numpy(np.ascontiguousarray(xt[route.token_of_row]).view(np.int16)).view(bf).pin_memory()
+        self.h_xm = torch.from_numpy(xt.view(np.int16)).view(bf).pin_memory()       # MoE tokens, token order
+        self.h_rows = torch.from_numpy(route.token_of_row.astype(np.int32)).pin_memory()   # expert row -> token
         self.h_off = torch.from_numpy(route.offsets.astype(np.int32)).pin_memory()
         self.w = dev_bf16(W.weights(OUT, HID, seed=seed))                      # model state, resident
         self.x = torch.empty((TOK, HID), dtype=bf, device=device)
         self.dy = torch.empty((TOK, OUT), dtype=bf, device=device)
-        self.xp = torch.empty((self.mt, HID), dtype=bf, device=device)
+        self.xm = torch.empty((MOE_TOK, HID), dtype=bf, device=device)
+        self.rows = torch.empty((self.mt,), dtype=torch.int32, device=device)
         self.off = torch.empty((MOE_E + 1,), dtype=torch.int32, device=device)
         self.upload()
         # quantized operands and outputs
@@ -341,7 +345,6 @@ class DeviceStep:
             del wb
         self.xpq = torch.empty((self.mt, HID), dtype=u8, device=device)
         self.sxp = torch.empty((HID // 128, ld(self.mt)), dtype=f32, device=device)
-        self.h = torch.empty((self.mt, MOE_FF), dtype=bf, device=device)
         self.hq = torch.empty((self.mt, MOE_FF), dtype=u8, device=device)
         self.sh = torch.empty((MOE_FF // 128, ld(self.mt)), dtype=f32, device=device)
         self.out = torch.empty((self.mt, HID), dtype=bf, device=device)
@@ -356,7 +359,7 @@ class DeviceStep:
         self.slots.append({k: torch.empty_like(v) for k, v in self.slots[0].items()})
         torch.cuda.synchronize()
 
-    _SLOT = ("x", "dy", "xp", "off", "y", "dx", "dw", "out")
+    _SLOT = ("x", "dy", "xm", "rows", "off", "y", "dx", "dw", "out")
 
     def _slot_tensors(self):
         return {k: getattr(self, k) for k in self._SLOT}
@@ -366,7 +369,7 @@ class DeviceStep:
             setattr(self, k, v)
 
     def h2d_bytes(self):
-        return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_dy, self.h_xp, self.h_off))
+        return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_dy, self.h_xm, self.h_rows, self.h_off))
 
     def d2h_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.h_y, self.h_dx, self.h_dw, self.h_out))
@@ -374,7 +377,8 @@ class DeviceStep:
     def upload(self):
         self.x.copy_(self.h_x, non_blocking=True)
         self.dy.copy_(self.h_dy, non_blocking=True)
-        self.xp.copy_(self.h_xp, non_blocking=True)
+        self.xm.copy_(self.h_xm, non_blocking=True)
+        self.rows.copy_(self.h_rows, non_blocking=True)
         self.off.copy_(self.h_off, non_blocking=True)
 
     def download(self):
@@ -384,7 +388,7 @@ class DeviceStep:
         self.h_out.copy_(self.out, non_blocking=True)
 
     def step(self, events=None):
-        """Launch the 12 kernels; if `events` is a list, append (name, start, end) CUDA events."""
+        """Launch the 11 kernels; if `events` is a list, append (name, start, end) CUDA events."""
         import torch
         f = self.fp8q
         ops = (
@@ -398,10 +402,9 @@ class DeviceStep:
             ("quant_x_t", lambda: f.fp8q_quant_act_128x1(self.x, self.xqt, self.sxt)),
             ("wgrad", lambda: f.fp8q_gemm_blockscaled(self.dyqt, self.sdyt, self.xqt, self.sxt, f.FP8Q_SFB_ROW,
                                                       self.dw)),
-            ("quant_moe_x", lambda: f.fp8q_quant_act_1x128(self.xp, self.xpq, self.sxp)),
-            ("moe_up", lambda: f.fp8q_grouped_gemm_blockscaled(self.xpq, self.sxp, self.wup_q, self.wup_s, self.off,
-                                                               self.h)),
-            ("quant_moe_h", lambda: f.fp8q_quant_act_1x128(self.h, self.hq, self.sh)),
+            ("quant_moe_x", lambda: f.fp8q_quant_act_1x128_gather(self.xm, self.rows, self.xpq, self.sxp)),
+            ("moe_up", lambda: f.fp8q_grouped_gemm_blockscaled_q1x128(self.xpq, self.sxp, self.wup_q, self.wup_s,
+                                                                      self.off, self.hq, self.sh)),
             ("moe_down", lambda: f.fp8q_grouped_gemm_blockscaled(self.hq, self.sh, self.wdn_q, self.wdn_s, self.off,
                                                                  self.out)),
         )
@@ -423,7 +426,8 @@ def config_block(world):
     return {
         "workload": ("one training step of a 8192-token linear layer 7168->18432 (weight quant with W^T, "
                      "Fprop, Dgrad, Wgrad with 1x128 / 128x1 / 128x128 quantization) plus a 4096-token MoE "
-                     "layer (top-8 of 256 experts, Zipf 1.1, 8 empty; grouped up 7168->2048 and down 2048->7168)"),
+                     "layer (top-8 of 256 experts, Zipf 1.1, 8 empty; dispatch gather fused into the 1x128 "
+                     "quantizer, grouped up 7168->2048 with FP8 epilogue, grouped down 2048->7168)"),
         "tokens": TOK, "hidden": HID, "out_features": OUT,
         "moe_tokens": MOE_TOK, "experts": MOE_E, "top_k": MOE_K, "expert_ffn": MOE_FF,
         "tile": "1x128 activations, 128x1 (Wgrad), 128x128 weights; promotion every 128 of K",
@@ -581,7 +585,7 @@ def run_fp8q(args):
     nz = int((st.h_off[1:] - st.h_off[:-1] > 0).sum())
     moe_w = nz * MOE_FF * HID + nz * (MOE_FF // 128) * (HID // 128) * 4
     mt = st.mt
-    moe_other = {"moe_up": mt * HID + (HID // 128) * mt * 4 + mt * MOE_FF * 2,
+    moe_other = {"moe_up": mt * HID + (HID // 128) * mt * 4 + mt * MOE_FF + (MOE_FF // 128) * mt * 4,
                  "moe_down": mt * MOE_FF + (MOE_FF // 128) * mt * 4 + mt * HID * 2}
     breakdown = build_breakdown(stats, pk, moe_w, moe_other)
     dominant = max(stats, key=lambda n: stats[n][1])
@@ -640,7 +644,8 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "moe_up", "moe_down")
+SINGLE_KERNELS = ("quant_x", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+                  "moe_down")
 
 
 def run_single(args):
@@ -693,18 +698,31 @@ def run_single(args):
             mode = fp8q.FP8Q_SFB_BLOCK128
         fn = lambda: fp8q.fp8q_gemm_blockscaled(qa, sa, qb, sb, mode, d)
         work = ("flops", 2.0 * M * N * K)
-    elif name in ("moe_up", "moe_down"):
+    elif name in ("quant_moe_x", "moe_up", "moe_up_q", "moe_down"):
         moe_tokens = MOE_TOK if T == TOK else T          # --tokens counts MoE tokens before top-k
         route = W.moe_routing(tokens=moe_tokens, experts=MOE_E, top_k=MOE_K, seed=0)
         mt = int(route.offsets[-1])
-        K, N = (HID, MOE_FF) if name == "moe_up" else (MOE_FF, HID)
-        qa, sa = fp8q.quant_act_1x128(randn(mt, K))
-        wq = torch.randint(0, 0x7E, (MOE_E, N, K), generator=gen, device=dev, dtype=torch.int32).to(u8)
-        ws = torch.rand((MOE_E, N // 128, K // 128), generator=gen, device=dev) * 1e-3
-        off = torch.from_numpy(route.offsets.astype(np.int32)).to(dev)
-        d = torch.empty((mt, N), dtype=bf, device=dev)
-        fn = lambda: fp8q.fp8q_grouped_gemm_blockscaled(qa, sa, wq, ws, off, d)
-        work = ("flops", 2.0 * mt * N * K)
+        if name == "quant_moe_x":
+            xm = randn(moe_tokens, HID)
+            rows = torch.from_numpy(route.token_of_row.astype(np.int32)).to(dev)
+            q = torch.empty((mt, HID), dtype=u8, device=dev)
+            sf = torch.empty((HID // 128, ld(mt)), dtype=f32, device=dev)
+            fn = lambda: fp8q.fp8q_quant_act_1x128_gather(xm, rows, q, sf)
+            work = ("bytes", moe_tokens * HID * 2 + mt * HID + mt * HID // 128 * 4)
+        else:
+            K, N = (MOE_FF, HID) if name == "moe_down" else (HID, MOE_FF)
+            qa, sa = fp8q.quant_act_1x128(randn(mt, K))
+            wq = torch.randint(0, 0x7E, (MOE_E, N, K), generator=gen, device=dev, dtype=torch.int32).to(u8)
+            ws = torch.rand((MOE_E, N // 128, K // 128), generator=gen, device=dev) * 1e-3
+            off = torch.from_numpy(route.offsets.astype(np.int32)).to(dev)
+            if name == "moe_up_q":
+                dq = torch.empty((mt, N), dtype=u8, device=dev)
+                sfd = torch.empty((N // 128, ld(mt)), dtype=f32, device=dev)
+                fn = lambda: fp8q.fp8q_grouped_gemm_blockscaled_q1x128(qa, sa, wq, ws, off, dq, sfd)
+            else:
+                d = torch.empty((mt, N), dtype=bf, device=dev)
+                fn = lambda: fp8q.fp8q_grouped_gemm_blockscaled(qa, sa, wq, ws, off, d)
+            work = ("flops", 2.0 * mt * N * K)
     else:
         raise SystemExit(f"unknown kernel {name}; choose from {SINGLE_KERNELS}")
     scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)

@@ -38,8 +38,9 @@ FP8Q_OUT_F32 = 1
 
 EXPORTS = (
     "fp8q_version", "fp8q_status_string", "fp8q_device_status",
-    "fp8q_quant_act_1x128", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
-    "fp8q_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled",
+    "fp8q_quant_act_1x128", "fp8q_quant_act_1x128_gather", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
+    "fp8q_gemm_blockscaled", "fp8q_gemm_blockscaled_q1x128",
+    "fp8q_grouped_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled_q1x128",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
 )
 
@@ -50,11 +51,15 @@ _lib.fp8q_status_string.argtypes = [ctypes.c_int]
 _lib.fp8q_status_string.restype = ctypes.c_char_p
 _lib.fp8q_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int)]
 _lib.fp8q_quant_act_1x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_1x128_gather.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_128x1.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_w_128x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_gemm_blockscaled.argtypes = [_P, _I, _P, _I, _P, _I, _P, _I, ctypes.c_int, _P, _I, ctypes.c_int,
                                        _I, _I, _I, _P]
+_lib.fp8q_gemm_blockscaled_q1x128.argtypes = [_P, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P, _I, _I, _I, _I, _P]
 _lib.fp8q_grouped_gemm_blockscaled.argtypes = [_P, _I, _P, _I, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P]
+_lib.fp8q_grouped_gemm_blockscaled_q1x128.argtypes = [_P, _I, _P, _I, _P, _P, _P, _I, _I, _P, _I, _P, _I, _I, _I,
+                                                      _P]
 _lib.fp8q_debug_cast_e4m3_bits.argtypes = [ctypes.c_uint32, _I, _P, _P]
 _lib.fp8q_debug_wait_timeout.argtypes = [_I, _P]
 for _n in EXPORTS[2:]:
@@ -119,6 +124,14 @@ def fp8q_quant_act_1x128(x, q, sf, stream=None):
                                      _stream(stream)), "fp8q_quant_act_1x128")
 
 
+def fp8q_quant_act_1x128_gather(x, rows, q, sf, stream=None):
+    """q[m] / sf[:, m] = 1x128 quantization of x[rows[m]]; rows int32 [M] on device."""
+    M_src, K = x.shape
+    M = rows.shape[0]
+    _check(_lib.fp8q_quant_act_1x128_gather(_ptr(x), M_src, K, _ld(x), _ptr(rows), M, _ptr(q), _ld(q), _ptr(sf),
+                                            _ld(sf), _stream(stream)), "fp8q_quant_act_1x128_gather")
+
+
 def fp8q_quant_act_128x1(x, qt, sf, stream=None):
     """x bf16 [T][C] -> qt uint8 [C][T], sf float32 [T/128][ld_sf >= C]."""
     T, C = x.shape
@@ -145,6 +158,15 @@ def fp8q_gemm_blockscaled(a, sfa, b, sfb, sfb_mode, d, stream=None):
            "fp8q_gemm_blockscaled")
 
 
+def fp8q_gemm_blockscaled_q1x128(a, sfa, b, sfb, dq, sfd, stream=None):
+    """dq[M][N] uint8, sfd [N/128][ld >= M]: 1x128 quantization of the bf16 GEMM result."""
+    M, K = a.shape
+    N = b.shape[0]
+    _check(_lib.fp8q_gemm_blockscaled_q1x128(_ptr(a), _ld(a), _ptr(sfa), _ld(sfa), _ptr(b), _ld(b), _ptr(sfb),
+                                             _ld(sfb), _ptr(dq), _ld(dq), _ptr(sfd), _ld(sfd), M, N, K,
+                                             _stream(stream)), "fp8q_gemm_blockscaled_q1x128")
+
+
 def fp8q_grouped_gemm_blockscaled(a, sfa, w, sfw, group_offsets, d, stream=None):
     """Per-expert block-scaled GEMM; w [G][N][K], sfw [G][N/128][K/128], offsets int32 [G+1] on device."""
     M_total, K = a.shape
@@ -152,6 +174,16 @@ def fp8q_grouped_gemm_blockscaled(a, sfa, w, sfw, group_offsets, d, stream=None)
     _check(_lib.fp8q_grouped_gemm_blockscaled(_ptr(a), _ld(a), _ptr(sfa), _ld(sfa), _ptr(w), _ptr(sfw),
                                               _ptr(group_offsets), G, M_total, _ptr(d), _ld(d), N, K,
                                               _stream(stream)), "fp8q_grouped_gemm_blockscaled")
+
+
+def fp8q_grouped_gemm_blockscaled_q1x128(a, sfa, w, sfw, group_offsets, dq, sfd, stream=None):
+    """Grouped GEMM whose per-expert rows come out as 1x128 E4M3 tiles (dq uint8 [M_total][N]) and scales."""
+    M_total, K = a.shape
+    G, N, _ = w.shape
+    _check(_lib.fp8q_grouped_gemm_blockscaled_q1x128(_ptr(a), _ld(a), _ptr(sfa), _ld(sfa), _ptr(w), _ptr(sfw),
+                                                     _ptr(group_offsets), G, M_total, _ptr(dq), _ld(dq), _ptr(sfd),
+                                                     _ld(sfd), N, K, _stream(stream)),
+           "fp8q_grouped_gemm_blockscaled_q1x128")
 
 
 def fp8q_debug_cast_e4m3_bits(start: int, count: int, out, stream=None):

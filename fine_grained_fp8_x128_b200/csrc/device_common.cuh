@@ -29,6 +29,7 @@ enum : uint32_t {
   WAIT_DRAIN = 5,
   WAIT_DEBUG = 6,
   BAD_GROUP_OFFSETS = 7,
+  BAD_ROW_INDEX = 8,
 };
 
 __device__ __forceinline__ void report_status(uint32_t code, uint32_t where) {

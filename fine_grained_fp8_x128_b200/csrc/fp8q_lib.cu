@@ -26,10 +26,10 @@ std::mutex g_mu;
 struct DeviceInfo {
   bool ready = false;
   int sm_count = 0;
-  bool gemm_attr[2][2][2] = {};   // [grouped][row mode][f32 out]
+  bool gemm_attr[2][2][3] = {};   // [grouped][row mode][output mode]
   bool q2_attr = false;
-  bool pair_attr[2][2] = {};       // [row mode][f32 out]
-  int pair_clusters[2][2] = {};    // co-resident CTA pairs per kernel instance
+  bool pair_attr[2][3] = {};       // [row mode][output mode]
+  int pair_clusters[2][3] = {};    // co-resident CTA pairs per kernel instance
   int q1_per_sm = 0;               // resident blocks per SM of each quantizer
   int q2_per_sm = 0;
   int qw_per_sm = 0;
@@ -129,12 +129,12 @@ fp8q_status make_tmap_f32(CUtensorMap* map, const float* base, int64_t inner, in
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-template <bool G, int MODE, bool F32>
+template <bool G, int MODE, int OUT>
 fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const fp8q::GemmArgs& args,
                         int grid, cudaStream_t stream) {
   const uint32_t smem = (G ? fp8q::GemmSmemLayout::bytes_grouped : fp8q::GemmSmemLayout::bytes_dense) + 1024;
-  auto kern = fp8q::gemm_blockscaled_kernel<G, MODE, F32>;
-  bool& attr = dev->gemm_attr[G ? 1 : 0][MODE == FP8Q_SFB_ROW ? 1 : 0][F32 ? 1 : 0];
+  auto kern = fp8q::gemm_blockscaled_kernel<G, MODE, OUT>;
+  bool& attr = dev->gemm_attr[G ? 1 : 0][MODE == FP8Q_SFB_ROW ? 1 : 0][OUT];
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
@@ -145,13 +145,13 @@ fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMa
   return launch_status();
 }
 
-template <int MODE, bool F32>
+template <int MODE, int OUT>
 fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
                              const CUtensorMap& tsb, const fp8q::GemmArgs& args, int64_t pair_tiles,
                              cudaStream_t stream) {
   const uint32_t smem = fp8q::PairSmemLayout::bytes + 1024;
-  auto kern = fp8q::gemm_pair_kernel<MODE, F32>;
-  const int mi = MODE == FP8Q_SFB_ROW ? 1 : 0, fi = F32 ? 1 : 0;
+  auto kern = fp8q::gemm_pair_kernel<MODE, OUT>;
+  const int mi = MODE == FP8Q_SFB_ROW ? 1 : 0, fi = OUT;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -210,6 +210,145 @@ bool use_pair_kernel(int64_t M, const float* sfa, int64_t ld_sfa, const float* s
   return M > fp8q::BM;
 }
 
+// Dense GEMM launch for one scale mode: the pair or the one-CTA kernel, and
+// the output mode (the FP8 output exists for 128x128-block B scales only).
+template <int MODE>
+fp8q_status dense_launch(DeviceInfo* dev, bool pair, int out, const CUtensorMap& ta, const CUtensorMap& tb,
+                         const CUtensorMap& tsa, const CUtensorMap& tsb, const fp8q::GemmArgs& args,
+                         int64_t pair_tiles, int grid, cudaStream_t s) {
+  if (out == fp8q::kOutF32)
+    return pair ? launch_gemm_pair<MODE, fp8q::kOutF32>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+                : launch_gemm<false, MODE, fp8q::kOutF32>(dev, ta, tb, args, grid, s);
+  if constexpr (MODE == FP8Q_SFB_BLOCK128) {
+    if (out == fp8q::kOutE4m3)
+      return pair ? launch_gemm_pair<MODE, fp8q::kOutE4m3>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+                  : launch_gemm<false, MODE, fp8q::kOutE4m3>(dev, ta, tb, args, grid, s);
+  }
+  return pair ? launch_gemm_pair<MODE, fp8q::kOutBf16>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+              : launch_gemm<false, MODE, fp8q::kOutBf16>(dev, ta, tb, args, grid, s);
+}
+
+// Body of both dense GEMM entry points.  out: fp8q::kOutBf16 / kOutF32 / kOutE4m3
+// (d = E4M3 codes [M][ldd], sfd[(n/128) * ld_sfd + m] the scales of their 1x128 tiles).
+fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* b, int64_t ldb,
+                       const float* sfb, int64_t ld_sfb, int sfb_mode, void* d, int64_t ldd, int out, float* sfd,
+                       int64_t ld_sfd, int64_t M, int64_t N, int64_t K, void* stream) {
+  const int64_t kIntMax = 0x7FFFFFFF;
+  if (M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M > kIntMax || N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  if (lda < K || ldb < K || ldd < N || ld_sfa < M) return FP8Q_ERR_INVALID_ARG;
+  if (sfb_mode != FP8Q_SFB_BLOCK128 && sfb_mode != FP8Q_SFB_ROW) return FP8Q_ERR_INVALID_ARG;
+  if (sfb_mode == FP8Q_SFB_BLOCK128 && ld_sfb < K / 128) return FP8Q_ERR_INVALID_ARG;
+  if (sfb_mode == FP8Q_SFB_ROW && ld_sfb < N) return FP8Q_ERR_INVALID_ARG;
+  if (a == nullptr || b == nullptr || sfa == nullptr || sfb == nullptr || d == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (out == fp8q::kOutE4m3) {
+    if (sfb_mode != FP8Q_SFB_BLOCK128) return FP8Q_ERR_UNSUPPORTED;
+    if (sfd == nullptr || ld_sfd < M) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned(sfd, 4)) return FP8Q_ERR_ALIGNMENT;
+  }
+  const int64_t esz = out == fp8q::kOutF32 ? 4 : (out == fp8q::kOutE4m3 ? 1 : 2);
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfb, 4) ||
+      lda % 16 != 0 || ldb % 16 != 0 || (ldd * esz) % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  if (sfb_mode == FP8Q_SFB_ROW && (!aligned(sfb, 16) || ld_sfb % 4 != 0)) return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const bool pair = use_pair_kernel(M, sfa, ld_sfa, sfb, ld_sfb);
+  CUtensorMap ta, tb, tsa, tsb;
+  if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, b, K, N, ldb, pair ? fp8q::BN / 2 : fp8q::BN)) != FP8Q_OK) return st;
+  if (pair) {
+    // sa[K/128][ld_sfa]: 128 row scales per load
+    if ((st = make_tmap_f32(&tsa, sfa, M, K / 128, ld_sfa, fp8q::BM, 1)) != FP8Q_OK) return st;
+    // sb: [K/128][ld_sfb] per-column scales, 256 per load; or [N/128][ld_sfb]
+    // block scales, 4 chunks x the tile's 2 column blocks per load
+    st = sfb_mode == FP8Q_SFB_ROW ? make_tmap_f32(&tsb, sfb, N, K / 128, ld_sfb, fp8q::BN, 1)
+                                  : make_tmap_f32(&tsb, sfb, K / 128, N / 128, ld_sfb, 4, 2);
+    if (st != FP8Q_OK) return st;
+  } else {
+    tsa = tb;   // not read by the one-CTA kernel
+    tsb = tb;
+  }
+  fp8q::GemmArgs args{};
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfb;
+  args.ld_sfb = ld_sfb;
+  args.d = d;
+  args.ldd = ldd;
+  args.sfd = sfd;
+  args.ld_sfd = ld_sfd;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
+  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
+  args.num_m_tiles = static_cast<int>((M + fp8q::BM - 1) / fp8q::BM);
+  args.group_offsets = nullptr;
+  args.G = 1;
+  const int64_t tiles = static_cast<int64_t>(args.num_m_tiles) * args.num_n_tiles;
+  if (tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
+  const int64_t m_pairs = (M + 2 * fp8q::BM - 1) / (2 * fp8q::BM);
+  const int64_t pair_tiles = m_pairs * args.num_n_tiles;
+  args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return sfb_mode == FP8Q_SFB_BLOCK128
+             ? dense_launch<FP8Q_SFB_BLOCK128>(dev, pair, out, ta, tb, tsa, tsb, args, pair_tiles, grid, s)
+             : dense_launch<FP8Q_SFB_ROW>(dev, pair, out, ta, tb, tsa, tsb, args, pair_tiles, grid, s);
+}
+
+// Body of both grouped GEMM entry points (out: kOutBf16 or kOutE4m3).
+fp8q_status gemm_grouped(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* w,
+                         const float* sfw, const int32_t* group_offsets, int64_t G, int64_t M_total, void* d,
+                         int64_t ldd, int out, float* sfd, int64_t ld_sfd, int64_t N, int64_t K, void* stream) {
+  const int64_t kIntMax = 0x7FFFFFFF;
+  if (G < 1 || M_total < 0 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (G > fp8q::kMaxGroups || M_total > kIntMax || G * N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  if (lda < K || ldd < N || ld_sfa < M_total) return FP8Q_ERR_INVALID_ARG;
+  if (out == fp8q::kOutE4m3 && ld_sfd < M_total) return FP8Q_ERR_INVALID_ARG;
+  if (M_total == 0) return FP8Q_OK;
+  if (a == nullptr || w == nullptr || sfa == nullptr || sfw == nullptr || group_offsets == nullptr || d == nullptr ||
+      (out == fp8q::kOutE4m3 && sfd == nullptr))
+    return FP8Q_ERR_INVALID_ARG;
+  const int64_t esz = out == fp8q::kOutE4m3 ? 1 : 2;
+  if (!aligned(a, 16) || !aligned(w, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfw, 4) ||
+      !aligned(group_offsets, 4) || lda % 16 != 0 || (ldd * esz) % 16 != 0 ||
+      (out == fp8q::kOutE4m3 && !aligned(sfd, 4)))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = make_tmap(&ta, a, K, M_total, lda, fp8q::BM)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, w, K, G * N, K, fp8q::BN)) != FP8Q_OK) return st;
+  fp8q::GemmArgs args{};
+  args.sfa = sfa;
+  args.ld_sfa = ld_sfa;
+  args.sfb = sfw;
+  args.ld_sfb = K / 128;
+  args.d = d;
+  args.ldd = ldd;
+  args.sfd = sfd;
+  args.ld_sfd = ld_sfd;
+  args.M = static_cast<int>(M_total);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
+  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
+  args.num_m_tiles = 0;
+  args.group_offsets = group_offsets;
+  args.G = static_cast<int>(G);
+  // upper bound on the device-side tile count: every expert wastes at most one partial m-tile
+  const int64_t bound = ((M_total + fp8q::BM - 1) / fp8q::BM + G) * args.num_n_tiles;
+  if (bound > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(bound < dev->sm_count ? bound : dev->sm_count);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return out == fp8q::kOutE4m3 ? launch_gemm<true, FP8Q_SFB_BLOCK128, fp8q::kOutE4m3>(dev, ta, tb, args, grid, s)
+                               : launch_gemm<true, FP8Q_SFB_BLOCK128, fp8q::kOutBf16>(dev, ta, tb, args, grid, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -257,7 +396,26 @@ fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ld
   const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel, fp8q::kQ1Threads, 0);
   const int64_t grid = grid_for(items, dev->sm_count, per_sm);
   fp8q::quant_act_1x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf);
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, nullptr, M);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K, int64_t ldx, const int32_t* rows,
+                                        int64_t M, void* q, int64_t ldq, float* sf, int64_t ld_sf, void* stream) {
+  if (M_src < 0 || M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || rows == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || !aligned(rows, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  fp8q::quant_act_1x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, rows, M_src);
   return launch_status();
 }
 
@@ -316,113 +474,31 @@ fp8q_status fp8q_quant_w_128x128(const void* w, int64_t N, int64_t K, int64_t ld
 fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* b,
                                   int64_t ldb, const float* sfb, int64_t ld_sfb, int sfb_mode, void* d, int64_t ldd,
                                   int d_dtype, int64_t M, int64_t N, int64_t K, void* stream) {
-  const int64_t kIntMax = 0x7FFFFFFF;
-  if (M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
-  if (M > kIntMax || N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
-  if (lda < K || ldb < K || ldd < N || ld_sfa < M) return FP8Q_ERR_INVALID_ARG;
-  if (sfb_mode != FP8Q_SFB_BLOCK128 && sfb_mode != FP8Q_SFB_ROW) return FP8Q_ERR_INVALID_ARG;
   if (d_dtype != FP8Q_OUT_BF16 && d_dtype != FP8Q_OUT_F32) return FP8Q_ERR_INVALID_ARG;
-  if (sfb_mode == FP8Q_SFB_BLOCK128 && ld_sfb < K / 128) return FP8Q_ERR_INVALID_ARG;
-  if (sfb_mode == FP8Q_SFB_ROW && ld_sfb < N) return FP8Q_ERR_INVALID_ARG;
-  if (a == nullptr || b == nullptr || sfa == nullptr || sfb == nullptr || d == nullptr) return FP8Q_ERR_INVALID_ARG;
-  const int64_t esz = d_dtype == FP8Q_OUT_F32 ? 4 : 2;
-  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfb, 4) ||
-      lda % 16 != 0 || ldb % 16 != 0 || (ldd * esz) % 16 != 0)
-    return FP8Q_ERR_ALIGNMENT;
-  if (sfb_mode == FP8Q_SFB_ROW && (!aligned(sfb, 16) || ld_sfb % 4 != 0)) return FP8Q_ERR_ALIGNMENT;
-  DeviceInfo* dev = nullptr;
-  fp8q_status st = device_info(&dev);
-  if (st != FP8Q_OK) return st;
-  const bool pair = use_pair_kernel(M, sfa, ld_sfa, sfb, ld_sfb);
-  CUtensorMap ta, tb, tsa, tsb;
-  if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
-  if ((st = make_tmap(&tb, b, K, N, ldb, pair ? fp8q::BN / 2 : fp8q::BN)) != FP8Q_OK) return st;
-  if (pair) {
-    // sa[K/128][ld_sfa]: 128 row scales per load
-    if ((st = make_tmap_f32(&tsa, sfa, M, K / 128, ld_sfa, fp8q::BM, 1)) != FP8Q_OK) return st;
-    // sb: [K/128][ld_sfb] per-column scales, 256 per load; or [N/128][ld_sfb]
-    // block scales, 4 chunks x the tile's 2 column blocks per load
-    st = sfb_mode == FP8Q_SFB_ROW ? make_tmap_f32(&tsb, sfb, N, K / 128, ld_sfb, fp8q::BN, 1)
-                                  : make_tmap_f32(&tsb, sfb, K / 128, N / 128, ld_sfb, 4, 2);
-    if (st != FP8Q_OK) return st;
-  }
-  fp8q::GemmArgs args{};
-  args.sfa = sfa;
-  args.ld_sfa = ld_sfa;
-  args.sfb = sfb;
-  args.ld_sfb = ld_sfb;
-  args.d = d;
-  args.ldd = ldd;
-  args.M = static_cast<int>(M);
-  args.N = static_cast<int>(N);
-  args.K = static_cast<int>(K);
-  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
-  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
-  args.num_m_tiles = static_cast<int>((M + fp8q::BM - 1) / fp8q::BM);
-  args.group_offsets = nullptr;
-  args.G = 1;
-  const int64_t tiles = static_cast<int64_t>(args.num_m_tiles) * args.num_n_tiles;
-  if (tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
-  const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (pair) {
-    const int64_t m_pairs = (M + 2 * fp8q::BM - 1) / (2 * fp8q::BM);
-    const int64_t pair_tiles = m_pairs * args.num_n_tiles;
-    args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
-    if (sfb_mode == FP8Q_SFB_BLOCK128)
-      return d_dtype == FP8Q_OUT_F32
-                 ? launch_gemm_pair<FP8Q_SFB_BLOCK128, true>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
-                 : launch_gemm_pair<FP8Q_SFB_BLOCK128, false>(dev, ta, tb, tsa, tsb, args, pair_tiles, s);
-    return d_dtype == FP8Q_OUT_F32 ? launch_gemm_pair<FP8Q_SFB_ROW, true>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
-                                   : launch_gemm_pair<FP8Q_SFB_ROW, false>(dev, ta, tb, tsa, tsb, args, pair_tiles, s);
-  }
-  if (sfb_mode == FP8Q_SFB_BLOCK128) {
-    return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_BLOCK128, true>(dev, ta, tb, args, grid, s)
-                                   : launch_gemm<false, FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, grid, s);
-  }
-  return d_dtype == FP8Q_OUT_F32 ? launch_gemm<false, FP8Q_SFB_ROW, true>(dev, ta, tb, args, grid, s)
-                                 : launch_gemm<false, FP8Q_SFB_ROW, false>(dev, ta, tb, args, grid, s);
+  return gemm_dense(a, lda, sfa, ld_sfa, b, ldb, sfb, ld_sfb, sfb_mode, d, ldd,
+                    d_dtype == FP8Q_OUT_F32 ? fp8q::kOutF32 : fp8q::kOutBf16, nullptr, 0, M, N, K, stream);
+}
+
+fp8q_status fp8q_gemm_blockscaled_q1x128(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* b,
+                                         int64_t ldb, const float* sfb, int64_t ld_sfb, void* dq, int64_t lddq,
+                                         float* sfd, int64_t ld_sfd, int64_t M, int64_t N, int64_t K, void* stream) {
+  return gemm_dense(a, lda, sfa, ld_sfa, b, ldb, sfb, ld_sfb, FP8Q_SFB_BLOCK128, dq, lddq, fp8q::kOutE4m3, sfd,
+                    ld_sfd, M, N, K, stream);
 }
 
 fp8q_status fp8q_grouped_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* w,
                                           const float* sfw, const int32_t* group_offsets, int64_t G, int64_t M_total,
                                           void* d, int64_t ldd, int64_t N, int64_t K, void* stream) {
-  const int64_t kIntMax = 0x7FFFFFFF;
-  if (G < 1 || M_total < 0 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
-  if (G > fp8q::kMaxGroups || M_total > kIntMax || G * N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
-  if (lda < K || ldd < N || ld_sfa < M_total) return FP8Q_ERR_INVALID_ARG;
-  if (M_total == 0) return FP8Q_OK;
-  if (a == nullptr || w == nullptr || sfa == nullptr || sfw == nullptr || group_offsets == nullptr || d == nullptr)
-    return FP8Q_ERR_INVALID_ARG;
-  if (!aligned(a, 16) || !aligned(w, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfw, 4) ||
-      !aligned(group_offsets, 4) || lda % 16 != 0 || (ldd * 2) % 16 != 0)
-    return FP8Q_ERR_ALIGNMENT;
-  DeviceInfo* dev = nullptr;
-  fp8q_status st = device_info(&dev);
-  if (st != FP8Q_OK) return st;
-  CUtensorMap ta, tb;
-  if ((st = make_tmap(&ta, a, K, M_total, lda, fp8q::BM)) != FP8Q_OK) return st;
-  if ((st = make_tmap(&tb, w, K, G * N, K, fp8q::BN)) != FP8Q_OK) return st;
-  fp8q::GemmArgs args{};
-  args.sfa = sfa;
-  args.ld_sfa = ld_sfa;
-  args.sfb = sfw;
-  args.ld_sfb = K / 128;
-  args.d = d;
-  args.ldd = ldd;
-  args.M = static_cast<int>(M_total);
-  args.N = static_cast<int>(N);
-  args.K = static_cast<int>(K);
-  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
-  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
-  args.num_m_tiles = 0;
-  args.group_offsets = group_offsets;
-  args.G = static_cast<int>(G);
-  // upper bound on the device-side tile count: every expert wastes at most one partial m-tile
-  const int64_t bound = ((M_total + fp8q::BM - 1) / fp8q::BM + G) * args.num_n_tiles;
-  if (bound > kIntMax) return FP8Q_ERR_UNSUPPORTED;
-  const int grid = static_cast<int>(bound < dev->sm_count ? bound : dev->sm_count);
-  return launch_gemm<true, FP8Q_SFB_BLOCK128, false>(dev, ta, tb, args, grid, static_cast<cudaStream_t>(stream));
+  return gemm_grouped(a, lda, sfa, ld_sfa, w, sfw, group_offsets, G, M_total, d, ldd, fp8q::kOutBf16, nullptr, 0, N, K,
+                      stream);
+}
+
+fp8q_status fp8q_grouped_gemm_blockscaled_q1x128(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                                 const void* w, const float* sfw, const int32_t* group_offsets,
+                                                 int64_t G, int64_t M_total, void* dq, int64_t lddq, float* sfd,
+                                                 int64_t ld_sfd, int64_t N, int64_t K, void* stream) {
+  return gemm_grouped(a, lda, sfa, ld_sfa, w, sfw, group_offsets, G, M_total, dq, lddq, fp8q::kOutE4m3, sfd, ld_sfd, N,
+                      K, stream);
 }
 
 fp8q_status fp8q_debug_cast_e4m3_bits(uint32_t start, int64_t count, void* out, void* stream) {

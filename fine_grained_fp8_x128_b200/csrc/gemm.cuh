@@ -40,6 +40,7 @@
 #pragma once
 
 #include "device_common.cuh"
+#include "quant.cuh"
 
 namespace fp8q {
 
@@ -79,8 +80,10 @@ struct GemmArgs {
   int64_t ld_sfa;
   const float* sfb;      // dense: per sfb_mode; grouped: sfw [G][N/128][K/128]
   int64_t ld_sfb;
-  void* d;
+  void* d;               // BF16 / FP32 output, or E4M3 codes (kOut == kOutE4m3)
   int64_t ldd;
+  float* sfd;            // kOut == kOutE4m3: scales of the output's 1x128 tiles, sfd[(n/128) * ld_sfd + m]
+  int64_t ld_sfd;
   int M;                 // dense: rows of A; grouped: M_total
   int N;
   int K;
@@ -140,6 +143,54 @@ __device__ __forceinline__ TileCoord tile_coord(int t, const GemmArgs& p, const 
   return c;
 }
 
+// Output modes of the GEMM kernels.
+constexpr int kOutBf16 = 0;   // round-to-nearest-even BF16
+constexpr int kOutF32 = 1;    // FP32
+constexpr int kOutE4m3 = 2;   // the next layer's operand: BF16-rounded rows quantized in 1x128 tiles
+
+// Store one thread's 128 consecutive outputs of row `row`, columns ncol0 ..
+// ncol0 + 127 (ncol0 a multiple of 128).  In kOutE4m3 mode the 128 values are
+// one 1x128 tile: they are rounded to BF16 and quantized exactly as
+// quant_act_1x128_kernel quantizes a BF16 row ("Fine-Grained FP8 Quantization
+// in DeepSeek", section 2: per-tile amax, s = amax/448, E4M3 cast), so the
+// result equals quantizing the BF16 output -- without writing or re-reading it.
+template <int kOut>
+__device__ __forceinline__ void store_row128(const float* acc, int row, int ncol0, const GemmArgs& p) {
+  if (kOut == kOutF32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+  } else {
+    uint32_t w[64];   // BF16 pairs
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    if (kOut == kOutBf16) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    } else {
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) m = amax_word(m, w[j]);
+      const float s = tile_scale(m);
+      const float r = __frcp_rn(s);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint32_t c[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          c[j] = quant_word(w[8 * i + 2 * j], r, s) | (quant_word(w[8 * i + 2 * j + 1], r, s) << 16);
+        dst[i] = make_uint4(c[0], c[1], c[2], c[3]);
+      }
+      p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row] = s;
+    }
+  }
+}
+
 __device__ __forceinline__ void setmaxnreg_inc232() { asm volatile("setmaxnreg.inc.sync.aligned.u32 232;"); }
 __device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.dec.sync.aligned.u32 40;"); }
 
@@ -168,7 +219,7 @@ __device__ __forceinline__ void promote64_rows(float* acc, const uint32_t (&v)[6
   }
 }
 
-template <bool kGrouped, int kSfbMode, bool kOutF32>
+template <bool kGrouped, int kSfbMode, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const GemmArgs p) {
@@ -382,25 +433,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         }
       }
       if (!ok) break;
-      if (vrow && vcol) {
-        if (kOutF32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * i + 2 * j], acc[8 * i + 2 * j + 1]);
-              w[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      }
+      if (vrow && vcol) store_row128<kOut>(acc, row, ncol0, p);
     }
   }
 

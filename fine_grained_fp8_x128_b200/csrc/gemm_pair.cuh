@@ -87,7 +87,7 @@ __device__ __forceinline__ void promote_rows16(float* acc, const uint32_t (&v)[6
   }
 }
 
-template <int kSfbMode, bool kOutF32>
+template <int kSfbMode, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
@@ -280,7 +280,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
               for (int k = 0; k < 16; ++k) {   // k < 8: first 64 columns, k >= 8: second
                 const int x = 64 * (k >> 3) + 32 * g + 4 * (k & 7) + 2 * i;
                 const float x0 = acc[x], x1 = acc[x + 1];
-                if (kOutF32) {
+                if (kOut == kOutF32) {
                   *reinterpret_cast<float2*>(static_cast<float*>(p.d) + base + 8 * k) = make_float2(x0, x1);
                 } else {
                   const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
@@ -291,23 +291,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           }
         }
       } else if (vrow && vcol) {
-        if (kOutF32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(acc[8 * i + 2 * j], acc[8 * i + 2 * j + 1]);
-              w[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+        store_row128<kOut>(acc, row, ncol0, p);
       }
     }
   }

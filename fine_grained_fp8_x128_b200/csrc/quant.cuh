@@ -32,6 +32,9 @@ __device__ __forceinline__ uint32_t quant_word(uint32_t w, float r, float s) {
 // covers 64 tiles: rows r0..r0+63 of one 128-column chunk kb, so the 64 scales
 // it writes, sf[kb*ld_sf + r0 ..], are contiguous.  The loads of the block's
 // next grid-stride item are issued before the current item is cast.
+// With a row map (rows != nullptr) output row m is the quantization of source
+// row rows[m] -- the gather of MoE dispatch fused into the quantizer; an index
+// outside [0, M_src) gives the all-zero tile and records FP8Q_ERR_INVALID_ARG.
 // ---------------------------------------------------------------------------
 constexpr int kQ1Threads = 256;
 constexpr int kQ1Rows = 64;
@@ -41,12 +44,21 @@ struct Q1Slice {
 };
 
 __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB,
-                                        int64_t ldx, int64_t it, int tile, int sub) {
+                                        int64_t ldx, const int32_t* __restrict__ rows, int64_t M_src, int64_t it,
+                                        int tile, int sub) {
   const int64_t rb = it / KB;
   const int64_t kb = it - rb * KB;
   const int64_t row = rb * kQ1Rows + tile;
-  if (row < M) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + row * ldx + kb * 128 + sub * 8);
+  int64_t src_row = row;
+  if (rows != nullptr && row < M) {
+    src_row = __ldg(rows + row);
+    if (src_row < 0 || src_row >= M_src) {
+      if (sub == 0 && kb == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_ROW_INDEX);
+      src_row = -1;
+    }
+  }
+  if (row < M && src_row >= 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + src_row * ldx + kb * 128 + sub * 8);
 #pragma unroll
     for (int i = 0; i < 4; ++i) d.v[i] = __ldcs(src + 4 * i);
   } else {
@@ -57,7 +69,8 @@ __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restr
 
 __global__ void __launch_bounds__(kQ1Threads)
 quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
-                       uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf) {
+                       uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
+                       const int32_t* __restrict__ rows, int64_t M_src) {
   const int tid = threadIdx.x;
   const int sub = tid & 3;           // 32-element slice within the tile
   const int tile = tid >> 2;         // 0..63: row within the block's 64 rows
@@ -66,10 +79,10 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
   int64_t it = blockIdx.x;
   if (it >= items) return;
   Q1Slice cur, nxt;
-  q1_load(cur, x, M, KB, ldx, it, tile, sub);
+  q1_load(cur, x, M, KB, ldx, rows, M_src, it, tile, sub);
   for (; it < items; it += gridDim.x) {
     const int64_t it_next = it + gridDim.x;
-    if (it_next < items) q1_load(nxt, x, M, KB, ldx, it_next, tile, sub);
+    if (it_next < items) q1_load(nxt, x, M, KB, ldx, rows, M_src, it_next, tile, sub);
     const int64_t rb = it / KB;
     const int64_t kb = it - rb * KB;
     const int64_t row = rb * kQ1Rows + tile;

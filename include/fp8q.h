@@ -94,6 +94,28 @@ fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ld
                                  void* stream);
 
 /*
+ * fp8q_quant_act_1x128 over a row gather: output row m quantizes input row
+ * rows[m] of x.  This is the MoE dispatch's permutation (tokens copied to the
+ * rows of their experts, one copy per routed expert) fused into the online
+ * quantization, so the permuted BF16 activations never exist in HBM ("FP8
+ * Mixed Precision: DeepSeek-V3 Training Architecture", section 2 "The MoE
+ * Inter-Node All-to-All Communication Wall": dispatch activations travel in
+ * FP8; "Fine-Grained FP8 Quantization in DeepSeek", section 2).
+ *
+ *   x    : BF16 [M_src][ldx] (source tokens).
+ *   rows : device int32 [M]; each in [0, M_src).  An index outside that
+ *          range makes the output row's tiles quantize zeros (q = 0,
+ *          sf = 1e-12) and records FP8Q_ERR_INVALID_ARG in the device status
+ *          word (read with fp8q_device_status).
+ *   q, sf: as fp8q_quant_act_1x128 with M output rows.
+ * Requirements: as fp8q_quant_act_1x128 plus M_src >= 0, rows 4-byte aligned.
+ */
+fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K, int64_t ldx,
+                                        const int32_t* rows, int64_t M,
+                                        void* q, int64_t ldq, float* sf, int64_t ld_sf,
+                                        void* stream);
+
+/*
  * Online 128x1 quantization along the token dimension, written transposed:
  * the layout both Wgrad operands need (dL/dW = x^T (dL/dz), "Introduction to
  * LLM Quantization", "3) Backward propagation"; "Fine-Grained FP8 Quantization
@@ -158,6 +180,25 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
                                   int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * fp8q_gemm_blockscaled (FP8Q_SFB_BLOCK128) whose output is the next layer's
+ * FP8 input: the epilogue rounds each FP32 result to BF16, then quantizes
+ * every 1x128 tile of the row exactly as fp8q_quant_act_1x128 does on that
+ * BF16 row.  The result equals fp8q_gemm_blockscaled (BF16 out) followed by
+ * fp8q_quant_act_1x128, bit for bit, without the BF16 round trip through HBM
+ * ("Fine-Grained FP8 Quantization in DeepSeek", section 2: activations are
+ * quantized online per 1x128 tile; "FP8 Mixed Precision: DeepSeek-V3 Training
+ * Architecture", section 1: activations cached in FP8 for the next layer).
+ *
+ *   dq  : E4M3 [M][lddq].   sfd : FP32 sfd[(n/128) * ld_sfd + m], ld_sfd >= M.
+ * Requirements: as fp8q_gemm_blockscaled with FP8Q_SFB_BLOCK128, plus
+ * dq 16-byte aligned, lddq % 16 == 0, sfd 4-byte aligned.
+ */
+fp8q_status fp8q_gemm_blockscaled_q1x128(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                         const void* b, int64_t ldb, const float* sfb, int64_t ld_sfb,
+                                         void* dq, int64_t lddq, float* sfd, int64_t ld_sfd,
+                                         int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
  * Grouped (MoE expert) block-scaled FP8 GEMM.  For each expert g, rows
  * [off[g], off[g+1]) of the expert-packed activations are multiplied by that
  * expert's 128x128-block weight, with the semantics of fp8q_gemm_blockscaled
@@ -182,6 +223,22 @@ fp8q_status fp8q_grouped_gemm_blockscaled(const void* a, int64_t lda, const floa
                                           const int32_t* group_offsets, int64_t G, int64_t M_total,
                                           void* d, int64_t ldd, int64_t N, int64_t K,
                                           void* stream);
+
+/*
+ * fp8q_grouped_gemm_blockscaled with the FP8 output of
+ * fp8q_gemm_blockscaled_q1x128: each expert's rows come out as E4M3 1x128
+ * tiles plus their scales, ready to be operand A of the next expert GEMM.
+ *
+ *   dq  : E4M3 [M_total][lddq].   sfd : FP32 sfd[(n/128) * ld_sfd + m],
+ *         ld_sfd >= M_total.
+ * Requirements: as fp8q_grouped_gemm_blockscaled plus dq 16-byte aligned,
+ * lddq % 16 == 0, sfd 4-byte aligned.
+ */
+fp8q_status fp8q_grouped_gemm_blockscaled_q1x128(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                                 const void* w, const float* sfw,
+                                                 const int32_t* group_offsets, int64_t G, int64_t M_total,
+                                                 void* dq, int64_t lddq, float* sfd, int64_t ld_sfd,
+                                                 int64_t N, int64_t K, void* stream);
 
 /* ---- diagnostics (used by the test suite; not on the hot path) ---------- */
 

@@ -66,6 +66,20 @@ def test_quant_act_validation(fp8q):
     assert L.fp8q_quant_act_128x1(None, 0, 8, 8, None, 0, None, 8, None) == 0
 
 
+def test_quant_gather_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+
+    def qg(x=FAKE, Ms=16, K=256, ldx=256, rows=FAKE, M=8, q=FAKE, ldq=256, sf=FAKE, ld_sf=8):
+        return L.fp8q_quant_act_1x128_gather(x, Ms, K, ldx, rows, M, q, ldq, sf, ld_sf, None)
+
+    assert qg(Ms=-1) == INV and qg(M=-1) == INV and qg(K=200) == INV
+    assert qg(ldx=128) == INV and qg(ldq=128) == INV and qg(ld_sf=4) == INV
+    assert qg(rows=None) == INV and qg(x=None) == INV
+    assert qg(rows=FAKE + 2) == ALN and qg(x=FAKE + 8) == ALN and qg(ldq=264) == ALN
+    assert qg(M=0, rows=None, q=None, sf=None, ld_sf=0) == 0    # no output rows: nothing launched
+
+
 def test_quant_w_validation(fp8q):
     L = fp8q.lib()
     INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
@@ -97,6 +111,28 @@ def test_gemm_validation(fp8q):
     assert g(mode=ROW, ld_sfb=258) == ALN          # row-mode scales are bulk-copied: ld % 4
     assert g(sfa=FAKE + 2) == ALN
     assert g(a=None) == INV
+
+
+def test_gemm_q1x128_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+
+    def gq(M=8, N=256, K=256, ldd=256, sfd=FAKE, ld_sfd=8, d=FAKE, ld_sfb=2):
+        return L.fp8q_gemm_blockscaled_q1x128(FAKE, K, FAKE, 8, FAKE, K, FAKE, ld_sfb, d, ldd, sfd, ld_sfd, M, N, K,
+                                              None)
+
+    assert gq(M=0) == INV and gq(N=200) == INV and gq(ldd=128) == INV
+    assert gq(ld_sfd=4) == INV and gq(sfd=None) == INV and gq(ld_sfb=1) == INV
+    assert gq(ldd=264) == ALN                       # FP8 rows: ld % 16
+    assert gq(sfd=FAKE + 2) == ALN and gq(d=FAKE + 8) == ALN
+
+    def ggq(G=4, Mt=64, ldd=256, sfd=FAKE, ld_sfd=64):
+        return L.fp8q_grouped_gemm_blockscaled_q1x128(FAKE, 256, FAKE, 64, FAKE, FAKE, FAKE, G, Mt, FAKE, ldd, sfd,
+                                                      ld_sfd, 256, 256, None)
+
+    assert ggq(G=0) == INV and ggq(ld_sfd=32) == INV and ggq(sfd=None) == INV and ggq(ldd=128) == INV
+    assert ggq(ldd=264) == ALN and ggq(sfd=FAKE + 1) == ALN
+    assert ggq(Mt=0, sfd=None, ld_sfd=0) == 0
 
 
 def test_grouped_validation(fp8q):
