@@ -712,7 +712,7 @@ def run_single(args):
         else:
             K, N = (MOE_FF, HID) if name == "moe_down" else (HID, MOE_FF)
             qa, sa = fp8q.quant_act_1x128(randn(mt, K))
-            wq = torch.randint(0, 0x7E, (MOE_E, N, K), generator=gen, device=dev, dtype=torch.int32).to(u8)
+            wq = torch.randint(0, 0x7E, (MOE_E, N, K), generator=gen, device=dev, dtype=u8)
             ws = torch.rand((MOE_E, N // 128, K // 128), generator=gen, device=dev) * 1e-3
             off = torch.from_numpy(route.offsets.astype(np.int32)).to(dev)
             if name == "moe_up_q":

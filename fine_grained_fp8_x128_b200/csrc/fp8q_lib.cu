@@ -31,6 +31,7 @@ struct DeviceInfo {
   bool pair_attr[2][3] = {};       // [row mode][output mode]
   int pair_clusters[2][3] = {};    // co-resident CTA pairs per kernel instance
   int q1_per_sm = 0;               // resident blocks per SM of each quantizer
+  int q1g_per_sm = 0;
   int q2_per_sm = 0;
   int qw_per_sm = 0;
 };
@@ -393,9 +394,9 @@ fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ld
   if (st != FP8Q_OK) return st;
   const int64_t KB = K / 128;
   const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
-  const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel, fp8q::kQ1Threads, 0);
+  const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel<false>, fp8q::kQ1Threads, 0);
   const int64_t grid = grid_for(items, dev->sm_count, per_sm);
-  fp8q::quant_act_1x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  fp8q::quant_act_1x128_kernel<false><<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, nullptr, M);
   return launch_status();
 }
@@ -412,9 +413,9 @@ fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K,
   if (st != FP8Q_OK) return st;
   const int64_t KB = K / 128;
   const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
-  const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel, fp8q::kQ1Threads, 0);
+  const int per_sm = blocks_per_sm(&dev->q1g_per_sm, fp8q::quant_act_1x128_kernel<true>, fp8q::kQ1Threads, 0);
   const int64_t grid = grid_for(items, dev->sm_count, per_sm);
-  fp8q::quant_act_1x128_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  fp8q::quant_act_1x128_kernel<true><<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, rows, M_src);
   return launch_status();
 }

@@ -172,18 +172,17 @@ __device__ __forceinline__ void store_row128(const float* acc, int row, int ncol
 #pragma unroll
       for (int i = 0; i < 16; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
     } else {
-      float m = 0.0f;
+      uint32_t m2 = 0;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) m = amax_word(m, w[j]);
-      const float s = tile_scale(m);
-      const float r = __frcp_rn(s);
+      for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
+      const float s = tile_scale(amax2_value(m2));
+      const float nr = -__frcp_rn(s);
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         uint32_t c[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          c[j] = quant_word(w[8 * i + 2 * j], r, s) | (quant_word(w[8 * i + 2 * j + 1], r, s) << 16);
+        for (int j = 0; j < 4; ++j) c[j] = quant_words(w[8 * i + 2 * j], w[8 * i + 2 * j + 1], nr, s);
         dst[i] = make_uint4(c[0], c[1], c[2], c[3]);
       }
       p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row] = s;

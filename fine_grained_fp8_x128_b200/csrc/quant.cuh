@@ -15,13 +15,24 @@ namespace fp8q {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ float amax_word(float m, uint32_t w) {
-  return fmaxf(m, fmaxf(fabsf(bf16lo(w)), fabsf(bf16hi(w))));
+// Lane-wise maximum magnitude of BF16 pairs.  For finite BF16 values |a| <= |b|
+// exactly when their 15 low bits compare that way as unsigned integers, so one
+// 16x2 integer max per word keeps both lanes' running maxima (m starts at 0).
+__device__ __forceinline__ uint32_t amax2(uint32_t m, uint32_t w) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(w & 0x7FFF7FFFu));
+  return r;
 }
+__device__ __forceinline__ float amax2_value(uint32_t m) { return fmaxf(bf16lo(m), bf16hi(m)); }
 
-// Two BF16 values (one word) -> two E4M3 codes (low byte first).
-__device__ __forceinline__ uint32_t quant_word(uint32_t w, float r, float s) {
-  return cvt_e4m3x2(scaled_for_cast(bf16lo(w), r, s), scaled_for_cast(bf16hi(w), r, s));
+// Four BF16 values (two words) -> four E4M3 codes, one byte each in element
+// order: q = e4m3(fl32(x / s)), with nr = -fl32(1/s) (see e4m3x2_neg_quot,
+// which returns the codes with inverted signs; one XOR flips all four back).
+constexpr uint32_t kFlipSigns = 0x80808080u;
+__device__ __forceinline__ uint32_t quant_words(uint32_t w0, uint32_t w1, float nr, float s) {
+  const uint32_t c0 = e4m3x2_neg_quot(bf16lo(w0), bf16hi(w0), nr, nr, s, s);
+  const uint32_t c1 = e4m3x2_neg_quot(bf16lo(w1), bf16hi(w1), nr, nr, s, s);
+  return (c0 | (c1 << 16)) ^ kFlipSigns;
 }
 
 // ---------------------------------------------------------------------------
@@ -43,6 +54,7 @@ struct Q1Slice {
   uint4 v[4];
 };
 
+template <bool kGather>
 __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB,
                                         int64_t ldx, const int32_t* __restrict__ rows, int64_t M_src, int64_t it,
                                         int tile, int sub) {
@@ -50,7 +62,7 @@ __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restr
   const int64_t kb = it - rb * KB;
   const int64_t row = rb * kQ1Rows + tile;
   int64_t src_row = row;
-  if (rows != nullptr && row < M) {
+  if (kGather && row < M) {
     src_row = __ldg(rows + row);
     if (src_row < 0 || src_row >= M_src) {
       if (sub == 0 && kb == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_ROW_INDEX);
@@ -59,14 +71,22 @@ __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restr
   }
   if (row < M && src_row >= 0) {
     const uint4* src = reinterpret_cast<const uint4*>(x + src_row * ldx + kb * 128 + sub * 8);
+    if (kGather) {
+      // a source row is read once per output row that maps to it: default
+      // caching keeps the rows in the L2 between their reads
 #pragma unroll
-    for (int i = 0; i < 4; ++i) d.v[i] = __ldcs(src + 4 * i);
+      for (int i = 0; i < 4; ++i) d.v[i] = __ldg(src + 4 * i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d.v[i] = __ldcs(src + 4 * i);
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) d.v[i] = make_uint4(0, 0, 0, 0);
   }
 }
 
+template <bool kGather>
 __global__ void __launch_bounds__(kQ1Threads)
 quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
                        uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
@@ -79,31 +99,35 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
   int64_t it = blockIdx.x;
   if (it >= items) return;
   Q1Slice cur, nxt;
-  q1_load(cur, x, M, KB, ldx, rows, M_src, it, tile, sub);
+  q1_load<kGather>(cur, x, M, KB, ldx, rows, M_src, it, tile, sub);
   for (; it < items; it += gridDim.x) {
     const int64_t it_next = it + gridDim.x;
-    if (it_next < items) q1_load(nxt, x, M, KB, ldx, rows, M_src, it_next, tile, sub);
+    if (it_next < items) q1_load<kGather>(nxt, x, M, KB, ldx, rows, M_src, it_next, tile, sub);
     const int64_t rb = it / KB;
     const int64_t kb = it - rb * KB;
     const int64_t row = rb * kQ1Rows + tile;
-    float m = 0.0f;
+    uint32_t m2 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      m = amax_word(m, cur.v[i].x); m = amax_word(m, cur.v[i].y);
-      m = amax_word(m, cur.v[i].z); m = amax_word(m, cur.v[i].w);
+      m2 = amax2(m2, cur.v[i].x); m2 = amax2(m2, cur.v[i].y);
+      m2 = amax2(m2, cur.v[i].z); m2 = amax2(m2, cur.v[i].w);
     }
+    float m = amax2_value(m2);
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     const float s = tile_scale(m);
-    const float r = __frcp_rn(s);
+    const float nr = -__frcp_rn(s);
     if (row < M) {
       uint8_t* dst = q + row * ldq + kb * 128 + sub * 8;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint2 o;
-        o.x = quant_word(cur.v[i].x, r, s) | (quant_word(cur.v[i].y, r, s) << 16);
-        o.y = quant_word(cur.v[i].z, r, s) | (quant_word(cur.v[i].w, r, s) << 16);
-        *reinterpret_cast<uint2*>(dst + 32 * i) = o;
+        o.x = quant_words(cur.v[i].x, cur.v[i].y, nr, s);
+        o.y = quant_words(cur.v[i].z, cur.v[i].w, nr, s);
+        if (kGather)
+          __stcs(reinterpret_cast<uint2*>(dst + 32 * i), o);   // evict-first: leave the L2 to the source rows
+        else
+          *reinterpret_cast<uint2*>(dst + 32 * i) = o;
       }
       if (sub == 0) sf[kb * ld_sf + row] = s;
     }
@@ -173,12 +197,11 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
     const bool active = 2 * p < ncols;
     float ma = 0.0f, mb = 0.0f;
     if (active) {
+      uint32_t m2 = 0;   // channel 2p in the low half, 2p+1 in the high half
 #pragma unroll 8
-      for (int t = 32 * r; t < 32 * r + 32; ++t) {
-        const uint32_t w = tile[t * kWords + p];
-        ma = fmaxf(ma, fabsf(bf16lo(w)));
-        mb = fmaxf(mb, fabsf(bf16hi(w)));
-      }
+      for (int t = 32 * r; t < 32 * r + 32; ++t) m2 = amax2(m2, tile[t * kWords + p]);
+      ma = bf16lo(m2);
+      mb = bf16hi(m2);
     }
     qmax[r * kQTCols + 2 * p] = ma;
     qmax[r * kQTCols + 2 * p + 1] = mb;
@@ -188,7 +211,7 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
       mb = fmaxf(fmaxf(qmax[2 * p + 1], qmax[kQTCols + 2 * p + 1]),
                  fmaxf(qmax[2 * kQTCols + 2 * p + 1], qmax[3 * kQTCols + 2 * p + 1]));
       const float sa = tile_scale(ma), sb = tile_scale(mb);
-      const float ra = __frcp_rn(sa), rb = __frcp_rn(sb);
+      const float nra = -__frcp_rn(sa), nrb = -__frcp_rn(sb);
       const int64_t ca = c0 + 2 * p;
       uint8_t* qa = qt + ca * ldqt + tb * 128 + 32 * r;
       uint8_t* qb = qa + ldqt;
@@ -203,11 +226,11 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
             const int t = 32 * r + 16 * h + 4 * j + 2 * e;
             const uint32_t w0 = tile[t * kWords + p];
             const uint32_t w1 = tile[(t + 1) * kWords + p];
-            a4 |= cvt_e4m3x2(scaled_for_cast(bf16lo(w0), ra, sa), scaled_for_cast(bf16lo(w1), ra, sa)) << (16 * e);
-            b4 |= cvt_e4m3x2(scaled_for_cast(bf16hi(w0), rb, sb), scaled_for_cast(bf16hi(w1), rb, sb)) << (16 * e);
+            a4 |= e4m3x2_neg_quot(bf16lo(w0), bf16lo(w1), nra, nra, sa, sa) << (16 * e);
+            b4 |= e4m3x2_neg_quot(bf16hi(w0), bf16hi(w1), nrb, nrb, sb, sb) << (16 * e);
           }
-          oa[j] = a4;
-          ob[j] = b4;
+          oa[j] = a4 ^ kFlipSigns;
+          ob[j] = b4 ^ kFlipSigns;
         }
         *reinterpret_cast<uint4*>(qa + 16 * h) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
         *reinterpret_cast<uint4*>(qb + 16 * h) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
@@ -261,12 +284,13 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       v[i] = __ldg(reinterpret_cast<const uint4*>(w + (n0 + 8 * a + i) * ldw + k0 + 8 * b));
-    float m = 0.0f;
+    uint32_t m2 = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      m = amax_word(m, v[i].x); m = amax_word(m, v[i].y);
-      m = amax_word(m, v[i].z); m = amax_word(m, v[i].w);
+      m2 = amax2(m2, v[i].x); m2 = amax2(m2, v[i].y);
+      m2 = amax2(m2, v[i].z); m2 = amax2(m2, v[i].w);
     }
+    float m = amax2_value(m2);
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((tid & 31) == 0) warp_max[tid >> 5] = m;
@@ -275,12 +299,12 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
 #pragma unroll
     for (int i = 1; i < kQWThreads / 32; ++i) m = fmaxf(m, warp_max[i]);
     const float s = tile_scale(m);
-    const float r = __frcp_rn(s);
+    const float nr = -__frcp_rn(s);
     uint32_t lo[8], hi[8];   // row i: bytes of columns 0-3 (lo) and 4-7 (hi)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      lo[i] = quant_word(v[i].x, r, s) | (quant_word(v[i].y, r, s) << 16);
-      hi[i] = quant_word(v[i].z, r, s) | (quant_word(v[i].w, r, s) << 16);
+      lo[i] = quant_words(v[i].x, v[i].y, nr, s);
+      hi[i] = quant_words(v[i].z, v[i].w, nr, s);
       *reinterpret_cast<uint2*>(q + (n0 + 8 * a + i) * ldq + k0 + 8 * b) = make_uint2(lo[i], hi[i]);
     }
     if (qt != nullptr) {

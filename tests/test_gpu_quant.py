@@ -245,3 +245,49 @@ def test_device_cast_matches_oracle_encoder_all_fp32(fp8q):
             bad = np.nonzero(~ok)[0][:8]
             raise AssertionError([(hex(int(bits[i])), float(x[i]), int(dev[i]), int(ref[i])) for i in bad])
     assert fp8q.fp8q_device_status() == 0
+
+
+def _amax_sweep(n_random=384, seed=0):
+    """Rows of 128 BF16 values; each row holds a tile maximum amax first and
+    then BF16 inputs with |x| <= amax.  For every amax sampled (all-zero tiles,
+    the smallest subnormal, the largest finite value, 448, powers of two and a
+    seeded sample of the rest) the rows cover EVERY BF16 x with |x| <= amax,
+    both signs and both zeros.  Rows of one amax are padded to a multiple of
+    128 so that 128x128 blocks and 128-token columns share it as well."""
+    rng = np.random.default_rng(seed)
+    specials = [0x0000, 0x0001, 0x007F, 0x0080, 0x3F80, 0x43E0, 0x43E1, 0x7F7F, 0x0100, 0x2000, 0x5F00]
+    picks = np.unique(np.concatenate([np.array(specials), rng.integers(1, 0x7F80, n_random)])).astype(np.uint32)
+    blocks = []
+    for ab in picks:
+        mags = np.arange(ab + 1, dtype=np.uint32)
+        xs = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)
+        rows = -(-xs.size // 127)
+        rows = -(-rows // 128) * 128
+        body = np.zeros(rows * 127, np.uint16)
+        body[:xs.size] = xs
+        blk = np.empty((rows, 128), np.uint16)
+        blk[:, 0] = ab
+        blk[:, 1:] = body.reshape(rows, 127)
+        blocks.append(blk)
+    return np.concatenate(blocks, axis=0)
+
+
+def test_quantizers_every_input_under_sampled_tile_maxima(fp8q):
+    """The division-free cast on the device: all three quantizers equal the
+    oracle's IEEE-quotient codes for every BF16 input under each sampled tile
+    maximum."""
+    x = _amax_sweep()
+    R = x.shape[0]
+    oq, osf = oracle.quant_act_1x128(x)
+    q, sf = run_q1(fp8q, x)
+    assert np.array_equal(sf.view(np.uint32), osf.view(np.uint32))
+    assert np.array_equal(q, oq)
+    # the same tiles as 128-token columns: x^T is [128 tokens][R channels]
+    qt, sft = run_qt(fp8q, np.ascontiguousarray(x.T))
+    assert np.array_equal(qt, oq) and np.array_equal(sft[0], osf[:, 0])
+    # and as 128x128 blocks (each block's rows share one maximum)
+    wq, wsf = run_qw(fp8q, x, transposed=False)
+    owq, owsf = oracle.quant_w_128x128(x)
+    assert np.array_equal(wsf, owsf) and np.array_equal(wq, owq)
+    assert np.array_equal(wq, oq)       # every block's maximum is its rows' maximum
+    assert R > 100000
