@@ -239,22 +239,13 @@ __device__ __forceinline__ void tmem_ld_wait_tied(uint32_t (&r)[32]) {
                : "memory");
 }
 
-// Packed FP32 pair arithmetic (sm_100a): two IEEE round-to-nearest FMAs /
-// products in one instruction; each lane is bit-identical to fmaf / __fmul_rn.
-__device__ __forceinline__ void fma2(float& a0, float& a1, float x0, float x1, float s0, float s1) {
-  asm("{\n\t.reg .b64 ra, rx, rs;\n\t"
-      "mov.b64 ra, {%0, %1};\n\tmov.b64 rx, {%2, %3};\n\tmov.b64 rs, {%4, %5};\n\t"
-      "fma.rn.f32x2 ra, rx, rs, ra;\n\tmov.b64 {%0, %1}, ra;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(x0), "f"(x1), "f"(s0), "f"(s1));
-}
-__device__ __forceinline__ void mul2(float& d0, float& d1, float x0, float x1, float s0, float s1) {
-  asm("{\n\t.reg .b64 rd, rx, rs;\n\t"
-      "mov.b64 rx, {%2, %3};\n\tmov.b64 rs, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, rx, rs;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(x0), "f"(x1), "f"(s0), "f"(s1));
-}
+// Packed FP32 pair arithmetic (sm_100a, f32x2): two IEEE round-to-nearest
+// FMAs / products in one instruction; each lane is bit-identical to fmaf /
+// __fmul_rn.  float2 operands keep the pairs in aligned register pairs.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
+__device__ __forceinline__ float2 f2u(uint32_t lo, uint32_t hi) { return make_float2(__uint_as_float(lo), __uint_as_float(hi)); }
 
 // ---------------------------------------------------------------------------
 // E4M3 conversion: round-to-nearest-even with saturation to +-448 (the PTX
@@ -285,13 +276,11 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
 // s = max(fl32(amax/448), fl32(1e-12)) -- about 1.07e9 pairs, no mismatch.
 // All three steps run as packed FP32x2 operations.
 __device__ __forceinline__ uint32_t e4m3x2_neg_quot(float x0, float x1, float nr0, float nr1, float s0, float s1) {
-  float n0, n1;
-  mul2(n0, n1, x0, x1, nr0, nr1);
-  float e0 = x0, e1 = x1;
-  fma2(e0, e1, n0, n1, s0, s1);
-  float t0 = n0, t1 = n1;
-  fma2(t0, t1, e0, e1, nr0, nr1);
-  return cvt_e4m3x2(t0, t1);
+  const float2 x = make_float2(x0, x1), nr = make_float2(nr0, nr1);
+  const float2 n = fmul2(x, nr);
+  const float2 e = ffma2(n, make_float2(s0, s1), x);
+  const float2 t = ffma2(e, nr, n);
+  return cvt_e4m3x2(t.x, t.y);
 }
 
 // Tile scale s = max(fl32(amax / 448), fl32(1e-12)).
@@ -421,6 +410,29 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8x2_sync(uint32_t taddr, uint32
       "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr), "r"(taddr + (16u << 16))
+      : "memory");
+}
+
+// 32 lanes x 32 columns, waited for inside the same asm statement.
+__device__ __forceinline__ void tmem_ld_32x32b_x32_sync(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 16x256b fragments of 32 lanes x 32 columns: lanes +0..15 (r[0..15]) and
+// +16..31 (r[16..31]) of the warp's quadrant, 4 column groups of 8 each;
+// r[16g + 4k + 2i + j] is row 16g + 8i + lane/4, column 8k + 2*(lane%4) + j.
+__device__ __forceinline__ void tmem_ld_16x256b_x4x2_sync(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr), "r"(taddr + (16u << 16))
       : "memory");
 }

@@ -58,7 +58,7 @@ constexpr uint32_t kABytes = BM * BK;               // 16 KB
 constexpr uint32_t kBBytes = BN * BK;               // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes; // 48 KB
 constexpr uint32_t kSbBytes = BN * 4;               // 1 KB
-constexpr int kMaxGroups = 2048;
+constexpr int kMaxGroups = 1024;
 constexpr int kGroupM = 16;                          // L2 swizzle: m-tiles per group
 
 struct GemmSmemLayout {
@@ -69,7 +69,8 @@ struct GemmSmemLayout {
   // barriers: go[S], done[S], sbfull[R], sbempty[R]
   static constexpr uint32_t nbars = 2 * kStages + 2 * kSbRing;
   static constexpr uint32_t misc = bars + nbars * 8;           // tmem base, abort flag
-  static constexpr uint32_t prefix = misc + 16;                // grouped: tile prefix [G+1]
+  static constexpr uint32_t out_stage = misc + 16;             // 8 epilogue warps x 2 KB (staged stores)
+  static constexpr uint32_t prefix = out_stage + 8 * 2048;     // grouped: tile prefix [G+1]
   static constexpr uint32_t offs = prefix + (kMaxGroups + 1) * 4;  // grouped: clamped offsets [G+1]
   static constexpr uint32_t bytes_dense = prefix;
   static constexpr uint32_t bytes_grouped = offs + (kMaxGroups + 1) * 4;
@@ -148,44 +149,162 @@ constexpr int kOutBf16 = 0;   // round-to-nearest-even BF16
 constexpr int kOutF32 = 1;    // FP32
 constexpr int kOutE4m3 = 2;   // the next layer's operand: BF16-rounded rows quantized in 1x128 tiles
 
-// Store one thread's 128 consecutive outputs of row `row`, columns ncol0 ..
-// ncol0 + 127 (ncol0 a multiple of 128).  In kOutE4m3 mode the 128 values are
-// one 1x128 tile: they are rounded to BF16 and quantized exactly as
-// quant_act_1x128_kernel quantizes a BF16 row ("Fine-Grained FP8 Quantization
-// in DeepSeek", section 2: per-tile amax, s = amax/448, E4M3 cast), so the
-// result equals quantizing the BF16 output -- without writing or re-reading it.
-template <int kOut>
-__device__ __forceinline__ void store_row128(const float* acc, int row, int ncol0, const GemmArgs& p) {
-  if (kOut == kOutF32) {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+// One pass of a warp's staged store: lane l brings 8 16-byte chunks of row l
+// (128 consecutive bytes of its output row); they go through the warp's 4 KB
+// shared buffer -- chunk j of row r at chunk slot j ^ (r & 7), so each group
+// of 8 lanes covers all 32 banks on the way in and on the way out -- and leave
+// as 16-byte global stores in which the warp covers 4 whole 128-byte row
+// segments at a time (instead of 32 scattered 16-byte pieces).  Rows at or
+// past rows_valid are not written.  Every lane of the warp takes part.
+__device__ __forceinline__ void stage_store_pass(uint4* stage, const uint4 (&chunk)[8], int lane, uint8_t* gbase,
+                                                 int64_t ld_bytes, int rows_valid) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+  for (int j = 0; j < 8; ++j) stage[lane * 8 + (j ^ (lane & 7))] = chunk[j];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    const int c = lane & 7;
+    const uint4 val = stage[r * 8 + (c ^ (r & 7))];
+    if (r < rows_valid) *reinterpret_cast<uint4*>(gbase + r * ld_bytes + 16 * c) = val;
+  }
+  __syncwarp();
+}
+
+// stage_store_pass with 64-byte row segments and a 2 KB buffer: lane l brings
+// 4 16-byte chunks of row l (chunk j of row r at slot j ^ ((r / 2) % 4), so 8
+// consecutive rows cover all 32 banks both ways); each 16-byte global store of
+// the warp covers 8 whole 64-byte row segments.
+__device__ __forceinline__ void stage_store_pass4(uint4* stage, const uint4 (&chunk)[4], int lane, uint8_t* gbase,
+                                                  int64_t ld_bytes, int rows_valid) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) stage[lane * 4 + (j ^ ((lane >> 1) & 3))] = chunk[j];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + (lane >> 2);
+    const int c = lane & 3;
+    const uint4 val = stage[r * 4 + (c ^ ((r >> 1) & 3))];
+    if (r < rows_valid) *reinterpret_cast<uint4*>(gbase + r * ld_bytes + 16 * c) = val;
+  }
+  __syncwarp();
+}
+
+// store_rows128_staged through a 2 KB buffer: 8 passes of 16 FP32 columns, 4
+// of 32 BF16 columns or 2 of 64 E4M3 codes.
+template <int kOut>
+__device__ __forceinline__ void store_rows128_staged4(const float2* acc, int lane, int row0, int rows_valid, int ncol0,
+                                                      const GemmArgs& p, uint4* stage) {
+  uint4 chunk[4];
+  if (kOut == kOutF32) {
+    uint8_t* base = reinterpret_cast<uint8_t*>(static_cast<float*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 a = acc[8 * h + 2 * j], b = acc[8 * h + 2 * j + 1];
+        chunk[j] = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
+      }
+      stage_store_pass4(stage, chunk, lane, base + 64 * h, p.ldd * 4, rows_valid);
+    }
   } else {
     uint32_t w[64];   // BF16 pairs
 #pragma unroll
     for (int j = 0; j < 64; ++j) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+      const __nv_bfloat162 h = __float22bfloat162_rn(acc[j]);
       w[j] = *reinterpret_cast<const uint32_t*>(&h);
     }
     if (kOut == kOutBf16) {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+      uint8_t* base =
+          reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      for (int h = 0; h < 4; ++h) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          chunk[j] = make_uint4(w[16 * h + 4 * j], w[16 * h + 4 * j + 1], w[16 * h + 4 * j + 2], w[16 * h + 4 * j + 3]);
+        stage_store_pass4(stage, chunk, lane, base + 64 * h, p.ldd * 2, rows_valid);
+      }
     } else {
       uint32_t m2 = 0;
 #pragma unroll
       for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
       const float s = tile_scale(amax2_value(m2));
       const float nr = -__frcp_rn(s);
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row) * p.ldd + ncol0);
+      uint8_t* base = static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t c[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            c[j] = quant_words(w[32 * h + 8 * i + 2 * j], w[32 * h + 8 * i + 2 * j + 1], nr, s);
+          chunk[i] = make_uint4(c[0], c[1], c[2], c[3]);
+        }
+        stage_store_pass4(stage, chunk, lane, base + 64 * h, p.ldd, rows_valid);
+      }
+      if (lane < rows_valid) p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
+    }
+  }
+}
+
+// The warp's 32 rows x 128 columns (row row0 + lane in acc, columns ncol0 ..
+// ncol0 + 127) through stage_store_pass: 4 passes of 32 FP32 columns, 2 of 64
+// BF16 columns, or 1 of 128 E4M3 codes plus the row's tile scale.  In
+// kOutE4m3 mode a thread's 128 values are one 1x128 tile: they are rounded to
+// BF16 and quantized exactly as quant_act_1x128_kernel quantizes a BF16 row
+// ("Fine-Grained FP8 Quantization in DeepSeek", section 2: per-tile amax,
+// s = amax/448, E4M3 cast), so the result equals quantizing the BF16 output
+// -- without writing or re-reading it.
+template <int kOut>
+__device__ __forceinline__ void store_rows128_staged(const float2* acc, int lane, int row0, int rows_valid, int ncol0,
+                                                     const GemmArgs& p, uint4* stage) {
+  if (rows_valid <= 0) return;
+  uint4 chunk[8];
+  if (kOut == kOutF32) {
+    uint8_t* base = reinterpret_cast<uint8_t*>(static_cast<float*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 a = acc[16 * h + 2 * j], b = acc[16 * h + 2 * j + 1];
+        chunk[j] = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
+      }
+      stage_store_pass(stage, chunk, lane, base + 128 * h, p.ldd * 4, rows_valid);
+    }
+  } else {
+    uint32_t w[64];   // BF16 pairs
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      const __nv_bfloat162 h = __float22bfloat162_rn(acc[j]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    if (kOut == kOutBf16) {
+      uint8_t* base =
+          reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          chunk[j] = make_uint4(w[32 * h + 4 * j], w[32 * h + 4 * j + 1], w[32 * h + 4 * j + 2], w[32 * h + 4 * j + 3]);
+        stage_store_pass(stage, chunk, lane, base + 128 * h, p.ldd * 2, rows_valid);
+      }
+    } else {
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
+      const float s = tile_scale(amax2_value(m2));
+      const float nr = -__frcp_rn(s);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         uint32_t c[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) c[j] = quant_words(w[8 * i + 2 * j], w[8 * i + 2 * j + 1], nr, s);
-        dst[i] = make_uint4(c[0], c[1], c[2], c[3]);
+        chunk[i] = make_uint4(c[0], c[1], c[2], c[3]);
       }
-      p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row] = s;
+      stage_store_pass(stage, chunk, lane, static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0,
+                       p.ldd, rows_valid);
+      if (lane < rows_valid) p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
     }
   }
 }
@@ -198,23 +317,23 @@ __device__ __forceinline__ void setmaxnreg_dec40() { asm volatile("setmaxnreg.de
 namespace fp8q {
 
 // acc[j] += v[j] * scale for 64 columns (packed FP32 pairs).
-__device__ __forceinline__ void promote64(float* acc, const uint32_t (&v)[64], float scale) {
+__device__ __forceinline__ void promote64(float2* acc, const uint32_t (&v)[64], float scale) {
+  const float2 s = f2(scale);
 #pragma unroll
-  for (int j = 0; j < 64; j += 2)
-    fma2(acc[j], acc[j + 1], __uint_as_float(v[j]), __uint_as_float(v[j + 1]), scale, scale);
+  for (int j = 0; j < 32; ++j) acc[j] = ffma2(f2u(v[2 * j], v[2 * j + 1]), s, acc[j]);
 }
 
 // Per-column scales (FP8Q_SFB_ROW): acc[j] += v[j] * (sa * sb[j]).
-__device__ __forceinline__ void promote64_rows(float* acc, const uint32_t (&v)[64], float sa, const float* sb) {
+__device__ __forceinline__ void promote64_rows(float2* acc, const uint32_t (&v)[64], float sa, const float* sb) {
   const float4* s4 = reinterpret_cast<const float4*>(sb);
+  const float2 a = f2(sa);
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const float4 s = s4[q];
-    float c0, c1, c2, c3;
-    mul2(c0, c1, s.x, s.y, sa, sa);
-    mul2(c2, c3, s.z, s.w, sa, sa);
-    fma2(acc[4 * q + 0], acc[4 * q + 1], __uint_as_float(v[4 * q + 0]), __uint_as_float(v[4 * q + 1]), c0, c1);
-    fma2(acc[4 * q + 2], acc[4 * q + 3], __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]), c2, c3);
+    const float2 c01 = fmul2(make_float2(s.x, s.y), a);
+    const float2 c23 = fmul2(make_float2(s.z, s.w), a);
+    acc[2 * q] = ffma2(f2u(v[4 * q + 0], v[4 * q + 1]), c01, acc[2 * q]);
+    acc[2 * q + 1] = ffma2(f2u(v[4 * q + 2], v[4 * q + 3]), c23, acc[2 * q + 1]);
   }
 }
 
@@ -370,7 +489,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
     const int r_in_tile = quad * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     const int nb_per_group = p.N / 128;
-    float acc[128];
+    float2 acc[64];
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
@@ -380,7 +499,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
       const int ncol0 = c.n0 + half * 128;
       const bool vcol = ncol0 < p.N;
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
       // Scale factors of chunk kc are loaded kScalePrefetch chunks ahead (a
       // register shift ring) so their L2 latency stays off the promotion path.
       const float* sa_ptr = p.sfa + row;
@@ -422,7 +541,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&go[(it + 2) % kStages]);   // buffer b is free for chunk it + 2
-        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 64, v, sa, sbv + 64); else promote64(acc + 64, v, scale);
+        if (kSfbMode == FP8Q_SFB_ROW) promote64_rows(acc + 32, v, sa, sbv + 64); else promote64(acc + 32, v, scale);
         if (kSfbMode == FP8Q_SFB_ROW) {
           // the ring slot was read with ordinary loads and is refilled by a bulk
           // copy (async proxy): order the reads before the release across proxies
@@ -432,7 +551,13 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         }
       }
       if (!ok) break;
-      if (vrow && vcol) store_row128<kOut>(acc, row, ncol0, p);
+      if (vcol) {   // warp-uniform
+        const int row0 = c.a_row0 + quad * 32;
+        const int rows_valid = min(32, c.row_end - row0);
+        if (rows_valid > 0)
+          store_rows128_staged4<kOut>(acc, lane, row0, rows_valid, ncol0, p,
+                                      reinterpret_cast<uint4*>(smem + GemmSmemLayout::out_stage + warp * 2048));
+      }
     }
   }
 

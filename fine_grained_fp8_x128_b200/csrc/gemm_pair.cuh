@@ -30,6 +30,9 @@
 // c + kPairScaleSlots - S - 2 >= c + 1, issued after the warp's last read of
 // slot c; a proxy fence before each release orders those reads before the
 // refill.
+// At the end of a tile each epilogue warp writes its 32 rows through a 4 KB
+// shared buffer (stage_store_pass) so that the global stores cover whole
+// 128-byte row segments.
 #pragma once
 
 #include "gemm.cuh"
@@ -37,13 +40,13 @@
 namespace fp8q {
 
 #ifndef FP8Q_PAIR_STAGES
-#define FP8Q_PAIR_STAGES 6
+#define FP8Q_PAIR_STAGES 5
 #endif
 constexpr int kPairStages = FP8Q_PAIR_STAGES;
 constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
 constexpr uint32_t kPairBBytes = 128 * BK;                    // 16 KB (half of the 256-row B tile)
 constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
-constexpr int kPairScaleSlots = 12;                           // scale ring (>= S + 3)
+constexpr int kPairScaleSlots = 8;                            // scale ring (>= S + 3)
 static_assert(kPairScaleSlots >= kPairStages + 3, "a scale slot may be refilled while still being read");
 // One slot: B scales at 0 (256 per-column floats, or a 4 x 2 box of block
 // scales: chunks (c & ~3)..+3 of the tile's two 128-column blocks), the 128
@@ -54,10 +57,12 @@ constexpr uint32_t kPairSaBytes = 128 * 4;
 template <int kSfbMode>
 __host__ __device__ constexpr uint32_t pair_sb_bytes() { return kSfbMode == FP8Q_SFB_ROW ? BN * 4 : 4 * 2 * 4; }
 
+constexpr uint32_t kPairOutStageBytes = 4096;                 // per epilogue warp: 32 rows x 128 bytes
 struct PairSmemLayout {
   static constexpr uint32_t stages = 0;
   static constexpr uint32_t scales = stages + kPairStages * kPairStageBytes;
-  static constexpr uint32_t bars = scales + kPairScaleSlots * kPairSlotBytes;
+  static constexpr uint32_t out_stage = scales + kPairScaleSlots * kPairSlotBytes;
+  static constexpr uint32_t bars = out_stage + kEpiWarps * kPairOutStageBytes;
   // go[S], done[S]
   static constexpr uint32_t nbars = 2 * kPairStages;
   static constexpr uint32_t misc = bars + nbars * 8;
@@ -69,7 +74,7 @@ struct PairSmemLayout {
 // (sa[2g + i] * sb[8k + 2c + j]) with c = lane % 4.  Each column-scale pair is
 // one 8-byte shared load (shared by 8 lanes) used for all 4 rows, where a
 // 32x32b row fragment would need all 128 column scales in every thread.
-__device__ __forceinline__ void promote_rows16(float* acc, const uint32_t (&v)[64], const float* sa_rows,
+__device__ __forceinline__ void promote_rows16(float2* acc, const uint32_t (&v)[64], const float* sa_rows,
                                                const float* sb_cols) {
   float sa[4];   // rows l4, l4 + 8, l4 + 16, l4 + 24
 #pragma unroll
@@ -80,9 +85,8 @@ __device__ __forceinline__ void promote_rows16(float* acc, const uint32_t (&v)[6
 #pragma unroll
     for (int q = 0; q < 4; ++q) {   // q = 2g + i
       const int x = 32 * (q >> 1) + 4 * k + 2 * (q & 1);
-      float c0, c1;
-      mul2(c0, c1, sb.x, sb.y, sa[q], sa[q]);
-      fma2(acc[x], acc[x + 1], __uint_as_float(v[x]), __uint_as_float(v[x + 1]), c0, c1);
+      const float2 c = fmul2(make_float2(sb.x, sb.y), f2(sa[q]));
+      acc[x / 2] = ffma2(f2u(v[x], v[x + 1]), c, acc[x / 2]);
     }
   }
 }
@@ -216,18 +220,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     const int r_in_tile = quad * 32 + lane;
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t leader_go0 = mapa_shared(smem_u32(&go[0]), 0);
-    float acc[128];
+    float2 acc[64];
     int it = 0;
     bool ok = true;
     for (int t = cluster; ok && t < total_tiles; t += nclusters) {
       int a_row0, n0;
       tile_rows(t, a_row0, n0);
-      const int row = a_row0 + r_in_tile;
-      const bool vrow = row < p.M;
       const int ncol0 = n0 + half * 128;
       const bool vcol = ncol0 < p.N;
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
       for (int kc = 0; kc < nk; ++kc, ++it) {
         const int b = it & 1;
         const int s = it % kPairStages;
@@ -258,9 +260,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         if (lane == 0)   // buffer b is free for chunk it + 2
           mbar_arrive_cluster(leader_go0 + static_cast<uint32_t>((it + 2) % kPairStages) * 8u);
         if (kSfbMode == FP8Q_SFB_ROW) {
-          promote_rows16(acc + 64, v, sa_rows, slot + half * 128 + 64 + 2 * (lane & 3));
+          promote_rows16(acc + 32, v, sa_rows, slot + half * 128 + 64 + 2 * (lane & 3));
         } else {
-          promote64(acc + 64, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
+          promote64(acc + 32, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
         }
       }
       if (!ok) break;
@@ -279,7 +281,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
 #pragma unroll
               for (int k = 0; k < 16; ++k) {   // k < 8: first 64 columns, k >= 8: second
                 const int x = 64 * (k >> 3) + 32 * g + 4 * (k & 7) + 2 * i;
-                const float x0 = acc[x], x1 = acc[x + 1];
+                const float x0 = acc[x / 2].x, x1 = acc[x / 2].y;
                 if (kOut == kOutF32) {
                   *reinterpret_cast<float2*>(static_cast<float*>(p.d) + base + 8 * k) = make_float2(x0, x1);
                 } else {
@@ -290,8 +292,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             }
           }
         }
-      } else if (vrow && vcol) {
-        store_row128<kOut>(acc, row, ncol0, p);
+      } else if (vcol) {
+        const int row0 = a_row0 + quad * 32;
+        store_rows128_staged<kOut>(acc, lane, row0, min(32, p.M - row0), ncol0, p,
+                                   reinterpret_cast<uint4*>(smem + PairSmemLayout::out_stage + warp * kPairOutStageBytes));
       }
     }
   }

@@ -215,7 +215,8 @@ fp8q_status fp8q_gemm_blockscaled_q1x128(const void* a, int64_t lda, const float
  *         off[G] = M_total.  Offsets outside [0, M_total] are clamped and the
  *         device status word records FP8Q_ERR_INVALID_ARG.
  *   d   : BF16 [M_total][ldd].
- * Requirements: G >= 1, M_total >= 0, N % 128 == 0, K % 128 == 0, lda >= K,
+ * Requirements: 1 <= G <= 1024 (larger G: FP8Q_ERR_UNSUPPORTED), M_total >= 0,
+ * N % 128 == 0, K % 128 == 0, lda >= K,
  * ldd >= N; alignment as for fp8q_gemm_blockscaled.
  */
 fp8q_status fp8q_grouped_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa,
