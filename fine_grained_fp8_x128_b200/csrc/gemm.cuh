@@ -337,6 +337,53 @@ __device__ __forceinline__ void promote64_rows(float2* acc, const uint32_t (&v)[
   }
 }
 
+// Grouped GEMMs, run by one warp before the main loop: clamp the device-side
+// offsets into [0, M_total], force them nondecreasing (warp max-scan), write
+// them to offs[0..G] and the exclusive prefix of each expert's tile count
+// (ceil(rows / 128) * tiles_per_block) to prefix[0..G].  Offsets that had to
+// be changed are reported through the status word (FP8Q_ERR_INVALID_ARG).
+__device__ __forceinline__ void build_group_prefix(const GemmArgs& p, int* offs, int* prefix, int tiles_per_block,
+                                                   int lane) {
+  bool bad = false;
+  int carry = 0;
+  for (int g0 = 0; g0 <= p.G; g0 += 32) {
+    const int g = g0 + lane;
+    int o = 0;
+    if (g <= p.G) {
+      const int raw = p.group_offsets[g];
+      o = min(max(raw, 0), p.M);
+      bad |= (o != raw);
+    }
+    int m = o;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, m, d);
+      if (lane >= d) m = max(m, v);
+    }
+    m = max(m, carry);
+    if (g <= p.G) { bad |= (m != o); offs[g] = m; }
+    carry = __shfl_sync(0xFFFFFFFFu, m, 31);
+  }
+  __syncwarp();
+  if (lane == 0) bad |= (offs[0] != 0) || (offs[p.G] != p.M);
+  int tcarry = 0;
+  for (int g0 = 0; g0 < p.G; g0 += 32) {
+    const int g = g0 + lane;
+    const int tg = (g < p.G) ? ((offs[g + 1] - offs[g] + BM - 1) / BM) * tiles_per_block : 0;
+    int s = tg;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, s, d);
+      if (lane >= d) s += v;
+    }
+    if (g < p.G) prefix[g] = tcarry + s - tg;
+    tcarry += __shfl_sync(0xFFFFFFFFu, s, 31);
+  }
+  if (lane == 0) prefix[p.G] = tcarry;
+  bad = __any_sync(0xFFFFFFFFu, bad);
+  if (bad && lane == 0 && blockIdx.x == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_GROUP_OFFSETS);
+}
+
 template <bool kGrouped, int kSfbMode, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -367,48 +414,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
   }
   if (warp == 8 && lane == 0) { prefetch_tmap(&tmap_a); prefetch_tmap(&tmap_b); }
   if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
-  if (kGrouped && warp == 0) {
-    // Clamp the device-side offsets into [0, M_total], force them nondecreasing
-    // (warp max-scan), then the exclusive prefix of each expert's tile count.
-    bool bad = false;
-    int carry = 0;
-    for (int g0 = 0; g0 <= p.G; g0 += 32) {
-      const int g = g0 + lane;
-      int o = 0;
-      if (g <= p.G) {
-        const int raw = p.group_offsets[g];
-        o = min(max(raw, 0), p.M);
-        bad |= (o != raw);
-      }
-      int m = o;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, m, d);
-        if (lane >= d) m = max(m, v);
-      }
-      m = max(m, carry);
-      if (g <= p.G) { bad |= (m != o); offs[g] = m; }
-      carry = __shfl_sync(0xFFFFFFFFu, m, 31);
-    }
-    __syncwarp();
-    if (lane == 0) bad |= (offs[0] != 0) || (offs[p.G] != p.M);
-    int tcarry = 0;
-    for (int g0 = 0; g0 < p.G; g0 += 32) {
-      const int g = g0 + lane;
-      const int tg = (g < p.G) ? ((offs[g + 1] - offs[g] + BM - 1) / BM) * p.num_n_tiles : 0;
-      int s = tg;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, s, d);
-        if (lane >= d) s += v;
-      }
-      if (g < p.G) prefix[g] = tcarry + s - tg;
-      tcarry += __shfl_sync(0xFFFFFFFFu, s, 31);
-    }
-    if (lane == 0) prefix[p.G] = tcarry;
-    bad = __any_sync(0xFFFFFFFFu, bad);
-    if (bad && lane == 0 && blockIdx.x == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_GROUP_OFFSETS);
-  }
+  if (kGrouped && warp == 0) build_group_prefix(p, offs, prefix, p.num_n_tiles, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

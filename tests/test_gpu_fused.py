@@ -126,6 +126,7 @@ def test_gemm_q1x128_saturating_values(fp8q, dense_kernel):
     [3, 0, 1, 130, 0, 257],          # empty experts, a 1-row expert, ragged tiles
     [1] * 9,                         # many one-row experts
     [128, 128, 0, 256],              # exact tile multiples
+    [17, 33, 48, 0, 96, 100, 5],     # assorted small experts
 ])
 def test_grouped_q1x128_equals_quantized_bf16_gemm(fp8q, counts):
     import torch
