@@ -74,18 +74,29 @@ struct PairSmemLayout {
 // (sa[2g + i] * sb[8k + 2c + j]) with c = lane % 4.  Each column-scale pair is
 // one 8-byte shared load (shared by 8 lanes) used for all 4 rows, where a
 // 32x32b row fragment would need all 128 column scales in every thread.
-__device__ __forceinline__ void promote_rows16(float2* acc, const uint32_t (&v)[64], const float* sa_rows,
-                                               const float* sb_cols) {
-  float sa[4];   // rows l4, l4 + 8, l4 + 16, l4 + 24
+// The scales are read from shared memory by the caller before the TMEM load
+// (load_rows16_scales), so their latency hides behind it.
+struct Rows16Scales {
+  float sa[4];     // rows l4, l4 + 8, l4 + 16, l4 + 24
+  float2 sb[8];    // column pairs 8k + 2c, +1
+};
+__device__ __forceinline__ void load_rows16_scales(Rows16Scales& sc, const float* sa_rows, const float* sb_cols,
+                                                   bool with_sa) {
+  if (with_sa) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) sa[q] = sa_rows[8 * ((q & 1) + 2 * (q >> 1))];
+    for (int q = 0; q < 4; ++q) sc.sa[q] = sa_rows[8 * ((q & 1) + 2 * (q >> 1))];
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) sc.sb[k] = *reinterpret_cast<const float2*>(sb_cols + 8 * k);
+}
+__device__ __forceinline__ void promote_rows16(float2* acc, const uint32_t (&v)[64], const Rows16Scales& sc) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const float2 sb = *reinterpret_cast<const float2*>(sb_cols + 8 * k);
+    const float2 sb = sc.sb[k];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {   // q = 2g + i
       const int x = 32 * (q >> 1) + 4 * k + 2 * (q & 1);
-      const float2 c = fmul2(make_float2(sb.x, sb.y), f2(sa[q]));
+      const float2 c = fmul2(make_float2(sb.x, sb.y), f2(sc.sa[q]));
       acc[x / 2] = ffma2(f2u(v[x], v[x + 1]), c, acc[x / 2]);
     }
   }
@@ -243,13 +254,20 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         // FP8Q_SFB_ROW, 16x256b fragments: rows 32*quad + {l4, l4+8, l4+16, l4+24}
         // with l4 = lane/4; columns 8k + 2*(lane%4) + {0,1} of each 64-column half
         const float* sa_rows = slot + kPairSlotSa / 4 + quad * 32 + (lane >> 2);
+        // the scales are read before the TMEM loads so that their shared-memory
+        // latency overlaps the loads instead of following them
+        Rows16Scales sc;
+        float scale = 0.0f;
         if (kSfbMode == FP8Q_SFB_ROW) {
+          load_rows16_scales(sc, sa_rows, slot + half * 128 + 2 * (lane & 3), true);
           tmem_ld_16x256b_x8x2_sync(taddr, v);
-          promote_rows16(acc, v, sa_rows, slot + half * 128 + 2 * (lane & 3));
+          promote_rows16(acc, v, sc);
+          load_rows16_scales(sc, sa_rows, slot + half * 128 + 64 + 2 * (lane & 3), false);
           tmem_ld_16x256b_x8x2_sync(taddr + 64, v);
         } else {
+          scale = slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)];
           tmem_ld_32x32b_x64_sync(taddr, v);
-          promote64(acc, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
+          promote64(acc, v, scale);
           tmem_ld_32x32b_x64_sync(taddr + 64, v);
         }
         // scale slots read so far (ordinary loads) are refilled by TMA (async
@@ -260,9 +278,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         if (lane == 0)   // buffer b is free for chunk it + 2
           mbar_arrive_cluster(leader_go0 + static_cast<uint32_t>((it + 2) % kPairStages) * 8u);
         if (kSfbMode == FP8Q_SFB_ROW) {
-          promote_rows16(acc + 32, v, sa_rows, slot + half * 128 + 64 + 2 * (lane & 3));
+          promote_rows16(acc + 32, v, sc);
         } else {
-          promote64(acc + 32, v, slot[kPairSlotSa / 4 + r_in_tile] * slot[half * 4 + (kc & 3)]);
+          promote64(acc + 32, v, scale);
         }
       }
       if (!ok) break;
