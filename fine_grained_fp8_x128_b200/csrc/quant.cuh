@@ -142,8 +142,8 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
 // cast.  Thread t owns the channel pair p = t % 64 for the 32-token
 // quarter r = t / 64: a bank-conflict-free 32-bit shared load per token gives
 // both channels, the four quarters' maxima combine through shared memory, and
-// each thread writes its 32 codes per channel as two 16-byte stores (whole
-// 32-byte sectors of the rows qt[c]).
+// the codes go back through the staged tile as [channel][128 tokens] rows so
+// that the block writes whole 128-byte rows of qt.
 // ---------------------------------------------------------------------------
 constexpr int kQTThreads = 256;
 constexpr int kQTCols = 128;
@@ -195,6 +195,7 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
     const int64_t c0 = (it - tb * col_blocks) * kQTCols;
     const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;
     const bool active = 2 * p < ncols;
+    uint4 codes[4];                  // channel 2p: tokens 32r .. +15, +16 .. +31; then channel 2p+1
     float ma = 0.0f, mb = 0.0f;
     if (active) {
       uint32_t m2 = 0;   // channel 2p in the low half, 2p+1 in the high half
@@ -213,8 +214,6 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
       const float sa = tile_scale(ma), sb = tile_scale(mb);
       const float nra = -__frcp_rn(sa), nrb = -__frcp_rn(sb);
       const int64_t ca = c0 + 2 * p;
-      uint8_t* qa = qt + ca * ldqt + tb * 128 + 32 * r;
-      uint8_t* qb = qa + ldqt;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t oa[4], ob[4];
@@ -232,13 +231,34 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
           oa[j] = a4 ^ kFlipSigns;
           ob[j] = b4 ^ kFlipSigns;
         }
-        *reinterpret_cast<uint4*>(qa + 16 * h) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        *reinterpret_cast<uint4*>(qb + 16 * h) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        codes[h] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        codes[2 + h] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
       }
       if (r == 0) {
         sf[tb * ld_sf + ca] = sa;
         sf[tb * ld_sf + ca + 1] = sb;
       }
+    }
+    // Transpose the codes through the staged tile (every read of it is done):
+    // channel row c holds its 128 token codes, 16-byte chunk j at slot
+    // j ^ ((c / 2) % 8), so the 8 lanes of a wavefront hit 8 different bank
+    // groups both when the rows are written and when they are read back; each
+    // warp store instruction then writes 4 whole 128-byte rows of qt.
+    __syncthreads();
+    uint4* crows = reinterpret_cast<uint4*>(q2_smem + buf * kQTTileBytes);
+    if (active) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = 2 * r + h;
+        crows[(2 * p) * 8 + (j ^ (p & 7))] = codes[h];
+        crows[(2 * p + 1) * 8 + (j ^ (p & 7))] = codes[2 + h];
+      }
+    }
+    __syncthreads();
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int row = 4 * warp + (lane >> 3); row < ncols; row += 4 * (kQTThreads / 32)) {
+      const int j = lane & 7;
+      *reinterpret_cast<uint4*>(qt + (c0 + row) * ldqt + tb * 128 + 16 * j) = crows[row * 8 + (j ^ ((row >> 1) & 7))];
     }
     __syncthreads();   // this buffer is refilled two items later; the maxima are reused next item
   }
