@@ -270,7 +270,8 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
 // 8*(t/16).., columns 8*(t%16)..: eight 16-byte row loads (16 lanes cover one
 // 256-byte row), block amax via shuffles and shared memory, eight 8-byte Q
 // stores, and, for Q^T, an in-register 8x8 byte transpose (byte permutes)
-// followed by eight 8-byte stores of the transposed rows.
+// whose rows go through a 16 KB shared buffer so that the block writes whole
+// 128-byte rows of Q^T.
 // ---------------------------------------------------------------------------
 constexpr int kQWThreads = 256;
 
@@ -292,6 +293,7 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
                        uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
                        uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sft, int64_t ld_sft) {
   __shared__ float warp_max[kQWThreads / 32];
+  __shared__ __align__(16) uint2 tstage[128 * 16];   // the block's codes transposed: [k][16 x 8 n]
   const int tid = threadIdx.x;
   const int a = tid >> 4;        // rows 8a .. 8a+7
   const int b = tid & 15;        // cols 8b .. 8b+7
@@ -333,10 +335,21 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
       transpose4x4(hi[0], hi[1], hi[2], hi[3], c01);
       transpose4x4(lo[4], lo[5], lo[6], lo[7], c10);
       transpose4x4(hi[4], hi[5], hi[6], hi[7], c11);
+      // Q^T rows k0 + 8b + j, columns n0 + 8a .. +7, through shared memory:
+      // 8-byte chunk a of row kk at slot a ^ (kk / 8 % 16), so the 16 lanes of
+      // a wavefront (16 rows, one chunk each) hit 16 different slots; read back
+      // a warp instruction writes 2 whole 128-byte rows of qt.
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        *reinterpret_cast<uint2*>(qt + (k0 + 8 * b + j) * ldqt + n0 + 8 * a) = make_uint2(c00[j], c10[j]);
-        *reinterpret_cast<uint2*>(qt + (k0 + 8 * b + 4 + j) * ldqt + n0 + 8 * a) = make_uint2(c01[j], c11[j]);
+        tstage[(8 * b + j) * 16 + (a ^ b)] = make_uint2(c00[j], c10[j]);
+        tstage[(8 * b + 4 + j) * 16 + (a ^ b)] = make_uint2(c01[j], c11[j]);
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int kk = 16 * i + (tid >> 4);   // 16 rows per pass over the block's 256 threads
+        const int c = tid & 15;
+        *reinterpret_cast<uint2*>(qt + (k0 + kk) * ldqt + n0 + 8 * c) = tstage[kk * 16 + (c ^ ((kk >> 3) & 15))];
       }
     }
     if (tid == 0) {
