@@ -59,6 +59,8 @@ def _load():
     lib.orc_tile_scale.argtypes = [ctypes.c_float]
     lib.orc_tile_scale.restype = ctypes.c_float
     lib.orc_quant_act_1x128.argtypes = [P, I64, I64, I64, P, I64, P]
+    lib.orc_quant_act_1x128_scaled.argtypes = [P, I64, I64, I64, P, P, I64, P, P]
+    lib.orc_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, P, P, P, I64]
     lib.orc_quant_act_128x1.argtypes = [P, I64, I64, I64, P, I64, P]
     lib.orc_quant_w_128x128.argtypes = [P, I64, I64, I64, P, I64, P]
     lib.orc_quant_tiles_intgrid.argtypes = [P, I64, I64, P]
@@ -203,6 +205,87 @@ def quant_pertensor_e4m3(x_bf16: np.ndarray):
     s = ctypes.c_float()
     _load().orc_quant_pertensor_e4m3(_p(x), x.size, _p(deq), ctypes.cast(ctypes.pointer(s), ctypes.c_void_p))
     return deq, s.value
+
+
+# ---------------------------------------------------------------- scale policies
+POLICY_PREVIOUS = 0     # delayed: the previous step's tile maximum
+POLICY_EMA = 1          # exponential amax history
+POLICY_DECAYED_MAX = 2  # running maximum that decays by alpha per step
+
+
+def quant_act_1x128_scaled(x_bf16: np.ndarray, sf: np.ndarray):
+    """1x128 tiles cast with GIVEN scales sf [M][K/128] (a scale policy's).
+    Returns (q uint8 [M][K], amax float32 [M][K/128] of the current tiles,
+    clipped = number of elements the saturating cast clamps, |fl32(x / s)| > 464)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    sf = np.ascontiguousarray(sf, dtype=np.float32)
+    assert sf.shape == (M, K // 128)
+    q = np.empty((M, K), np.uint8)
+    amax = np.empty((M, K // 128), np.float32)
+    clipped = ctypes.c_int64(0)
+    _check(_load().orc_quant_act_1x128_scaled(_p(x), M, K, K, _p(sf), _p(q), K, _p(amax),
+                                              ctypes.cast(ctypes.pointer(clipped), ctypes.c_void_p)),
+           "quant_act_1x128_scaled")
+    return q, amax, int(clipped.value)
+
+
+def scale_history_update(policy: int, alpha: float, amax: np.ndarray, hist: np.ndarray):
+    """One history step for each tile: returns (new history, next scales), float32."""
+    a = np.ascontiguousarray(amax, dtype=np.float32)
+    h = np.array(hist, dtype=np.float32, copy=True)
+    sf = np.empty_like(a)
+    _check(_load().orc_scale_history_update(int(policy), float(alpha), _p(a), _p(h), _p(sf), a.size),
+           "scale_history_update")
+    return h, sf
+
+
+def scale_policy_drift(tiles_bf16: np.ndarray, alpha: float = 0.9):
+    """The [P1] worked example on the oracle: one 1x128 tile per step
+    (tiles_bf16 [steps][128], e.g. a standard deviation doubling over the steps
+    with a rare outlier) quantized under five policies -- current-max (online),
+    fixed calibration (the first step's scale), previous-step delayed, EMA
+    history and decaying maximum.  Returns {policy: (clip_rate [steps],
+    mean_rel_err [steps])}: the fraction of clipped elements, and
+    mean |dequant - x| / mean |x| of each step's tile."""
+    x = np.ascontiguousarray(tiles_bf16, dtype=np.uint16)
+    steps = x.shape[0]
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    table = e4m3_decode(np.arange(256, dtype=np.uint8))
+
+    def measure(row, s):
+        q, amax, clipped = quant_act_1x128_scaled(x[row:row + 1], np.array([[s]], np.float32))
+        deq = table[q[0]] * float(s)
+        err = np.abs(deq - xf[row]).mean() / max(np.abs(xf[row]).mean(), 1e-300)
+        return clipped / 128.0, err, float(amax[0, 0])
+
+    out = {}
+    # current-max: each step's own tile maximum
+    cr, er = np.zeros(steps), np.zeros(steps)
+    for t in range(steps):
+        _, s = quant_act_1x128(x[t:t + 1])
+        cr[t], er[t], _ = measure(t, s[0, 0])
+    out["current_max"] = (cr, er)
+    # fixed calibration: the first step's scale for every step
+    _, s0 = quant_act_1x128(x[0:1])
+    cr, er = np.zeros(steps), np.zeros(steps)
+    for t in range(steps):
+        cr[t], er[t], _ = measure(t, s0[0, 0])
+    out["fixed"] = (cr, er)
+    # history policies: step 0 is calibrated on itself, step t uses the history after step t-1
+    for name, pol in (("previous", POLICY_PREVIOUS), ("ema", POLICY_EMA), ("decayed_max", POLICY_DECAYED_MAX)):
+        cr, er = np.zeros(steps), np.zeros(steps)
+        _, s = quant_act_1x128(x[0:1])
+        hist = np.zeros(1, np.float32)
+        first = True
+        for t in range(steps):
+            cr[t], er[t], a = measure(t, s[0, 0] if first else s[0])
+            if first:
+                hist[0] = a            # the history starts at the calibration step's maximum
+                first = False
+            hist, s = scale_history_update(pol, alpha, np.array([a], np.float32), hist)
+        out[name] = (cr, er)
+    return out
 
 
 # ---------------------------------------------------------------- GEMMs

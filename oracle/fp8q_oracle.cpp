@@ -489,4 +489,74 @@ void orc_quant_pertensor_e4m3(const uint16_t* x, int64_t n, double* deq, float* 
   for (int64_t i = 0; i < n; ++i) deq[i] = e4m3_decode(e4m3_encode(bf16_to_float(x[i]) / s)) * s;
 }
 
+// ---- scale policies: quantizing with given scales, and history updates -------
+// [P1] "4. Max scaling is robust but noisy": percentile clipping, delayed
+// scaling or amax histories trade clipping against stability, and any smoother
+// lags; [P1] "Worked example": fixed calibration, current-max and an
+// exponential amax history compared on clipping rate and mean error; [P5]
+// "5) Online Quantization", "Delayed Quantization (Previous Method)": the scale
+// of the current tensor comes from past maxima, so a range change overflows.
+//
+// Readings: a policy supplies one scale per 1x128 tile; the tile is cast as the
+// online rule casts it, q = e4m3(fl32(x / s)) with IEEE division, and an
+// element is "clipped" when the cast saturates it: |fl32(x / s)| > 464, the
+// point above which round-to-nearest-even would leave 448, the E4M3 maximum
+// (448 < v <= 464 rounds to 448 by itself).
+// x: bf16 [M][ldx]; sf: [M][K/128] given scales; q: [M][ldq];
+// amax: [M][K/128] the tiles' current maxima (for the history update; may be
+// NULL); *clipped += the number of clipped elements (may be NULL).
+int orc_quant_act_1x128_scaled(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const float* sf,
+                               uint8_t* q, int64_t ldq, float* amax, int64_t* clipped) {
+  if (K % 128 != 0 || ldx < K || ldq < K || M < 0) return 1;
+  const int64_t KB = K / 128;
+  int64_t total = 0;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t kb = 0; kb < KB; ++kb) {
+      const uint16_t* t = x + m * ldx + kb * 128;
+      const float s = sf[m * KB + kb];
+      float mx = 0.0f;
+      for (int i = 0; i < 128; ++i) {
+        const float xv = bf16_to_float(t[i]);
+        mx = std::max(mx, std::fabs(xv));
+        const float v = xv / s;
+        if (std::fabs(v) > 464.0f) ++total;
+        q[m * ldq + kb * 128 + i] = e4m3_encode(v);
+      }
+      if (amax != nullptr) amax[m * KB + kb] = mx;
+    }
+  }
+  if (clipped != nullptr) *clipped += total;
+  return 0;
+}
+
+// One step of a tile-scale history ([P1] section 4 and worked example), for n
+// tiles: the state h is updated from the step's tile maxima a, and the next
+// step's scale is s = max(fl32(h / 448), fl32(1e-12)), the online rule applied
+// to the history instead of the current tile.
+//   policy 0, previous step (delayed):   h = a
+//   policy 1, exponential history:       h = fl32(fl32(alpha * h) + fl32(fl32(1 - alpha) * a))
+//   policy 2, decaying maximum:          h = max(a, fl32(alpha * h))
+// Every product and sum is rounded to FP32 on its own (the build disables
+// contraction), which fixes the result bit for bit.
+int orc_scale_history_update(int policy, float alpha, const float* a, float* h, float* sf, int64_t n) {
+  if (policy < 0 || policy > 2 || n < 0) return 1;
+  const float beta = 1.0f - alpha;
+  for (int64_t i = 0; i < n; ++i) {
+    float nh;
+    if (policy == 0) {
+      nh = a[i];
+    } else if (policy == 1) {
+      const float p = alpha * h[i];
+      const float r = beta * a[i];
+      nh = p + r;
+    } else {
+      const float d = alpha * h[i];
+      nh = std::max(a[i], d);
+    }
+    h[i] = nh;
+    sf[i] = orc_tile_scale(nh);
+  }
+  return 0;
+}
+
 }  // extern "C"

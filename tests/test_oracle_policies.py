@@ -1,0 +1,101 @@
+"""Pins of the oracle's scale-policy functions ("Online Quantization During
+Training", section 4 "Max scaling is robust but noisy" and its worked example;
+"Introduction to LLM Quantization", "5) Online Quantization", delayed versus
+online quantization).
+
+The quantizer with given scales reduces to the online quantizer when it is
+given the online scales; its cast and clip count are checked against NumPy's
+IEEE float32 division and the codec; the history updates are checked through
+their special cases and invariants; the drift simulation through the
+behaviour the pages describe.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+
+
+def test_given_online_scales_reproduce_the_online_quantizer():
+    x = W.activations_with_outliers(40, 512, seed=3, channel_frac=2 / 512, elem_frac=1e-2)
+    q_on, sf_on = oracle.quant_act_1x128(x)
+    q, amax, clipped = oracle.quant_act_1x128_scaled(x, sf_on)
+    assert np.array_equal(q, q_on)
+    assert clipped == 0                                # the online scale never saturates its tile
+    # the recorded maxima are the tiles' maxima: the online rule rebuilds the same scales
+    assert np.array_equal(np.vectorize(oracle.tile_scale, otypes=[np.float32])(amax), sf_on)
+    xf = W.bf16_bits_to_f32(x).reshape(40, 4, 128)
+    assert np.array_equal(amax, np.abs(xf).max(axis=2))
+
+
+@pytest.mark.parametrize("scale_mult", [1.0, 0.5, 0.01, 7.3])
+def test_scaled_cast_and_clip_count_against_numpy(scale_mult):
+    """Arbitrary scales: codes = codec(float32(x) / float32(s)) and the clip
+    count = #|x/s| > 464 (the saturating cast's threshold), by brute force."""
+    x = W.activations_with_outliers(16, 384, seed=5, channel_frac=0, elem_frac=1e-2)
+    _, sf_on = oracle.quant_act_1x128(x)
+    sf = (sf_on * np.float32(scale_mult)).astype(np.float32)
+    q, _, clipped = oracle.quant_act_1x128_scaled(x, sf)
+    xf = W.bf16_bits_to_f32(x)
+    v = (xf.reshape(16, 3, 128) / sf[:, :, None]).astype(np.float32).reshape(16, 384)
+    assert np.array_equal(q, oracle.e4m3_encode(v))
+    assert clipped == int((np.abs(v) > 464.0).sum())
+    if scale_mult < 1.0:
+        assert clipped > 0
+    # saturated elements carry the extreme codes
+    assert np.all(np.isin(q[np.abs(v) > 464.0], [0x7E, 0xFE]))
+
+
+def test_history_update_special_cases():
+    rng = np.random.default_rng(0)
+    a = rng.uniform(0.01, 50.0, 64).astype(np.float32)
+    h = rng.uniform(0.01, 50.0, 64).astype(np.float32)
+    tile = np.vectorize(oracle.tile_scale, otypes=[np.float32])
+    # previous step: the history is the last maximum, whatever alpha
+    h0, s0 = oracle.scale_history_update(oracle.POLICY_PREVIOUS, 0.7, a, h)
+    assert np.array_equal(h0, a) and np.array_equal(s0, tile(a))
+    # EMA with alpha = 0 forgets, alpha = 1 never moves; decayed max with alpha = 0 is the current max
+    h1, _ = oracle.scale_history_update(oracle.POLICY_EMA, 0.0, a, h)
+    assert np.array_equal(h1, a)
+    h2, _ = oracle.scale_history_update(oracle.POLICY_EMA, 1.0, a, h)
+    assert np.array_equal(h2, h)
+    h3, _ = oracle.scale_history_update(oracle.POLICY_DECAYED_MAX, 0.0, a, h)
+    assert np.array_equal(h3, a)
+    # EMA of a constant stays at it; decayed max never falls below the current maximum
+    hc, _ = oracle.scale_history_update(oracle.POLICY_EMA, 0.9, a, a)
+    assert np.allclose(hc, a, rtol=2 ** -22)
+    hd, sd = oracle.scale_history_update(oracle.POLICY_DECAYED_MAX, 0.8, a, h)
+    assert np.all(hd >= a) and np.all(hd >= (np.float32(0.8) * h).astype(np.float32))
+    assert np.array_equal(sd, tile(hd))
+    # EMA lies between its two inputs
+    he, _ = oracle.scale_history_update(oracle.POLICY_EMA, 0.9, a, h)
+    lo, hi = np.minimum(a, h), np.maximum(a, h)
+    assert np.all(he >= lo * (1 - 2 ** -22)) and np.all(he <= hi * (1 + 2 ** -22))
+
+
+def test_bad_policy_is_rejected():
+    with pytest.raises(Exception):
+        oracle.scale_history_update(3, 0.5, np.ones(4, np.float32), np.ones(4, np.float32))
+
+
+def test_drift_simulation_matches_the_pages_claims():
+    """The worked example: std doubling over 100 steps, one 20-sigma outlier.
+    Current-max never clips; a fixed calibration clips more and more as the
+    distribution widens; every history policy clips the outlier (it lags
+    behind a sudden range change) and pays for it in error at that step."""
+    tiles, t_out = W.drift_tiles(steps=100, seed=0)
+    res = oracle.scale_policy_drift(tiles, alpha=0.9)
+    clip_cur, err_cur = res["current_max"]
+    assert np.all(clip_cur == 0)
+    clip_fix, err_fix = res["fixed"]
+    assert clip_fix[:10].mean() < clip_fix[-10:].mean()
+    assert clip_fix[-10:].mean() > 0.1
+    for name in ("previous", "ema", "decayed_max"):
+        clip, err = res[name]
+        assert clip[t_out] >= 1 / 128, name                 # the outlier is clamped
+        assert err[t_out] > 5 * err_cur[t_out], name
+        assert clip.mean() < clip_fix.mean(), name          # but far less clipping than a fixed scale
+    # E4M3 is a floating-point grid: a 20-sigma tile maximum leaves the other
+    # values well inside the normal range, so current-max loses little there
+    neighbours = np.r_[err_cur[t_out - 3:t_out], err_cur[t_out + 1:t_out + 4]]
+    assert err_cur[t_out] < 2 * neighbours.mean()

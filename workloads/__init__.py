@@ -203,3 +203,16 @@ def expert_weights_device(G: int, N: int, K: int, seed: int = 0, sigma: float = 
     for g in range(G):
         out[g] = (torch.randn((N, K), generator=gen, device=device, dtype=torch.float32) * sigma).to(torch.bfloat16)
     return out
+
+
+def drift_tiles(steps: int = 100, seed: int = 0, outlier_sigmas: float = 20.0):
+    """The scale-policy drift workload: one 1x128 tile per step whose standard
+    deviation doubles over the steps (sigma_t = 2^(t / (steps - 1))), with one
+    element of one seeded step (in the middle half) replaced by an outlier of
+    outlier_sigmas * sigma_t.  Returns (bf16 bits [steps][128], outlier step)."""
+    g = _rng(seed, TID_MISC, 1)
+    sig = np.exp2(np.arange(steps, dtype=np.float64) / max(steps - 1, 1))
+    x = (g.standard_normal((steps, 128)) * sig[:, None]).astype(np.float32)
+    t_out = int(g.integers(steps // 4, 3 * steps // 4))
+    x[t_out, int(g.integers(0, 128))] = np.float32(outlier_sigmas * sig[t_out])
+    return f32_to_bf16_bits(x), t_out
