@@ -493,7 +493,11 @@ def run_fp8q(args):
     device = f"cuda:{local}"
     init_dist(world, "nccl")
     if rank == 0:
-        from fine_grained_fp8_x128_b200 import build as _b
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(
+            "fp8q_build", os.path.join(ROOT, "fine_grained_fp8_x128_b200", "build.py"))
+        _b = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(_b)
         _b.build()
     barrier(world, device)
     import fine_grained_fp8_x128_b200 as fp8q
@@ -644,7 +648,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -666,15 +670,22 @@ def run_single(args):
     ld = fp8q.sf_ld
     u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
     work = None
-    if name in ("quant_x", "quant_x_t"):
+    if name in ("quant_x", "quant_x_scaled", "quant_x_t"):
         x = randn(T, HID)
-        if name == "quant_x":
+        if name == "quant_x_scaled":
+            # a scale policy's pass: given scales (here the online ones), tile maxima and clip count out
+            q = torch.empty((T, HID), dtype=u8, device=dev); sf = torch.empty((HID // 128, ld(T)), dtype=f32, device=dev)
+            fp8q.fp8q_quant_act_1x128(x, q, sf)
+            amax = torch.empty_like(sf)
+            clipped = torch.zeros(1, dtype=torch.int64, device=dev)
+            fn = lambda: fp8q.fp8q_quant_act_1x128_scaled(x, sf, q, amax, clipped)
+        elif name == "quant_x":
             q = torch.empty((T, HID), dtype=u8, device=dev); sf = torch.empty((HID // 128, ld(T)), dtype=f32, device=dev)
             fn = lambda: fp8q.fp8q_quant_act_1x128(x, q, sf)
         else:
             q = torch.empty((HID, T), dtype=u8, device=dev); sf = torch.empty((T // 128, ld(HID)), dtype=f32, device=dev)
             fn = lambda: fp8q.fp8q_quant_act_128x1(x, q, sf)
-        work = ("bytes", T * HID * 3 + T * HID // 128 * 4)
+        work = ("bytes", T * HID * 3 + T * HID // 128 * (8 if name == "quant_x_scaled" else 4))
     elif name == "quant_w":
         w = randn(OUT, HID, sigma=0.02)
         q, sf, qt, sft = fp8q.quant_w_128x128(w, transposed=True)

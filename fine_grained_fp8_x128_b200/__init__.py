@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("FP8Q_LIBRARY") or os.path.join(_HERE, "libfp8q.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libfp8q.so is not built ({LIB_PATH}); run `python -m fine_grained_fp8_x128_b200.build`")
+    raise ImportError(f"libfp8q.so is not built ({LIB_PATH}); run `python fine_grained_fp8_x128_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -33,12 +33,16 @@ FP8Q_ERR_CUDA = 4
 FP8Q_ERR_TIMEOUT = 5
 FP8Q_SFB_BLOCK128 = 0
 FP8Q_SFB_ROW = 1
+FP8Q_POLICY_PREVIOUS = 0
+FP8Q_POLICY_EMA = 1
+FP8Q_POLICY_DECAYED_MAX = 2
 FP8Q_OUT_BF16 = 0
 FP8Q_OUT_F32 = 1
 
 EXPORTS = (
     "fp8q_version", "fp8q_status_string", "fp8q_device_status",
-    "fp8q_quant_act_1x128", "fp8q_quant_act_1x128_gather", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
+    "fp8q_quant_act_1x128", "fp8q_quant_act_1x128_gather", "fp8q_quant_act_1x128_scaled",
+    "fp8q_scale_history_update", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
     "fp8q_gemm_blockscaled", "fp8q_gemm_blockscaled_q1x128",
     "fp8q_grouped_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled_q1x128",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
@@ -52,6 +56,8 @@ _lib.fp8q_status_string.restype = ctypes.c_char_p
 _lib.fp8q_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int)]
 _lib.fp8q_quant_act_1x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_gather.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_1x128_scaled.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]
+_lib.fp8q_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, _P, _P, _P, _I, _P]
 _lib.fp8q_quant_act_128x1.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_w_128x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_gemm_blockscaled.argtypes = [_P, _I, _P, _I, _P, _I, _P, _I, ctypes.c_int, _P, _I, ctypes.c_int,
@@ -130,6 +136,22 @@ def fp8q_quant_act_1x128_gather(x, rows, q, sf, stream=None):
     M = rows.shape[0]
     _check(_lib.fp8q_quant_act_1x128_gather(_ptr(x), M_src, K, _ld(x), _ptr(rows), M, _ptr(q), _ld(q), _ptr(sf),
                                             _ld(sf), _stream(stream)), "fp8q_quant_act_1x128_gather")
+
+
+def fp8q_quant_act_1x128_scaled(x, sf, q, amax=None, clipped=None, stream=None):
+    """q = e4m3(x / sf) per 1x128 tile with given scales sf [K/128][ld >= M];
+    optional amax [K/128][ld] (tile maxima out) and clipped (int64 device
+    counter, += saturated elements)."""
+    M, K = x.shape
+    _check(_lib.fp8q_quant_act_1x128_scaled(_ptr(x), M, K, _ld(x), _ptr(sf), _ld(sf), _ptr(q), _ld(q), _ptr(amax),
+                                            _ld(amax) if amax is not None else 0, _ptr(clipped), _stream(stream)),
+           "fp8q_quant_act_1x128_scaled")
+
+
+def fp8q_scale_history_update(policy, alpha, amax, hist, sf, stream=None):
+    """Elementwise over n = amax.numel() tiles: hist <- policy(hist, amax), sf <- tile scale of hist."""
+    _check(_lib.fp8q_scale_history_update(int(policy), float(alpha), _ptr(amax), _ptr(hist), _ptr(sf), amax.numel(),
+                                          _stream(stream)), "fp8q_scale_history_update")
 
 
 def fp8q_quant_act_128x1(x, qt, sf, stream=None):

@@ -32,6 +32,7 @@ struct DeviceInfo {
   int pair_clusters[2][3] = {};    // co-resident CTA pairs per kernel instance
   int q1_per_sm = 0;               // resident blocks per SM of each quantizer
   int q1g_per_sm = 0;
+  int q1s_per_sm = 0;
   int q2_per_sm = 0;
   int qw_per_sm = 0;
 };
@@ -417,6 +418,46 @@ fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K,
   const int64_t grid = grid_for(items, dev->sm_count, per_sm);
   fp8q::quant_act_1x128_kernel<true><<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, rows, M_src);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_act_1x128_scaled(const void* x, int64_t M, int64_t K, int64_t ldx, const float* sf,
+                                        int64_t ld_sf, void* q, int64_t ldq, float* amax, int64_t ld_amax,
+                                        unsigned long long* clipped, void* stream) {
+  if (M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M) return FP8Q_ERR_INVALID_ARG;
+  if (amax != nullptr && ld_amax < M) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || sf == nullptr || q == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldq % 16 != 0 ||
+      (amax != nullptr && !aligned(amax, 4)) || (clipped != nullptr && !aligned(clipped, 8)))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  const int per_sm = blocks_per_sm(&dev->q1s_per_sm, fp8q::quant_act_1x128_scaled_kernel, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  fp8q::quant_act_1x128_scaled_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0,
+                                        static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, sf, ld_sf, static_cast<uint8_t*>(q), ldq, amax, ld_amax,
+      clipped);
+  return launch_status();
+}
+
+fp8q_status fp8q_scale_history_update(int policy, float alpha, const float* amax, float* hist, float* sf, int64_t n,
+                                      void* stream) {
+  if (policy < FP8Q_POLICY_PREVIOUS || policy > FP8Q_POLICY_DECAYED_MAX || n < 0) return FP8Q_ERR_INVALID_ARG;
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return FP8Q_ERR_INVALID_ARG;
+  if (n == 0) return FP8Q_OK;
+  if (amax == nullptr || hist == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(amax, 4) || !aligned(hist, 4) || !aligned(sf, 4)) return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t grid = grid_for((n + 255) / 256, dev->sm_count, 8);
+  fp8q::scale_history_update_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      policy, alpha, amax, hist, sf, n);
   return launch_status();
 }
 

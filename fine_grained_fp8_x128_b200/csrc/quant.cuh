@@ -136,6 +136,89 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
 }
 
 // ---------------------------------------------------------------------------
+// Scale policies ("Online Quantization During Training", section 4 and its
+// worked example; "Introduction to LLM Quantization", "5) Online Quantization",
+// delayed quantization): 1x128 tiles cast with GIVEN scales (a policy's, e.g.
+// from a tile-maximum history) instead of their own maxima.  Same tiling as
+// quant_act_1x128_kernel.  Each tile's maximum is recorded for the history
+// update, and the elements the saturating cast clamps (|fl32(x / s)| > 464:
+// above that, round-to-nearest-even would leave 448) are counted.  A given
+// scale need not bound the tile, so the cast divides (IEEE) instead of using
+// the reciprocal form, whose exactness was checked only for s = max|tile|/448.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQ1Threads)
+quant_act_1x128_scaled_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
+                              const float* __restrict__ sf_in, int64_t ld_sf_in, uint8_t* __restrict__ q, int64_t ldq,
+                              float* __restrict__ amax_out, int64_t ld_amax, unsigned long long* __restrict__ clipped) {
+  const int tid = threadIdx.x;
+  const int sub = tid & 3;
+  const int tile = tid >> 2;
+  const int64_t items = ((M + kQ1Rows - 1) / kQ1Rows) * KB;
+  unsigned int nclip = 0;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int64_t rb = it / KB;
+    const int64_t kb = it - rb * KB;
+    const int64_t row = rb * kQ1Rows + tile;
+    Q1Slice cur;
+    q1_load<false>(cur, x, M, KB, ldx, nullptr, 0, it, tile, sub);
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m2 = amax2(m2, cur.v[i].x); m2 = amax2(m2, cur.v[i].y);
+      m2 = amax2(m2, cur.v[i].z); m2 = amax2(m2, cur.v[i].w);
+    }
+    float m = amax2_value(m2);
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    if (row < M) {
+      const float s = sf_in[kb * ld_sf_in + row];
+      uint8_t* dst = q + row * ldq + kb * 128 + sub * 8;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t w[4] = {cur.v[i].x, cur.v[i].y, cur.v[i].z, cur.v[i].w};
+        uint32_t c[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float v0 = __fdiv_rn(bf16lo(w[2 * j]), s), v1 = __fdiv_rn(bf16hi(w[2 * j]), s);
+          const float v2 = __fdiv_rn(bf16lo(w[2 * j + 1]), s), v3 = __fdiv_rn(bf16hi(w[2 * j + 1]), s);
+          nclip += (fabsf(v0) > 464.0f) + (fabsf(v1) > 464.0f) + (fabsf(v2) > 464.0f) + (fabsf(v3) > 464.0f);
+          c[j] = cvt_e4m3x2(v0, v1) | (cvt_e4m3x2(v2, v3) << 16);
+        }
+        *reinterpret_cast<uint2*>(dst + 32 * i) = make_uint2(c[0], c[1]);
+      }
+      if (sub == 0 && amax_out != nullptr) amax_out[kb * ld_amax + row] = m;
+    }
+  }
+  if (clipped != nullptr) {
+    const unsigned int warp_clip = __reduce_add_sync(0xFFFFFFFFu, nclip);
+    if ((tid & 31) == 0 && warp_clip != 0) atomicAdd(clipped, static_cast<unsigned long long>(warp_clip));
+  }
+}
+
+// One history step per tile: h <- policy(h, amax), sf <- max(fl32(h / 448),
+// fl32(1e-12)).  Policies: 0 previous step (h = a), 1 exponential history
+// (h = fl32(fl32(alpha*h) + fl32(fl32(1 - alpha)*a))), 2 decaying maximum
+// (h = max(a, fl32(alpha*h))); every operation rounded on its own.
+__global__ void scale_history_update_kernel(int policy, float alpha, const float* __restrict__ a,
+                                            float* __restrict__ h, float* __restrict__ sf, int64_t n) {
+  const float beta = __fsub_rn(1.0f, alpha);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float ai = a[i];
+    float nh;
+    if (policy == 0) {
+      nh = ai;
+    } else if (policy == 1) {
+      nh = __fadd_rn(__fmul_rn(alpha, h[i]), __fmul_rn(beta, ai));
+    } else {
+      nh = fmaxf(ai, __fmul_rn(alpha, h[i]));
+    }
+    h[i] = nh;
+    sf[i] = tile_scale(nh);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 128x1 tiles along the token dimension, written transposed.  A 256-thread
 // block stages 128-token x 128-channel BF16 tiles (32 KB) in shared memory
 // with cp.async, double-buffered so the next tile's copy overlaps this one's

@@ -53,6 +53,13 @@ enum {
   FP8Q_SFB_ROW = 1       /* one scale per row and K chunk: sfb[kb * ld_sfb + n], ld_sfb >= N */
 };
 
+/* Scale-history policies of fp8q_scale_history_update. */
+enum {
+  FP8Q_POLICY_PREVIOUS = 0,    /* delayed: the previous step's tile maximum  */
+  FP8Q_POLICY_EMA = 1,         /* exponential history of tile maxima         */
+  FP8Q_POLICY_DECAYED_MAX = 2  /* running maximum that decays by alpha       */
+};
+
 /* Output element types of the GEMMs. */
 enum {
   FP8Q_OUT_BF16 = 0, /* round-to-nearest-even BF16 */
@@ -114,6 +121,43 @@ fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K,
                                         const int32_t* rows, int64_t M,
                                         void* q, int64_t ldq, float* sf, int64_t ld_sf,
                                         void* stream);
+
+/*
+ * 1x128 quantization with GIVEN tile scales -- a scale policy's (fixed
+ * calibration, delayed, or a tile-maximum history) instead of the tiles' own
+ * maxima.  "Online Quantization During Training", section 4 "Max scaling is
+ * robust but noisy" and its worked example; "Introduction to LLM
+ * Quantization", "5) Online Quantization", delayed quantization.
+ *
+ *   x      : BF16 [M][ldx].
+ *   sf     : FP32 scales to apply, sf[(k/128) * ld_sf + m] (the layout
+ *            fp8q_quant_act_1x128 writes), ld_sf >= M.
+ *   q      : E4M3 [M][ldq], q = e4m3(fl32(x / s)) (IEEE division, RNE,
+ *            saturating at +-448).
+ *   amax   : optional FP32 [K/128][ld_amax]: each tile's current maximum
+ *            |x| (the input of fp8q_scale_history_update); NULL to skip.
+ *   clipped: optional device counter (8-byte aligned): += the number of
+ *            elements the cast saturated, |fl32(x / s)| > 464; NULL to skip.
+ * Requirements: as fp8q_quant_act_1x128, plus ld_amax >= M when amax is given.
+ */
+fp8q_status fp8q_quant_act_1x128_scaled(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                        const float* sf, int64_t ld_sf, void* q, int64_t ldq,
+                                        float* amax, int64_t ld_amax, unsigned long long* clipped,
+                                        void* stream);
+
+/*
+ * One step of a per-tile scale history (same passages as above): for each of
+ * the n tiles, hist <- policy(hist, amax) and sf <- max(fl32(hist / 448),
+ * fl32(1e-12)), the scale the next step's fp8q_quant_act_1x128_scaled uses.
+ *   FP8Q_POLICY_PREVIOUS    : hist = amax
+ *   FP8Q_POLICY_EMA         : hist = fl32(fl32(alpha*hist) + fl32(fl32(1-alpha)*amax))
+ *   FP8Q_POLICY_DECAYED_MAX : hist = max(amax, fl32(alpha*hist))
+ * Each product and sum is rounded to FP32 on its own.
+ *   amax, hist, sf : device FP32 [n] (hist updated in place).
+ * Requirements: 0 <= alpha <= 1, n >= 0; pointers 4-byte aligned.
+ */
+fp8q_status fp8q_scale_history_update(int policy, float alpha, const float* amax, float* hist,
+                                      float* sf, int64_t n, void* stream);
 
 /*
  * Online 128x1 quantization along the token dimension, written transposed:

@@ -17,8 +17,14 @@ ROW_REL_TOL = 1e-3
 
 
 def load_fp8q():
-    """Import the CUDA binding, building libfp8q.so in-tree first if needed."""
-    from fine_grained_fp8_x128_b200 import build as _b
+    """Import the CUDA binding, building libfp8q.so in-tree first if needed
+    (build.py is loaded by path: importing the package would load the old library)."""
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("fp8q_build", os.path.join(root, "fine_grained_fp8_x128_b200", "build.py"))
+    _b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(_b)
     _b.build()
     import fine_grained_fp8_x128_b200 as fp8q
     return fp8q

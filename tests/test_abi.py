@@ -80,6 +80,25 @@ def test_quant_gather_validation(fp8q):
     assert qg(M=0, rows=None, q=None, sf=None, ld_sf=0) == 0    # no output rows: nothing launched
 
 
+def test_scale_policy_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+
+    def qs(M=8, K=256, ldx=256, sf=FAKE, ld_sf=8, q=FAKE, ldq=256, amax=FAKE, ld_amax=8, clipped=FAKE):
+        return L.fp8q_quant_act_1x128_scaled(FAKE, M, K, ldx, sf, ld_sf, q, ldq, amax, ld_amax, clipped, None)
+
+    assert qs(K=200) == INV and qs(ld_sf=4) == INV and qs(ld_amax=4) == INV and qs(ldq=128) == INV
+    assert qs(sf=None) == INV and qs(q=None) == INV
+    assert qs(sf=FAKE + 2) == ALN and qs(clipped=FAKE + 4) == ALN and qs(ldq=264) == ALN
+    assert qs(M=0, sf=None, q=None, amax=None, clipped=None, ld_sf=0, ld_amax=0) == 0
+    U = L.fp8q_scale_history_update
+    assert U(3, 0.5, FAKE, FAKE, FAKE, 16, None) == INV and U(-1, 0.5, FAKE, FAKE, FAKE, 16, None) == INV
+    assert U(1, 1.5, FAKE, FAKE, FAKE, 16, None) == INV and U(1, -0.1, FAKE, FAKE, FAKE, 16, None) == INV
+    assert U(1, float("nan"), FAKE, FAKE, FAKE, 16, None) == INV
+    assert U(1, 0.5, None, FAKE, FAKE, 16, None) == INV and U(1, 0.5, FAKE + 2, FAKE, FAKE, 16, None) == ALN
+    assert U(2, 0.5, None, None, None, 0, None) == 0
+
+
 def test_quant_w_validation(fp8q):
     L = fp8q.lib()
     INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
