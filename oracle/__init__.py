@@ -61,6 +61,7 @@ def _load():
     lib.orc_quant_act_1x128.argtypes = [P, I64, I64, I64, P, I64, P]
     lib.orc_quant_act_1x128_scaled.argtypes = [P, I64, I64, I64, P, P, I64, P, P]
     lib.orc_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, P, P, P, I64]
+    lib.orc_quant_act_1x128_percentile.argtypes = [P, I64, I64, I64, ctypes.c_int, P, I64, P, P]
     lib.orc_quant_act_128x1.argtypes = [P, I64, I64, I64, P, I64, P]
     lib.orc_quant_w_128x128.argtypes = [P, I64, I64, I64, P, I64, P]
     lib.orc_quant_tiles_intgrid.argtypes = [P, I64, I64, P]
@@ -230,6 +231,29 @@ def quant_act_1x128_scaled(x_bf16: np.ndarray, sf: np.ndarray):
     return q, amax, int(clipped.value)
 
 
+def percentile_rank(p: float, n: int = 128) -> int:
+    """The nearest-rank p-th percentile (0 < p <= 1) of n values is the
+    ceil(p*n)-th smallest, i.e. the r-th largest with r = n - ceil(p*n) + 1."""
+    if not 0.0 < p <= 1.0:
+        raise ValueError("percentile must lie in (0, 1]")
+    return n - int(np.ceil(p * n)) + 1
+
+
+def quant_act_1x128_percentile(x_bf16: np.ndarray, rank: int):
+    """Percentile clipping per 1x128 tile: s from the rank-th largest magnitude
+    (rank 1 = the online rule).  Returns (q uint8 [M][K], sf float32 [M][K/128],
+    clipped = number of saturated elements, |fl32(x / s)| > 464)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    sf = np.empty((M, K // 128), np.float32)
+    clipped = ctypes.c_int64(0)
+    _check(_load().orc_quant_act_1x128_percentile(_p(x), M, K, K, int(rank), _p(q), K, _p(sf),
+                                                  ctypes.cast(ctypes.pointer(clipped), ctypes.c_void_p)),
+           "quant_act_1x128_percentile")
+    return q, sf, int(clipped.value)
+
+
 def scale_history_update(policy: int, alpha: float, amax: np.ndarray, hist: np.ndarray):
     """One history step for each tile: returns (new history, next scales), float32."""
     a = np.ascontiguousarray(amax, dtype=np.float32)
@@ -240,12 +264,12 @@ def scale_history_update(policy: int, alpha: float, amax: np.ndarray, hist: np.n
     return h, sf
 
 
-def scale_policy_drift(tiles_bf16: np.ndarray, alpha: float = 0.9):
+def scale_policy_drift(tiles_bf16: np.ndarray, alpha: float = 0.9, percentile: float = 0.99):
     """The [P1] worked example on the oracle: one 1x128 tile per step
     (tiles_bf16 [steps][128], e.g. a standard deviation doubling over the steps
-    with a rare outlier) quantized under five policies -- current-max (online),
+    with a rare outlier) quantized under six policies -- current-max (online),
     fixed calibration (the first step's scale), previous-step delayed, EMA
-    history and decaying maximum.  Returns {policy: (clip_rate [steps],
+    history, decaying maximum and percentile clipping of the current tile.  Returns {policy: (clip_rate [steps],
     mean_rel_err [steps])}: the fraction of clipped elements, and
     mean |dequant - x| / mean |x| of each step's tile."""
     x = np.ascontiguousarray(tiles_bf16, dtype=np.uint16)
@@ -266,6 +290,13 @@ def scale_policy_drift(tiles_bf16: np.ndarray, alpha: float = 0.9):
         _, s = quant_act_1x128(x[t:t + 1])
         cr[t], er[t], _ = measure(t, s[0, 0])
     out["current_max"] = (cr, er)
+    # percentile clipping: each step's own tile, scaled from an upper percentile
+    r = percentile_rank(percentile)
+    cr, er = np.zeros(steps), np.zeros(steps)
+    for t in range(steps):
+        _, s, _ = quant_act_1x128_percentile(x[t:t + 1], r)
+        cr[t], er[t], _ = measure(t, s[0, 0])
+    out["percentile"] = (cr, er)
     # fixed calibration: the first step's scale for every step
     _, s0 = quant_act_1x128(x[0:1])
     cr, er = np.zeros(steps), np.zeros(steps)

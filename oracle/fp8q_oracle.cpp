@@ -559,4 +559,38 @@ int orc_scale_history_update(int policy, float alpha, const float* a, float* h, 
   return 0;
 }
 
+// Percentile clipping ([P1] "4. Max scaling is robust but noisy" names it
+// beside delayed scaling and amax histories): the tile's scale comes from an
+// upper percentile of its magnitudes instead of their maximum, so the few
+// values above it saturate.  Reading: the p-th percentile of the tile's 128
+// magnitudes by the nearest-rank rule, i.e. the r-th largest magnitude with
+// r = 128 - ceil(p * 128) + 1; the call takes r (1 <= r <= 128) and r = 1 is
+// the online rule.  s = max(fl32(v / 448), fl32(1e-12)) with v that magnitude;
+// the cast, the IEEE division and the clip rule are those of the given-scale
+// quantizer above.
+// x: bf16 [M][ldx]; q: [M][ldq]; sf: [M][K/128]; *clipped += clipped count.
+int orc_quant_act_1x128_percentile(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int rank,
+                                   uint8_t* q, int64_t ldq, float* sf, int64_t* clipped) {
+  if (K % 128 != 0 || ldx < K || ldq < K || M < 0 || rank < 1 || rank > 128) return 1;
+  const int64_t KB = K / 128;
+  int64_t total = 0;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t kb = 0; kb < KB; ++kb) {
+      const uint16_t* t = x + m * ldx + kb * 128;
+      float mags[128];
+      for (int i = 0; i < 128; ++i) mags[i] = std::fabs(bf16_to_float(t[i]));
+      std::sort(mags, mags + 128, [](float a, float b) { return a > b; });   // descending
+      const float s = orc_tile_scale(mags[rank - 1]);
+      sf[m * KB + kb] = s;
+      for (int i = 0; i < 128; ++i) {
+        const float v = bf16_to_float(t[i]) / s;
+        if (std::fabs(v) > 464.0f) ++total;
+        q[m * ldq + kb * 128 + i] = e4m3_encode(v);
+      }
+    }
+  }
+  if (clipped != nullptr) *clipped += total;
+  return 0;
+}
+
 }  // extern "C"

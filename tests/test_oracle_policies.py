@@ -99,3 +99,80 @@ def test_drift_simulation_matches_the_pages_claims():
     # values well inside the normal range, so current-max loses little there
     neighbours = np.r_[err_cur[t_out - 3:t_out], err_cur[t_out + 1:t_out + 4]]
     assert err_cur[t_out] < 2 * neighbours.mean()
+
+
+# ---------------------------------------------------------------- percentile clipping
+def _nearest_rank_scales(xf_tiles, p):
+    """Per tile: v = NumPy's nearest-rank percentile (Hyndman-Fan type 1,
+    'inverted_cdf') of the magnitudes, then the online scale rule on v."""
+    v = np.percentile(np.abs(xf_tiles), 100.0 * p, axis=-1, method="inverted_cdf")
+    return np.vectorize(oracle.tile_scale, otypes=[np.float32])(v.astype(np.float32))
+
+
+def test_percentile_rank_is_the_nearest_rank_rule():
+    assert oracle.percentile_rank(1.0) == 1
+    assert oracle.percentile_rank(0.99) == 2          # ceil(126.72) = 127th smallest of 128
+    assert oracle.percentile_rank(0.5) == 65
+    assert oracle.percentile_rank(1 / 128) == 128     # the smallest value
+    vals = np.random.default_rng(1).permutation(128).astype(np.float64)
+    for p in (0.9, 0.95, 0.99, 0.999, 0.5, 0.01):
+        r = oracle.percentile_rank(p)
+        assert np.percentile(vals, 100 * p, method="inverted_cdf") == np.sort(vals)[::-1][r - 1]
+    with pytest.raises(ValueError):
+        oracle.percentile_rank(0.0)
+
+
+def test_percentile_rank_one_is_the_online_quantizer():
+    x = W.activations_with_outliers(24, 512, seed=8, channel_frac=2 / 512, elem_frac=1e-2)
+    q_on, sf_on = oracle.quant_act_1x128(x)
+    q, sf, clipped = oracle.quant_act_1x128_percentile(x, 1)
+    assert np.array_equal(q, q_on) and np.array_equal(sf, sf_on) and clipped == 0
+
+
+@pytest.mark.parametrize("p", [0.99, 0.95, 0.9, 0.5])
+def test_percentile_against_numpy(p):
+    """Scales from NumPy's nearest-rank percentile, codes from NumPy's float32
+    division and the codec, the clip count by brute force."""
+    M, K = 20, 384
+    x = W.activations_with_outliers(M, K, seed=9, channel_frac=0, elem_frac=2e-2)
+    r = oracle.percentile_rank(p)
+    q, sf, clipped = oracle.quant_act_1x128_percentile(x, r)
+    xf = W.bf16_bits_to_f32(x).reshape(M, K // 128, 128)
+    s_np = _nearest_rank_scales(xf, p)
+    assert np.array_equal(sf, s_np)
+    v = (xf / s_np[:, :, None]).astype(np.float32)
+    assert np.array_equal(q, oracle.e4m3_encode(v.reshape(M, K)))
+    per_tile = (np.abs(v) > 464.0).sum(axis=2)
+    assert clipped == int(per_tile.sum())
+    assert np.all(per_tile <= r - 1)                  # only values above the r-th largest can saturate
+
+
+def test_percentile_ties_and_single_outlier():
+    # all-equal tile: every rank gives the same scale and nothing clips
+    x = np.full((1, 128), 0x3F80, np.uint16)          # 1.0
+    for r in (1, 2, 64, 128):
+        q, sf, clipped = oracle.quant_act_1x128_percentile(x, r)
+        assert sf[0, 0] == oracle.tile_scale(1.0) and clipped == 0 and np.all(q == 0x7E)
+    # one 20x outlier among values of magnitude <= 1: rank 2 clamps exactly it
+    rng = np.random.default_rng(4)
+    xf = rng.uniform(-1.0, 1.0, 128).astype(np.float32)
+    xf[37] = -20.0
+    xb = (xf.view(np.uint32) >> 16).astype(np.uint16)[None, :]
+    q, sf, clipped = oracle.quant_act_1x128_percentile(xb, 2)
+    assert clipped == 1 and q[0, 37] == 0xFE
+    second = np.sort(np.abs(W.bf16_bits_to_f32(xb)[0]))[-2]
+    assert sf[0, 0] == oracle.tile_scale(second)
+
+
+def test_percentile_in_the_drift_run():
+    """Clipping the current tile's top value protects the rest of the tile's
+    grid but clamps the 20-sigma outlier itself: on an E4M3 grid that costs
+    more than it saves (the online maximum keeps the lower error)."""
+    tiles, t_out = W.drift_tiles(steps=100, seed=0)
+    res = oracle.scale_policy_drift(tiles, alpha=0.9, percentile=0.99)
+    clip, err = res["percentile"]
+    _, err_cur = res["current_max"]
+    assert clip[t_out] == 1 / 128
+    assert err[t_out] > 5 * err_cur[t_out]
+    assert err.mean() > err_cur.mean()
+    assert np.all(clip <= 1 / 128)                    # rank 2: at most one element per tile
