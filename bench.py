@@ -648,7 +648,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -670,7 +670,7 @@ def run_single(args):
     ld = fp8q.sf_ld
     u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
     work = None
-    if name in ("quant_x", "quant_x_scaled", "quant_x_t"):
+    if name in ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_t"):
         x = randn(T, HID)
         if name == "quant_x_scaled":
             # a scale policy's pass: given scales (here the online ones), tile maxima and clip count out
@@ -679,6 +679,11 @@ def run_single(args):
             amax = torch.empty_like(sf)
             clipped = torch.zeros(1, dtype=torch.int64, device=dev)
             fn = lambda: fp8q.fp8q_quant_act_1x128_scaled(x, sf, q, amax, clipped)
+        elif name == "quant_x_pct":
+            # percentile clipping: the scale from each tile's rank-th largest magnitude
+            q = torch.empty((T, HID), dtype=u8, device=dev); sf = torch.empty((HID // 128, ld(T)), dtype=f32, device=dev)
+            clipped = torch.zeros(1, dtype=torch.int64, device=dev)
+            fn = lambda: fp8q.fp8q_quant_act_1x128_percentile(x, args.rank, q, sf, clipped)
         elif name == "quant_x":
             q = torch.empty((T, HID), dtype=u8, device=dev); sf = torch.empty((HID // 128, ld(T)), dtype=f32, device=dev)
             fn = lambda: fp8q.fp8q_quant_act_1x128(x, q, sf)
@@ -773,6 +778,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--single", choices=SINGLE_KERNELS, help="time one kernel alone (not the bench line)")
     ap.add_argument("--tokens", type=int, default=TOK, help="token count for --single")
+    ap.add_argument("--rank", type=int, default=2, help="rank for --single quant_x_pct (2 = 99th percentile)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

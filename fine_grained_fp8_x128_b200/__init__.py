@@ -42,7 +42,7 @@ FP8Q_OUT_F32 = 1
 EXPORTS = (
     "fp8q_version", "fp8q_status_string", "fp8q_device_status",
     "fp8q_quant_act_1x128", "fp8q_quant_act_1x128_gather", "fp8q_quant_act_1x128_scaled",
-    "fp8q_scale_history_update", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
+    "fp8q_quant_act_1x128_percentile", "fp8q_scale_history_update", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
     "fp8q_gemm_blockscaled", "fp8q_gemm_blockscaled_q1x128",
     "fp8q_grouped_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled_q1x128",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
@@ -57,6 +57,7 @@ _lib.fp8q_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int)]
 _lib.fp8q_quant_act_1x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_gather.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scaled.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]
+_lib.fp8q_quant_act_1x128_percentile.argtypes = [_P, _I, _I, _I, ctypes.c_int, _P, _I, _P, _I, _P, _P]
 _lib.fp8q_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, _P, _P, _P, _I, _P]
 _lib.fp8q_quant_act_128x1.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_w_128x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P]
@@ -146,6 +147,15 @@ def fp8q_quant_act_1x128_scaled(x, sf, q, amax=None, clipped=None, stream=None):
     _check(_lib.fp8q_quant_act_1x128_scaled(_ptr(x), M, K, _ld(x), _ptr(sf), _ld(sf), _ptr(q), _ld(q), _ptr(amax),
                                             _ld(amax) if amax is not None else 0, _ptr(clipped), _stream(stream)),
            "fp8q_quant_act_1x128_scaled")
+
+
+def fp8q_quant_act_1x128_percentile(x, rank, q, sf, clipped=None, stream=None):
+    """Percentile clipping per 1x128 tile: sf [K/128][ld >= M] from each tile's
+    rank-th largest magnitude (rank 1 = the online rule), q = e4m3(x / sf);
+    optional clipped (int64 device counter, += saturated elements)."""
+    M, K = x.shape
+    _check(_lib.fp8q_quant_act_1x128_percentile(_ptr(x), M, K, _ld(x), int(rank), _ptr(q), _ld(q), _ptr(sf), _ld(sf),
+                                                _ptr(clipped), _stream(stream)), "fp8q_quant_act_1x128_percentile")
 
 
 def fp8q_scale_history_update(policy, alpha, amax, hist, sf, stream=None):

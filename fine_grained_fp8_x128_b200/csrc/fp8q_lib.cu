@@ -33,6 +33,7 @@ struct DeviceInfo {
   int q1_per_sm = 0;               // resident blocks per SM of each quantizer
   int q1g_per_sm = 0;
   int q1s_per_sm = 0;
+  int q1p_per_sm = 0;
   int q2_per_sm = 0;
   int qw_per_sm = 0;
 };
@@ -442,6 +443,29 @@ fp8q_status fp8q_quant_act_1x128_scaled(const void* x, int64_t M, int64_t K, int
                                         static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, sf, ld_sf, static_cast<uint8_t*>(q), ldq, amax, ld_amax,
       clipped);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_act_1x128_percentile(const void* x, int64_t M, int64_t K, int64_t ldx, int rank, void* q,
+                                            int64_t ldq, float* sf, int64_t ld_sf, unsigned long long* clipped,
+                                            void* stream) {
+  if (M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M || rank < 1 || rank > 128)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldq % 16 != 0 ||
+      (clipped != nullptr && !aligned(clipped, 8)))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  const int per_sm = blocks_per_sm(&dev->q1p_per_sm, fp8q::quant_act_1x128_percentile_kernel, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  fp8q::quant_act_1x128_percentile_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0,
+                                            static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, rank, static_cast<uint8_t*>(q), ldq, sf, ld_sf, clipped);
   return launch_status();
 }
 

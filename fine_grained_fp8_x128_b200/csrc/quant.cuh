@@ -195,6 +195,130 @@ quant_act_1x128_scaled_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, in
   }
 }
 
+// ---------------------------------------------------------------------------
+// Percentile clipping ("Online Quantization During Training", section 4): the
+// tile's scale comes from its rank-th largest magnitude v (nearest-rank
+// percentile; rank 1 is the online rule), s = max(fl32(v/448), fl32(1e-12)),
+// and the values above v saturate.  Same tiling as quant_act_1x128_kernel.
+//
+// Selection: BF16 magnitudes order like their 15-bit patterns, so the four
+// lanes of a tile walk the distinct magnitudes downwards from the maximum g:
+// each round counts #(|x| >= g) and finds the largest magnitude below g, two
+// 16x2 packed operations per word (bit 15 of (mag | 0x8000) - g is set exactly
+// when mag >= g, with no borrow between the halves).  The walk stops at the
+// first g whose count reaches rank, which is the rank-th largest magnitude.
+// Every round raises the count by at least one, so it ends within rank rounds;
+// the warp loops until all of its tiles are done, which keeps the shuffles
+// warp-uniform.
+//
+// Cast: |x| <= v is cast without division (exact for every BF16 x, v with
+// |x| <= v and s = tile_scale(v)) and never saturates.  A lane holding values
+// above v recasts them from the IEEE quotient fl32(x / s) (which the 1e-12
+// floor of s can keep small, and which can overflow to infinity: it is clamped
+// to +-448 first) and counts those with |fl32(x / s)| > 464 as clipped.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t slice_rank_walk(const Q1Slice& d, uint32_t g, uint32_t* next) {
+  const uint32_t gg = g * 0x00010001u;
+  uint32_t cnt2 = 0, nm = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {d.v[i].x, d.v[i].y, d.v[i].z, d.v[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t ge = ((w[j] | 0x80008000u) - gg) & 0x80008000u;   // bit 15/31: mag >= g
+      const uint32_t one = ge >> 15;
+      cnt2 += one;
+      const uint32_t below = w[j] & ~(ge - one) & 0x7FFF7FFFu;          // magnitudes < g, else 0
+      asm("max.u16x2 %0, %0, %1;" : "+r"(nm) : "r"(below));
+    }
+  }
+  *next = max(nm & 0xFFFFu, nm >> 16);
+  return (cnt2 & 0xFFFFu) + (cnt2 >> 16);
+}
+
+__global__ void __launch_bounds__(kQ1Threads)
+quant_act_1x128_percentile_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx, int rank,
+                                  uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
+                                  unsigned long long* __restrict__ clipped) {
+  const int tid = threadIdx.x;
+  const int sub = tid & 3;
+  const int tile = tid >> 2;
+  const int64_t items = ((M + kQ1Rows - 1) / kQ1Rows) * KB;
+  int64_t it = blockIdx.x;
+  unsigned int nclip = 0;
+  if (it < items) {
+    Q1Slice cur, nxt;
+    q1_load<false>(cur, x, M, KB, ldx, nullptr, 0, it, tile, sub);
+    for (; it < items; it += gridDim.x) {
+      const int64_t it_next = it + gridDim.x;
+      if (it_next < items) q1_load<false>(nxt, x, M, KB, ldx, nullptr, 0, it_next, tile, sub);
+      const int64_t rb = it / KB;
+      const int64_t kb = it - rb * KB;
+      const int64_t row = rb * kQ1Rows + tile;
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        m2 = amax2(m2, cur.v[i].x); m2 = amax2(m2, cur.v[i].y);
+        m2 = amax2(m2, cur.v[i].z); m2 = amax2(m2, cur.v[i].w);
+      }
+      const uint32_t lane_max = max(m2 & 0xFFFFu, m2 >> 16);
+      uint32_t g = max(lane_max, __shfl_xor_sync(0xFFFFFFFFu, lane_max, 1));
+      g = max(g, __shfl_xor_sync(0xFFFFFFFFu, g, 2));
+      bool done = rank <= 1;
+      for (int round = 0; round < 128; ++round) {
+        if (__all_sync(0xFFFFFFFFu, done)) break;
+        uint32_t next;
+        uint32_t cnt = slice_rank_walk(cur, g, &next);
+        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 1);
+        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 2);
+        next = max(next, __shfl_xor_sync(0xFFFFFFFFu, next, 1));
+        next = max(next, __shfl_xor_sync(0xFFFFFFFFu, next, 2));
+        if (!done) {
+          if (cnt >= static_cast<uint32_t>(rank)) done = true;
+          else g = next;
+        }
+      }
+      const float s = tile_scale(__uint_as_float(g << 16));
+      const float nr = -__frcp_rn(s);
+      if (row < M) {
+        uint2 o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          o[i].x = quant_words(cur.v[i].x, cur.v[i].y, nr, s);
+          o[i].y = quant_words(cur.v[i].z, cur.v[i].w, nr, s);
+        }
+        if (lane_max > g) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t w[4] = {cur.v[i].x, cur.v[i].y, cur.v[i].z, cur.v[i].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t bits = (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+              if ((bits & 0x7FFFu) > g) {
+                const float qv = __fdiv_rn(__uint_as_float(bits << 16), s);
+                nclip += fabsf(qv) > 464.0f;
+                const uint32_t code = cvt_e4m3x2(fminf(fmaxf(qv, -448.0f), 448.0f), 0.0f) & 0xFFu;
+                uint32_t& word = (e < 4) ? o[i].x : o[i].y;
+                const int sh = 8 * (e & 3);
+                word = (word & ~(0xFFu << sh)) | (code << sh);
+              }
+            }
+          }
+        }
+        uint8_t* dst = q + row * ldq + kb * 128 + sub * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2*>(dst + 32 * i) = o[i];
+        if (sub == 0) sf[kb * ld_sf + row] = s;
+      }
+      cur = nxt;
+    }
+  }
+  if (clipped != nullptr) {
+    const unsigned int warp_clip = __reduce_add_sync(0xFFFFFFFFu, nclip);
+    if ((tid & 31) == 0 && warp_clip != 0) atomicAdd(clipped, static_cast<unsigned long long>(warp_clip));
+  }
+}
+
 // One history step per tile: h <- policy(h, amax), sf <- max(fl32(h / 448),
 // fl32(1e-12)).  Policies: 0 previous step (h = a), 1 exponential history
 // (h = fl32(fl32(alpha*h) + fl32(fl32(1 - alpha)*a))), 2 decaying maximum

@@ -146,6 +146,28 @@ fp8q_status fp8q_quant_act_1x128_scaled(const void* x, int64_t M, int64_t K, int
                                         void* stream);
 
 /*
+ * 1x128 quantization with percentile clipping: each tile's scale comes from
+ * its rank-th largest magnitude v instead of its maximum, so the rank-1
+ * values above v saturate ("Online Quantization During Training", section 4
+ * "Max scaling is robust but noisy", percentile clipping).  The p-th
+ * percentile of a tile by the nearest-rank rule is rank = 128 - ceil(128 p) + 1;
+ * rank 1 gives exactly fp8q_quant_act_1x128.
+ *
+ *   x      : BF16 [M][ldx], finite values.
+ *   rank   : 1..128; anything else is FP8Q_ERR_INVALID_ARG.
+ *   q, sf  : as fp8q_quant_act_1x128, with s = max(fl32(v / 448), fl32(1e-12));
+ *            q = e4m3(fl32(x / s)) (RNE, saturating at +-448).
+ *   clipped: optional device counter (8-byte aligned): += the number of
+ *            elements with |fl32(x / s)| > 464; NULL to skip.
+ * Run time grows with rank (one pass over the tile's registers per distinct
+ * magnitude above v); the policy is meant for ranks of a few.
+ * Requirements: as fp8q_quant_act_1x128.
+ */
+fp8q_status fp8q_quant_act_1x128_percentile(const void* x, int64_t M, int64_t K, int64_t ldx, int rank,
+                                            void* q, int64_t ldq, float* sf, int64_t ld_sf,
+                                            unsigned long long* clipped, void* stream);
+
+/*
  * One step of a per-tile scale history (same passages as above): for each of
  * the n tiles, hist <- policy(hist, amax) and sf <- max(fl32(hist / 448),
  * fl32(1e-12)), the scale the next step's fp8q_quant_act_1x128_scaled uses.

@@ -91,6 +91,13 @@ def test_scale_policy_validation(fp8q):
     assert qs(sf=None) == INV and qs(q=None) == INV
     assert qs(sf=FAKE + 2) == ALN and qs(clipped=FAKE + 4) == ALN and qs(ldq=264) == ALN
     assert qs(M=0, sf=None, q=None, amax=None, clipped=None, ld_sf=0, ld_amax=0) == 0
+    def qp(M=64, K=256, ldx=256, rank=2, q=FAKE, ldq=256, sf=FAKE, ld_sf=64, clipped=None):
+        return L.fp8q_quant_act_1x128_percentile(FAKE, M, K, ldx, rank, q, ldq, sf, ld_sf, clipped, None)
+
+    assert qp(rank=0) == INV and qp(rank=129) == INV and qp(rank=-3) == INV
+    assert qp(K=200) == INV and qp(ld_sf=4) == INV and qp(ldq=128) == INV and qp(sf=None) == INV
+    assert qp(ldq=264) == ALN and qp(clipped=FAKE + 4) == ALN and qp(sf=FAKE + 2) == ALN
+    assert qp(M=0, q=None, sf=None, ld_sf=0) == 0
     U = L.fp8q_scale_history_update
     assert U(3, 0.5, FAKE, FAKE, FAKE, 16, None) == INV and U(-1, 0.5, FAKE, FAKE, FAKE, 16, None) == INV
     assert U(1, 1.5, FAKE, FAKE, FAKE, 16, None) == INV and U(1, -0.1, FAKE, FAKE, FAKE, 16, None) == INV
