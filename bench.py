@@ -648,7 +648,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -670,7 +670,22 @@ def run_single(args):
     ld = fp8q.sf_ld
     u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
     work = None
-    if name in ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_t"):
+    if name == "quant_x_pt":
+        # per-tensor baseline quantizer: amax pass + cast pass (reads x twice)
+        x = randn(T, HID)
+        q = torch.empty((T, HID), dtype=u8, device=dev)
+        amax_scale = torch.empty(2, dtype=f32, device=dev)
+        fn = lambda: fp8q.fp8q_quant_pertensor(x, q, amax_scale)
+        work = ("bytes", T * HID * 3)
+    elif name == "pt_fprop":
+        # per-tensor baseline GEMM at the Fprop shape: one TMEM accumulation over K, no promotion
+        M, N, K = T, OUT, HID
+        qa, sa = fp8q.quant_pertensor(randn(M, K))
+        qb, sb = fp8q.quant_pertensor(randn(N, K, sigma=0.02))
+        d = torch.empty((M, N), dtype=bf, device=dev)
+        fn = lambda: fp8q.fp8q_gemm_pertensor(qa, sa[1:2], qb, sb[1:2], d)
+        work = ("flops", 2.0 * M * N * K)
+    elif name in ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_t"):
         x = randn(T, HID)
         if name == "quant_x_scaled":
             # a scale policy's pass: given scales (here the online ones), tile maxima and clip count out

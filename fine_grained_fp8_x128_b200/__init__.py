@@ -45,6 +45,7 @@ EXPORTS = (
     "fp8q_quant_act_1x128_percentile", "fp8q_scale_history_update", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
     "fp8q_gemm_blockscaled", "fp8q_gemm_blockscaled_q1x128",
     "fp8q_grouped_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled_q1x128",
+    "fp8q_quant_pertensor", "fp8q_gemm_pertensor",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
 )
 
@@ -58,6 +59,8 @@ _lib.fp8q_quant_act_1x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_gather.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scaled.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]
 _lib.fp8q_quant_act_1x128_percentile.argtypes = [_P, _I, _I, _I, ctypes.c_int, _P, _I, _P, _I, _P, _P]
+_lib.fp8q_quant_pertensor.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
+_lib.fp8q_gemm_pertensor.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_int, _I, _I, _I, _P]
 _lib.fp8q_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, _P, _P, _P, _I, _P]
 _lib.fp8q_quant_act_128x1.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_w_128x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P]
@@ -190,6 +193,22 @@ def fp8q_gemm_blockscaled(a, sfa, b, sfb, sfb_mode, d, stream=None):
            "fp8q_gemm_blockscaled")
 
 
+def fp8q_quant_pertensor(x, q, amax_scale, stream=None):
+    """Per-tensor baseline: amax_scale float32 [2] <- {max|x|, s}, q = e4m3(x / s)."""
+    M, K = x.shape
+    _check(_lib.fp8q_quant_pertensor(_ptr(x), M, K, _ld(x), _ptr(q), _ld(q), _ptr(amax_scale), _stream(stream)),
+           "fp8q_quant_pertensor")
+
+
+def fp8q_gemm_pertensor(a, scale_a, b, scale_b, d, stream=None):
+    """d[M][N] = (*scale_a * *scale_b) * a[M][K] . b[N][K]^T, one TMEM accumulation over K."""
+    M, K = a.shape
+    N = b.shape[0]
+    dt = FP8Q_OUT_F32 if d.dtype == torch.float32 else FP8Q_OUT_BF16
+    _check(_lib.fp8q_gemm_pertensor(_ptr(a), _ld(a), _ptr(scale_a), _ptr(b), _ld(b), _ptr(scale_b), _ptr(d), _ld(d),
+                                    dt, M, N, K, _stream(stream)), "fp8q_gemm_pertensor")
+
+
 def fp8q_gemm_blockscaled_q1x128(a, sfa, b, sfb, dq, sfd, stream=None):
     """dq[M][N] uint8, sfd [N/128][ld >= M]: 1x128 quantization of the bf16 GEMM result."""
     M, K = a.shape
@@ -239,6 +258,15 @@ def quant_act_1x128(x, stream=None):
     sf = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=x.device)
     fp8q_quant_act_1x128(x, q, sf, stream)
     return q, sf
+
+
+def quant_pertensor(x, stream=None):
+    """Returns (q uint8 [M][K], amax_scale float32 [2] = {amax, s}) on x's device."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    amax_scale = torch.empty(2, dtype=torch.float32, device=x.device)
+    fp8q_quant_pertensor(x, q, amax_scale, stream)
+    return q, amax_scale
 
 
 def quant_act_128x1(x, stream=None):

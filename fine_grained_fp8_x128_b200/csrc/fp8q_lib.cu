@@ -15,6 +15,7 @@
 #include "device_common.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_pertensor.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -29,11 +30,15 @@ struct DeviceInfo {
   bool gemm_attr[2][2][3] = {};   // [grouped][row mode][output mode]
   bool q2_attr = false;
   bool pair_attr[2][3] = {};       // [row mode][output mode]
+  bool pt_attr[2] = {};            // per-tensor GEMM [output mode]
+  int pt_clusters[2] = {};
   int pair_clusters[2][3] = {};    // co-resident CTA pairs per kernel instance
   int q1_per_sm = 0;               // resident blocks per SM of each quantizer
   int q1g_per_sm = 0;
   int q1s_per_sm = 0;
   int q1p_per_sm = 0;
+  int pt_amax_per_sm = 0;
+  int pt_cast_per_sm = 0;
   int q2_per_sm = 0;
   int qw_per_sm = 0;
 };
@@ -182,6 +187,43 @@ fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUten
   const int64_t clusters = pair_tiles < dev->pair_clusters[mi][fi] ? pair_tiles : dev->pair_clusters[mi][fi];
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return launch_status();
+}
+
+// The per-tensor baseline GEMM: the same cluster launch as the pair kernel.
+template <int OUT>
+fp8q_status launch_gemm_pertensor(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb,
+                                  const fp8q::GemmArgs& args, const float* sa, const float* sb, int64_t pair_tiles,
+                                  cudaStream_t stream) {
+  const uint32_t smem = fp8q::PtSmemLayout::bytes + 1024;
+  auto kern = fp8q::gemm_pertensor_pair_kernel<OUT>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(fp8q::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!dev->pt_attr[OUT]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      cfg.gridDim = dim3(2 * (dev->sm_count / 2), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = dev->sm_count / 2;
+      dev->pt_clusters[OUT] = n;
+      dev->pt_attr[OUT] = true;
+    }
+  }
+  const int64_t clusters = pair_tiles < dev->pt_clusters[OUT] ? pair_tiles : dev->pt_clusters[OUT];
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args, sa, sb) != cudaSuccess) return FP8Q_ERR_CUDA;
   return launch_status();
 }
 
@@ -467,6 +509,75 @@ fp8q_status fp8q_quant_act_1x128_percentile(const void* x, int64_t M, int64_t K,
                                             static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, rank, static_cast<uint8_t*>(q), ldq, sf, ld_sf, clipped);
   return launch_status();
+}
+
+fp8q_status fp8q_quant_pertensor(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
+                                 float* amax_scale, void* stream) {
+  if (M < 0 || K < 0 || K % 8 != 0 || ldx < K || ldq < K) return FP8Q_ERR_INVALID_ARG;
+  if (amax_scale == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (M > 0 && K > 0 && (x == nullptr || q == nullptr)) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(amax_scale, 4) || (M > 0 && K > 0 && (!aligned(x, 16) || !aligned(q, 8) || ldx % 8 != 0 ||
+                                                      ldq % 8 != 0)))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // amax starts at zero (an empty tensor keeps it, and s = 1e-12)
+  if (cudaMemsetAsync(amax_scale, 0, sizeof(float), s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  const int64_t words = M * (K / 8);
+  if (words > 0) {
+    const int per_sm = blocks_per_sm(&dev->pt_amax_per_sm, fp8q::quant_pertensor_amax_kernel, fp8q::kPtQThreads, 0);
+    const int64_t grid = grid_for((words + fp8q::kPtQThreads - 1) / fp8q::kPtQThreads, dev->sm_count, per_sm);
+    fp8q::quant_pertensor_amax_kernel<<<static_cast<unsigned>(grid), fp8q::kPtQThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), M, K, ldx, reinterpret_cast<unsigned int*>(amax_scale));
+    if ((st = launch_status()) != FP8Q_OK) return st;
+  }
+  const int per_sm = blocks_per_sm(&dev->pt_cast_per_sm, fp8q::quant_pertensor_cast_kernel, fp8q::kPtQThreads, 0);
+  const int64_t grid = grid_for((words + fp8q::kPtQThreads - 1) / fp8q::kPtQThreads, dev->sm_count, per_sm);
+  fp8q::quant_pertensor_cast_kernel<<<static_cast<unsigned>(grid), fp8q::kPtQThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), M, K, ldx, static_cast<uint8_t*>(q), ldq, amax_scale, amax_scale + 1);
+  return launch_status();
+}
+
+fp8q_status fp8q_gemm_pertensor(const void* a, int64_t lda, const float* scale_a, const void* b, int64_t ldb,
+                                const float* scale_b, void* d, int64_t ldd, int d_dtype, int64_t M, int64_t N,
+                                int64_t K, void* stream) {
+  const int64_t kIntMax = 0x7FFFFFFF;
+  if (M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M > kIntMax || N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  if (lda < K || ldb < K || ldd < N) return FP8Q_ERR_INVALID_ARG;
+  if (d_dtype != FP8Q_OUT_BF16 && d_dtype != FP8Q_OUT_F32) return FP8Q_ERR_INVALID_ARG;
+  if (a == nullptr || b == nullptr || scale_a == nullptr || scale_b == nullptr || d == nullptr)
+    return FP8Q_ERR_INVALID_ARG;
+  const int64_t esz = d_dtype == FP8Q_OUT_F32 ? 4 : 2;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(scale_a, 4) || !aligned(scale_b, 4) ||
+      lda % 16 != 0 || ldb % 16 != 0 || (ldd * esz) % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, b, K, N, ldb, fp8q::BN / 2)) != FP8Q_OK) return st;
+  fp8q::GemmArgs args{};
+  args.d = d;
+  args.ldd = ldd;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_n_tiles = static_cast<int>((N + fp8q::BN - 1) / fp8q::BN);
+  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
+  args.num_m_tiles = static_cast<int>((M + fp8q::BM - 1) / fp8q::BM);
+  args.G = 1;
+  const int64_t m_pairs = (M + 2 * fp8q::BM - 1) / (2 * fp8q::BM);
+  const int64_t pair_tiles = m_pairs * args.num_n_tiles;
+  if (pair_tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d_dtype == FP8Q_OUT_F32
+             ? launch_gemm_pertensor<fp8q::kOutF32>(dev, ta, tb, args, scale_a, scale_b, pair_tiles, s)
+             : launch_gemm_pertensor<fp8q::kOutBf16>(dev, ta, tb, args, scale_a, scale_b, pair_tiles, s);
 }
 
 fp8q_status fp8q_scale_history_update(int policy, float alpha, const float* amax, float* hist, float* sf, int64_t n,

@@ -307,6 +307,35 @@ fp8q_status fp8q_grouped_gemm_blockscaled_q1x128(const void* a, int64_t lda, con
                                                  void* dq, int64_t lddq, float* sfd, int64_t ld_sfd,
                                                  int64_t N, int64_t K, void* stream);
 
+/*
+ * Per-tensor FP8 baseline ("FP8 Mixed Precision: DeepSeek-V3 Training
+ * Architecture", section 1: the per-tensor scaling that fine-grained tiles
+ * improve on; "Introduction to LLM Quantization", "Fine-grained
+ * Quantization").  Not part of the fine-grained path: it exists to measure
+ * what the fine-grained scales cost in error and in GEMM throughput.
+ *
+ * fp8q_quant_pertensor: one scale for all of x [M][ldx] (K columns):
+ *   amax = max |x|, s = max(fl32(amax / 448), fl32(1e-12)), q = e4m3(fl32(x / s)).
+ *   amax_scale : device FP32 [2], written {amax, s} (4-byte aligned).
+ *   q          : E4M3 [M][ldq].
+ * Requirements: K % 8 == 0, ldx >= K, ldq >= K; x 16-byte aligned, ldx % 8 == 0;
+ * q 8-byte aligned, ldq % 8 == 0.  Runs a memset and two kernels on `stream`.
+ */
+fp8q_status fp8q_quant_pertensor(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
+                                 float* amax_scale, void* stream);
+
+/*
+ * fp8q_gemm_pertensor: D[m,n] = (s_a * s_b) * sum_k A[m,k] * B[n,k], the whole
+ * K reduction accumulated in the tensor cores' FP32 accumulator (no per-chunk
+ * promotion: there is one scale per operand).
+ *   scale_a, scale_b : device FP32 scalars (e.g. amax_scale + 1 of the call above).
+ * Other arguments and requirements as fp8q_gemm_blockscaled (d_dtype
+ * FP8Q_OUT_BF16 or FP8Q_OUT_F32).
+ */
+fp8q_status fp8q_gemm_pertensor(const void* a, int64_t lda, const float* scale_a, const void* b, int64_t ldb,
+                                const float* scale_b, void* d, int64_t ldd, int d_dtype,
+                                int64_t M, int64_t N, int64_t K, void* stream);
+
 /* ---- diagnostics (used by the test suite; not on the hot path) ---------- */
 
 /*

@@ -71,6 +71,7 @@ def _load():
     lib.orc_grouped_gemm_sampled.argtypes = [P, I64, P, P, P, P, I64, I64, I64,
                                              P, I64, P, I64, P]
     lib.orc_quant_pertensor_e4m3.argtypes = [P, I64, P, P]
+    lib.orc_quant_pertensor.argtypes = [P, I64, I64, I64, P, I64, P, P]
     for name in ("orc_quant_act_1x128", "orc_quant_act_128x1", "orc_quant_w_128x128",
                  "orc_gemm_sampled", "orc_grouped_gemm_sampled"):
         getattr(lib, name).restype = ctypes.c_int
@@ -206,6 +207,29 @@ def quant_pertensor_e4m3(x_bf16: np.ndarray):
     s = ctypes.c_float()
     _load().orc_quant_pertensor_e4m3(_p(x), x.size, _p(deq), ctypes.cast(ctypes.pointer(s), ctypes.c_void_p))
     return deq, s.value
+
+
+def quant_pertensor(x_bf16: np.ndarray):
+    """Per-tensor E4M3 codes of a BF16 matrix: (q uint8 [M][K], amax, s)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    a = ctypes.c_float()
+    s = ctypes.c_float()
+    _check(_load().orc_quant_pertensor(_p(x), M, K, K, _p(q), K, ctypes.cast(ctypes.pointer(a), ctypes.c_void_p),
+                                       ctypes.cast(ctypes.pointer(s), ctypes.c_void_p)), "quant_pertensor")
+    return q, a.value, s.value
+
+
+def gemm_pertensor_sampled(a, sa: float, b, sb: float, rows=None, cols=None) -> np.ndarray:
+    """D = (sa * sb) * sum_k decode(a[m,k]) decode(b[n,k]) at the sampled
+    entries, FP64.  This is the block-scaled GEMM with every block scale equal:
+    it calls gemm_sampled with constant scale arrays."""
+    M, K = a.shape
+    N = b.shape[0]
+    sfa = np.full((M, K // 128), sa, np.float32)
+    sfb = np.full((N // 128, K // 128), sb, np.float32)
+    return gemm_sampled(a, sfa, b, sfb, SFB_BLOCK128, rows, cols)
 
 
 # ---------------------------------------------------------------- scale policies

@@ -489,6 +489,23 @@ void orc_quant_pertensor_e4m3(const uint16_t* x, int64_t n, double* deq, float* 
   for (int64_t i = 0; i < n; ++i) deq[i] = e4m3_decode(e4m3_encode(bf16_to_float(x[i]) / s)) * s;
 }
 
+// The same per-tensor rule on a BF16 matrix x [M][ldx], returning the codes:
+// amax over all M x K values, s = max(fl32(amax / 448), fl32(1e-12)),
+// q = e4m3(fl32(x / s)).  *amax_out and *scale_out receive amax and s.
+int orc_quant_pertensor(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                        float* amax_out, float* scale_out) {
+  if (K % 8 != 0 || ldx < K || ldq < K || M < 0) return 1;
+  float amax = 0.0f;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) amax = std::max(amax, std::fabs(bf16_to_float(x[m * ldx + k])));
+  const float s = orc_tile_scale(amax);
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) q[m * ldq + k] = e4m3_encode(bf16_to_float(x[m * ldx + k]) / s);
+  *amax_out = amax;
+  *scale_out = s;
+  return 0;
+}
+
 // ---- scale policies: quantizing with given scales, and history updates -------
 // [P1] "4. Max scaling is robust but noisy": percentile clipping, delayed
 // scaling or amax histories trade clipping against stability, and any smoother

@@ -98,6 +98,19 @@ def test_scale_policy_validation(fp8q):
     assert qp(K=200) == INV and qp(ld_sf=4) == INV and qp(ldq=128) == INV and qp(sf=None) == INV
     assert qp(ldq=264) == ALN and qp(clipped=FAKE + 4) == ALN and qp(sf=FAKE + 2) == ALN
     assert qp(M=0, q=None, sf=None, ld_sf=0) == 0
+    P = L.fp8q_quant_pertensor
+    assert P(FAKE, 4, 100, 128, FAKE, 128, FAKE, None) == INV                       # K % 8
+    assert P(FAKE, 4, 128, 120, FAKE, 128, FAKE, None) == INV                       # ldx < K
+    assert P(FAKE, 4, 128, 128, FAKE, 128, None, None) == INV                       # no scale output
+    assert P(FAKE, 4, 128, 128, FAKE + 4, 128, FAKE, None) == ALN
+    assert P(FAKE, 4, 128, 128, FAKE, 128, FAKE + 2, None) == ALN
+    G = L.fp8q_gemm_pertensor
+    assert G(FAKE, 256, FAKE, FAKE, 256, FAKE, FAKE, 256, 0, 0, 256, 256, None) == INV        # M = 0
+    assert G(FAKE, 256, FAKE, FAKE, 256, FAKE, FAKE, 256, 0, 8, 200, 256, None) == INV        # N % 128
+    assert G(FAKE, 256, FAKE, FAKE, 256, FAKE, FAKE, 256, 2, 8, 256, 256, None) == INV        # dtype
+    assert G(FAKE, 256, None, FAKE, 256, FAKE, FAKE, 256, 0, 8, 256, 256, None) == INV        # no scale
+    assert G(FAKE, 264, FAKE, FAKE, 256, FAKE, FAKE, 256, 0, 8, 256, 256, None) == ALN        # lda % 16
+    assert G(FAKE, 256, FAKE + 2, FAKE, 256, FAKE, FAKE, 256, 0, 8, 256, 256, None) == ALN
     U = L.fp8q_scale_history_update
     assert U(3, 0.5, FAKE, FAKE, FAKE, 16, None) == INV and U(-1, 0.5, FAKE, FAKE, FAKE, 16, None) == INV
     assert U(1, 1.5, FAKE, FAKE, FAKE, 16, None) == INV and U(1, -0.1, FAKE, FAKE, FAKE, 16, None) == INV
