@@ -72,6 +72,12 @@ def _load():
                                              P, I64, P, I64, P]
     lib.orc_quant_pertensor_e4m3.argtypes = [P, I64, P, P]
     lib.orc_quant_pertensor.argtypes = [P, I64, I64, I64, P, I64, P, P]
+    lib.orc_quant_act_1x128_e5m2.argtypes = [P, I64, I64, I64, P, I64, P]
+    lib.orc_quant_act_128x1_e5m2.argtypes = [P, I64, I64, I64, P, I64, P]
+    lib.orc_tile_scale_e5m2.argtypes = [ctypes.c_float]
+    lib.orc_tile_scale_e5m2.restype = ctypes.c_float
+    lib.orc_gemm_sampled_fmt.argtypes = [P, I64, P, P, I64, P, ctypes.c_int, I64, I64, I64,
+                                         P, I64, P, I64, ctypes.c_int, ctypes.c_int, P]
     for name in ("orc_quant_act_1x128", "orc_quant_act_128x1", "orc_quant_w_128x128",
                  "orc_gemm_sampled", "orc_grouped_gemm_sampled"):
         getattr(lib, name).restype = ctypes.c_int
@@ -171,6 +177,53 @@ def quant_act_128x1(x_bf16: np.ndarray):
     qt = np.empty((C, T), np.uint8)
     sf = np.empty((T // 128, C), np.float32)
     _check(_load().orc_quant_act_128x1(_p(x), T, C, C, _p(qt), T, _p(sf)), "quant_act_128x1")
+    return qt, sf
+
+
+def requant_1x128_to_128x1(q: np.ndarray, sf: np.ndarray):
+    """FP8 activation caching ([P3] section 4: activations cached in FP8 for
+    the backward pass).  From a 1x128 quantization (q uint8 [T][C], sf float32
+    [T][C/128]) rebuild Wgrad's operand: the BF16 dequantization xh =
+    RN_bf16(decode(q) * s) -- the product of a 4-bit and a 24-bit significand
+    is exact in FP64, so one rounding -- then the 128x1 quantizer on xh.
+    Returns (qt [C][T], sf_t [T/128][C], xh_bits uint16 [T][C])."""
+    q = np.ascontiguousarray(q, np.uint8)
+    T, C = q.shape
+    sf = np.ascontiguousarray(sf, np.float32)
+    assert sf.shape == (T, C // 128)
+    deq = e4m3_decode(q).reshape(T, C) * np.repeat(sf.astype(np.float64), 128, axis=1)
+    xh = round_bf16(deq)
+    bits = (xh.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)   # exact: xh is a BF16 value
+    qt, sft = quant_act_128x1(bits)
+    return qt, sft, bits
+
+
+FMT_E4M3 = 0
+FMT_E5M2 = 1
+
+
+def tile_scale_e5m2(amax: float) -> float:
+    """E5M2 gradient variant: s = max(fl32(amax / 57344), fl32(1e-12))."""
+    return float(_load().orc_tile_scale_e5m2(float(amax)))
+
+
+def quant_act_1x128_e5m2(x_bf16: np.ndarray):
+    """E5M2 gradient variant of quant_act_1x128: (q [M][K], sf [M][K/128])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    sf = np.empty((M, K // 128), np.float32)
+    _check(_load().orc_quant_act_1x128_e5m2(_p(x), M, K, K, _p(q), K, _p(sf)), "quant_act_1x128_e5m2")
+    return q, sf
+
+
+def quant_act_128x1_e5m2(x_bf16: np.ndarray):
+    """E5M2 gradient variant of quant_act_128x1: (qt [C][T], sf [T/128][C])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    T, C = x.shape
+    qt = np.empty((C, T), np.uint8)
+    sf = np.empty((T // 128, C), np.float32)
+    _check(_load().orc_quant_act_128x1_e5m2(_p(x), T, C, C, _p(qt), T, _p(sf)), "quant_act_128x1_e5m2")
     return qt, sf
 
 
@@ -348,11 +401,12 @@ SFB_BLOCK128 = 0
 SFB_ROW = 1
 
 
-def gemm_sampled(a, sfa, b, sfb, sfb_mode, rows=None, cols=None) -> np.ndarray:
+def gemm_sampled(a, sfa, b, sfb, sfb_mode, rows=None, cols=None, a_fmt=0, b_fmt=0) -> np.ndarray:
     """FP64 block-scaled GEMM D = A . B^T on the requested rows x cols.
 
     a: uint8 [M][K]; sfa: float32 [M][K/128]; b: uint8 [N][K];
     sfb: [N/128][K/128] (SFB_BLOCK128) or [N][K/128] (SFB_ROW).
+    a_fmt, b_fmt: operand formats, FMT_E4M3 (the method's) or FMT_E5M2.
     """
     a = np.ascontiguousarray(a, np.uint8)
     b = np.ascontiguousarray(b, np.uint8)
@@ -363,8 +417,9 @@ def gemm_sampled(a, sfa, b, sfb, sfb_mode, rows=None, cols=None) -> np.ndarray:
     rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, np.int64)
     cols = np.arange(N, dtype=np.int64) if cols is None else np.ascontiguousarray(cols, np.int64)
     out = np.empty((rows.size, cols.size), np.float64)
-    rc = _load().orc_gemm_sampled(_p(a), K, _p(sfa), _p(b), K, _p(sfb), int(sfb_mode),
-                                  M, N, K, _p(rows), rows.size, _p(cols), cols.size, _p(out))
+    rc = _load().orc_gemm_sampled_fmt(_p(a), K, _p(sfa), _p(b), K, _p(sfb), int(sfb_mode),
+                                      M, N, K, _p(rows), rows.size, _p(cols), cols.size, int(a_fmt), int(b_fmt),
+                                      _p(out))
     _check(rc, "gemm_sampled")
     return out
 

@@ -405,29 +405,34 @@ void orc_int8_absmax(const double* x, int64_t n, int8_t* q, double* scale_out) {
 // sfb_mode 0: sfb [N/128][K/128] row-major (128x128 weight blocks).
 // sfb_mode 1: sfb [N][K/128] row-major (per-row 1x128 / 128x1 tiles).
 // rows[nr], cols[nc]: the outputs wanted; out: [nr][nc] FP64.
-int orc_gemm_sampled(const uint8_t* a, int64_t lda, const float* sfa,
-                     const uint8_t* b, int64_t ldb, const float* sfb, int sfb_mode,
-                     int64_t M, int64_t N, int64_t K,
-                     const int64_t* rows, int64_t nr, const int64_t* cols, int64_t nc,
-                     double* out) {
+int orc_gemm_sampled_fmt(const uint8_t* a, int64_t lda, const float* sfa,
+                         const uint8_t* b, int64_t ldb, const float* sfb, int sfb_mode,
+                         int64_t M, int64_t N, int64_t K,
+                         const int64_t* rows, int64_t nr, const int64_t* cols, int64_t nc,
+                         int a_fmt, int b_fmt, double* out) {
   if (K % 128 != 0 || (sfb_mode == 0 && N % 128 != 0)) return 1;
   if (sfb_mode != 0 && sfb_mode != 1) return 1;
+  if (a_fmt < 0 || a_fmt > 1 || b_fmt < 0 || b_fmt > 1) return 1;
   const int64_t KB = K / 128;
-  double lut[256];
-  for (int c = 0; c < 256; ++c) lut[c] = e4m3_decode(static_cast<uint8_t>(c));
+  // operand codes -> values: format 0 E4M3, format 1 E5M2
+  double lut_a[256], lut_b[256];
+  for (int c = 0; c < 256; ++c) {
+    lut_a[c] = a_fmt == 0 ? e4m3_decode(static_cast<uint8_t>(c)) : e5m2_decode(static_cast<uint8_t>(c));
+    lut_b[c] = b_fmt == 0 ? e4m3_decode(static_cast<uint8_t>(c)) : e5m2_decode(static_cast<uint8_t>(c));
+  }
   for (int64_t i = 0; i < nr; ++i) if (rows[i] < 0 || rows[i] >= M) return 2;
   for (int64_t j = 0; j < nc; ++j) if (cols[j] < 0 || cols[j] >= N) return 2;
   parallel_for(nr, [&](int64_t i) {
     const int64_t m = rows[i];
     std::vector<double> arow(K);
-    for (int64_t k = 0; k < K; ++k) arow[k] = lut[a[m * lda + k]];
+    for (int64_t k = 0; k < K; ++k) arow[k] = lut_a[a[m * lda + k]];
     for (int64_t j = 0; j < nc; ++j) {
       const int64_t n = cols[j];
       const uint8_t* brow = b + n * ldb;
       double acc = 0.0;
       for (int64_t kb = 0; kb < KB; ++kb) {
         double chunk = 0.0;
-        for (int64_t k = kb * 128; k < kb * 128 + 128; ++k) chunk += arow[k] * lut[brow[k]];
+        for (int64_t k = kb * 128; k < kb * 128 + 128; ++k) chunk += arow[k] * lut_b[brow[k]];
         double sa = sfa[m * KB + kb];
         double sb = (sfb_mode == 0) ? sfb[(n / 128) * KB + kb] : sfb[n * KB + kb];
         acc += (sa * sb) * chunk;
@@ -436,6 +441,15 @@ int orc_gemm_sampled(const uint8_t* a, int64_t lda, const float* sfa,
     }
   });
   return 0;
+}
+
+// Both operands E4M3 (the method's format).
+int orc_gemm_sampled(const uint8_t* a, int64_t lda, const float* sfa,
+                     const uint8_t* b, int64_t ldb, const float* sfb, int sfb_mode,
+                     int64_t M, int64_t N, int64_t K,
+                     const int64_t* rows, int64_t nr, const int64_t* cols, int64_t nc,
+                     double* out) {
+  return orc_gemm_sampled_fmt(a, lda, sfa, b, ldb, sfb, sfb_mode, M, N, K, rows, nr, cols, nc, 0, 0, out);
 }
 
 // ---- grouped (MoE) GEMM ---------------------------------------------------------
@@ -572,6 +586,56 @@ int orc_scale_history_update(int policy, float alpha, const float* a, float* h, 
     }
     h[i] = nh;
     sf[i] = orc_tile_scale(nh);
+  }
+  return 0;
+}
+
+// ---- E5M2 gradient variant ------------------------------------------------------
+// [P3] "2. Universal E4M3" and [P5] "E4M3 vs E5M2": conventional FP8 recipes
+// store gradients in E5M2 (wider range, 2 mantissa bits), which DeepSeek drops
+// for E4M3 everywhere.  Reading: the same online tile rule with the E5M2
+// maximum in place of 448: s = max(fl32(amax / 57344), fl32(1e-12)),
+// q = e5m2(fl32(x / s)), round-to-nearest-even, saturating at +-57344.
+static float tile_scale_e5m2(float amax) {
+  const float s = amax / 57344.0f;
+  const float floor_s = 1e-12f;
+  return s < floor_s ? floor_s : s;
+}
+
+float orc_tile_scale_e5m2(float amax) { return tile_scale_e5m2(amax); }
+
+// 1x128 tiles (as orc_quant_act_1x128): x [M][ldx] -> q [M][ldq], sf [M][K/128].
+int orc_quant_act_1x128_e5m2(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                             float* sf) {
+  if (K % 128 != 0 || ldx < K || ldq < K || M < 0) return 1;
+  const int64_t KB = K / 128;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t kb = 0; kb < KB; ++kb) {
+      const uint16_t* t = x + m * ldx + kb * 128;
+      float amax = 0.0f;
+      for (int i = 0; i < 128; ++i) amax = std::max(amax, std::fabs(bf16_to_float(t[i])));
+      const float s = tile_scale_e5m2(amax);
+      sf[m * KB + kb] = s;
+      for (int i = 0; i < 128; ++i) q[m * ldq + kb * 128 + i] = e5m2_encode_sat(bf16_to_float(t[i]) / s);
+    }
+  }
+  return 0;
+}
+
+// 128x1 tiles along tokens, transposed (as orc_quant_act_128x1):
+// x [T][ldx] -> qt [C][ldqt], sf [T/128][C].
+int orc_quant_act_128x1_e5m2(const uint16_t* x, int64_t T, int64_t C, int64_t ldx, uint8_t* qt, int64_t ldqt,
+                             float* sf) {
+  if (T % 128 != 0 || ldx < C || ldqt < T || C < 0) return 1;
+  for (int64_t tb = 0; tb < T / 128; ++tb) {
+    for (int64_t c = 0; c < C; ++c) {
+      float amax = 0.0f;
+      for (int i = 0; i < 128; ++i) amax = std::max(amax, std::fabs(bf16_to_float(x[(tb * 128 + i) * ldx + c])));
+      const float s = tile_scale_e5m2(amax);
+      sf[tb * C + c] = s;
+      for (int i = 0; i < 128; ++i)
+        qt[c * ldqt + tb * 128 + i] = e5m2_encode_sat(bf16_to_float(x[(tb * 128 + i) * ldx + c]) / s);
+    }
   }
   return 0;
 }

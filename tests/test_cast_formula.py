@@ -29,6 +29,9 @@ def harness():
     lib.cfc_encode.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
     lib.cfc_check.argtypes = [ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_longlong)]
     lib.cfc_check.restype = ctypes.c_longlong
+    lib.cfc_encode_e5m2.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+    lib.cfc_check_e5m2.argtypes = [ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_longlong)]
+    lib.cfc_check_e5m2.restype = ctypes.c_longlong
     return lib
 
 
@@ -58,4 +61,32 @@ def test_division_free_cast_is_exact_for_every_bf16_pair(harness):
     # sum over amax patterns a = 0..0x7F7F of 2(a+1) signed inputs
     assert pairs.value == 0x7F80 * (0x7F80 + 1)
     assert plain.value > 0          # the uncorrected product differs somewhere: the walk sees it
+    assert bad == 0
+
+
+def test_harness_e5m2_encoder_matches_oracle(harness):
+    """The E5M2 gradient variant: the harness's E5M2 encoder against the
+    oracle's on BF16 values scaled into the cast's range, the E5M2 grid, its
+    midpoints and their neighbours, signed zeros and saturation."""
+    bf = (np.arange(0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    vals = [bf * np.float32(2.0 ** k) for k in (-120, -30, -16, 0, 10)]
+    codes = np.arange(0x7C, dtype=np.uint8)                      # finite magnitudes
+    grid = oracle.e5m2_decode(codes).astype(np.float32)
+    mids = ((grid[:-1].astype(np.float64) + grid[1:]) / 2).astype(np.float32)
+    vals += [grid, mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9)),
+             np.array([0.0, -0.0, 57344.0, 61439.0, 61440.0, 1e30], np.float32)]
+    v = np.concatenate(vals).astype(np.float32)
+    v = np.concatenate([v, -v])
+    v = v[np.isfinite(v)]
+    out = np.empty(v.size, np.uint8)
+    harness.cfc_encode_e5m2(v.ctypes.data, v.size, out.ctypes.data)
+    assert np.array_equal(out, oracle.e5m2_encode(v))
+
+
+def test_division_free_e5m2_cast_is_exact_for_every_bf16_pair(harness):
+    pairs = ctypes.c_longlong(0)
+    plain = ctypes.c_longlong(0)
+    bad = harness.cfc_check_e5m2(ctypes.byref(pairs), ctypes.byref(plain))
+    assert pairs.value == 0x7F80 * (0x7F80 + 1)
+    assert plain.value > 0
     assert bad == 0

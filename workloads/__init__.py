@@ -216,3 +216,35 @@ def drift_tiles(steps: int = 100, seed: int = 0, outlier_sigmas: float = 20.0):
     t_out = int(g.integers(steps // 4, 3 * steps // 4))
     x[t_out, int(g.integers(0, 128))] = np.float32(outlier_sigmas * sig[t_out])
     return f32_to_bf16_bits(x), t_out
+
+
+# E4M3 bytes of a few values with odd significands (3, 5, 7, 3.25, 1.875, 0.4375)
+MIDPOINT_CODES = {0x44: 3.0, 0x4A: 5.0, 0x4E: 7.0, 0x45: 3.25, 0x3F: 1.875, 0x2E: 0.4375}
+
+
+def midpoint_product_pairs(count: int = 64, seed: int = 0):
+    """(code, scale) pairs whose float32 product fl32(c * s) lies exactly on a
+    BF16 rounding midpoint while the exact product does not: the inputs on
+    which rounding c * s to BF16 through float32 (twice) and rounding the exact
+    product once disagree.  Found by walking float32 scales near m / c for
+    midpoints m in [8, 16); returns (codes uint8 [n], scales float32 [n]),
+    both directions of the exact product's offset included."""
+    g = _rng(seed, TID_MISC, 2)
+    codes, scales = [], []
+    for code, c in MIDPOINT_CODES.items():
+        for j in range(128):
+            m = (1.0 + (2 * j + 1) / 256.0) * 8.0
+            s0 = np.float32(m / c)
+            for step in (-2, -1, 1, 2):
+                s = s0
+                for _ in range(abs(step)):
+                    s = np.nextafter(s, np.float32(np.inf) if step > 0 else np.float32(0.0))
+                p = np.float32(np.float32(c) * s)
+                if (int(np.array([p], np.float32).view(np.uint32)[0]) & 0xFFFF) != 0x8000:
+                    continue
+                if np.float64(c) * np.float64(s) == np.float64(p):      # exact products are no trap
+                    continue
+                codes.append(code)
+                scales.append(s)
+    idx = g.permutation(len(codes))[:count]
+    return np.array(codes, np.uint8)[idx], np.array(scales, np.float32)[idx]
