@@ -648,7 +648,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -677,6 +677,28 @@ def run_single(args):
         amax_scale = torch.empty(2, dtype=f32, device=dev)
         fn = lambda: fp8q.fp8q_quant_pertensor(x, q, amax_scale)
         work = ("bytes", T * HID * 3)
+    elif name == "quant_dy_e5m2":
+        # E5M2 gradient variant of the dY quantizer (1x128, s = amax / 57344)
+        dy = randn(T, OUT, sigma=1e-3)
+        q = torch.empty((T, OUT), dtype=u8, device=dev); sf = torch.empty((OUT // 128, ld(T)), dtype=f32, device=dev)
+        fn = lambda: fp8q.fp8q_quant_act_1x128_e5m2(dy, q, sf)
+        work = ("bytes", T * OUT * 3 + T * OUT // 128 * 4)
+    elif name == "dgrad_e5m2":
+        # E5M2 gradient variant of Dgrad: dY (E5M2) x W^T (E4M3)
+        M, N, K = T, HID, OUT
+        qa = torch.empty((M, K), dtype=u8, device=dev); sa = torch.empty((K // 128, ld(M)), dtype=f32, device=dev)
+        fp8q.fp8q_quant_act_1x128_e5m2(randn(M, K, sigma=1e-3), qa, sa)
+        qb, sb = fp8q.quant_w_128x128(randn(N, K, sigma=0.02))
+        d = torch.empty((M, N), dtype=bf, device=dev)
+        fn = lambda: fp8q.fp8q_gemm_blockscaled_fmt(qa, fp8q.FP8Q_FMT_E5M2, sa, qb, fp8q.FP8Q_FMT_E4M3, sb,
+                                                    fp8q.FP8Q_SFB_BLOCK128, d)
+        work = ("flops", 2.0 * M * N * K)
+    elif name == "requant_x_t":
+        # FP8 activation cache -> Wgrad operand: 1x128 codes + scales in, 128x1 transposed codes + scales out
+        q, sf_in = fp8q.quant_act_1x128(randn(T, HID))
+        qt = torch.empty((HID, T), dtype=u8, device=dev); sf = torch.empty((T // 128, ld(HID)), dtype=f32, device=dev)
+        fn = lambda: fp8q.fp8q_requant_1x128_to_128x1(q, sf_in, qt, sf)
+        work = ("bytes", 2 * T * HID + 2 * T * HID // 128 * 4)
     elif name == "pt_fprop":
         # per-tensor baseline GEMM at the Fprop shape: one TMEM accumulation over K, no promotion
         M, N, K = T, OUT, HID

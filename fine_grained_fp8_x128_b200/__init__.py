@@ -38,6 +38,8 @@ FP8Q_POLICY_EMA = 1
 FP8Q_POLICY_DECAYED_MAX = 2
 FP8Q_OUT_BF16 = 0
 FP8Q_OUT_F32 = 1
+FP8Q_FMT_E4M3 = 0
+FP8Q_FMT_E5M2 = 1
 
 EXPORTS = (
     "fp8q_version", "fp8q_status_string", "fp8q_device_status",
@@ -45,7 +47,8 @@ EXPORTS = (
     "fp8q_quant_act_1x128_percentile", "fp8q_scale_history_update", "fp8q_quant_act_128x1", "fp8q_quant_w_128x128",
     "fp8q_gemm_blockscaled", "fp8q_gemm_blockscaled_q1x128",
     "fp8q_grouped_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled_q1x128",
-    "fp8q_quant_pertensor", "fp8q_gemm_pertensor",
+    "fp8q_quant_pertensor", "fp8q_gemm_pertensor", "fp8q_requant_1x128_to_128x1",
+    "fp8q_quant_act_1x128_e5m2", "fp8q_quant_act_128x1_e5m2", "fp8q_gemm_blockscaled_fmt",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
 )
 
@@ -59,6 +62,11 @@ _lib.fp8q_quant_act_1x128.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_gather.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scaled.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]
 _lib.fp8q_quant_act_1x128_percentile.argtypes = [_P, _I, _I, _I, ctypes.c_int, _P, _I, _P, _I, _P, _P]
+_lib.fp8q_requant_1x128_to_128x1.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_1x128_e5m2.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_128x1_e5m2.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_gemm_blockscaled_fmt.argtypes = [_P, ctypes.c_int, _I, _P, _I, _P, ctypes.c_int, _I, _P, _I, ctypes.c_int,
+                                           _P, _I, ctypes.c_int, _I, _I, _I, _P]
 _lib.fp8q_quant_pertensor.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_pertensor.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_int, _I, _I, _I, _P]
 _lib.fp8q_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, _P, _P, _P, _I, _P]
@@ -191,6 +199,39 @@ def fp8q_gemm_blockscaled(a, sfa, b, sfb, sfb_mode, d, stream=None):
     _check(_lib.fp8q_gemm_blockscaled(_ptr(a), _ld(a), _ptr(sfa), _ld(sfa), _ptr(b), _ld(b), _ptr(sfb), _ld(sfb),
                                       int(sfb_mode), _ptr(d), _ld(d), dt, M, N, K, _stream(stream)),
            "fp8q_gemm_blockscaled")
+
+
+def fp8q_requant_1x128_to_128x1(q, sf_in, qt, sf, stream=None):
+    """FP8 activation cache -> Wgrad operand: q uint8 [T][C] with sf_in [C/128][ld >= T]
+    (a 1x128 quantization) -> qt uint8 [C][T], sf [T/128][ld >= C] (128x1 tiles of the
+    BF16 dequantization)."""
+    T, C = q.shape
+    _check(_lib.fp8q_requant_1x128_to_128x1(_ptr(q), T, C, _ld(q), _ptr(sf_in), _ld(sf_in), _ptr(qt), _ld(qt),
+                                            _ptr(sf), _ld(sf), _stream(stream)), "fp8q_requant_1x128_to_128x1")
+
+
+def fp8q_quant_act_1x128_e5m2(x, q, sf, stream=None):
+    """E5M2 gradient variant of fp8q_quant_act_1x128 (s = amax / 57344)."""
+    M, K = x.shape
+    _check(_lib.fp8q_quant_act_1x128_e5m2(_ptr(x), M, K, _ld(x), _ptr(q), _ld(q), _ptr(sf), _ld(sf), _stream(stream)),
+           "fp8q_quant_act_1x128_e5m2")
+
+
+def fp8q_quant_act_128x1_e5m2(x, qt, sf, stream=None):
+    """E5M2 gradient variant of fp8q_quant_act_128x1 (s = amax / 57344)."""
+    T, C = x.shape
+    _check(_lib.fp8q_quant_act_128x1_e5m2(_ptr(x), T, C, _ld(x), _ptr(qt), _ld(qt), _ptr(sf), _ld(sf),
+                                          _stream(stream)), "fp8q_quant_act_128x1_e5m2")
+
+
+def fp8q_gemm_blockscaled_fmt(a, a_fmt, sfa, b, b_fmt, sfb, sfb_mode, d, stream=None):
+    """fp8q_gemm_blockscaled with operand formats FP8Q_FMT_E4M3 / FP8Q_FMT_E5M2."""
+    M, K = a.shape
+    N = b.shape[0]
+    dt = FP8Q_OUT_F32 if d.dtype == torch.float32 else FP8Q_OUT_BF16
+    _check(_lib.fp8q_gemm_blockscaled_fmt(_ptr(a), int(a_fmt), _ld(a), _ptr(sfa), _ld(sfa), _ptr(b), int(b_fmt), _ld(b),
+                                          _ptr(sfb), _ld(sfb), int(sfb_mode), _ptr(d), _ld(d), dt, M, N, K,
+                                          _stream(stream)), "fp8q_gemm_blockscaled_fmt")
 
 
 def fp8q_quant_pertensor(x, q, amax_scale, stream=None):

@@ -191,6 +191,10 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(uint32_t M, uint32_t N) {
   return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
+// Operand-format bits for another FP8 format (E5M2 = 1): A at bits 7-9, B at 10-12.
+__host__ __device__ constexpr uint32_t umma_idesc_formats(uint32_t a_fmt, uint32_t b_fmt) {
+  return (a_fmt << 7) | (b_fmt << 10);
+}
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void umma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -287,6 +291,40 @@ __device__ __forceinline__ uint32_t e4m3x2_neg_quot(float x0, float x1, float nr
 __device__ __forceinline__ float tile_scale(float amax) {
   float s = __fdiv_rn(amax, 448.0f);
   return fmaxf(s, 1e-12f);
+}
+
+// ---------------------------------------------------------------------------
+// The E5M2 gradient variant: FP8 formats as a template parameter (the values
+// are those of the MMA instruction descriptor's operand-format field).
+// ---------------------------------------------------------------------------
+constexpr int kFmtE4M3 = 0;
+constexpr int kFmtE5M2 = 1;
+
+__device__ __forceinline__ uint32_t cvt_e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Tile scale of the format: max(fl32(amax / fmt_max), fl32(1e-12)), fmt_max =
+// 448 (E4M3) or 57344 (E5M2).
+template <int kFmt>
+__device__ __forceinline__ float tile_scale_fmt(float amax) {
+  if (kFmt == kFmtE4M3) return tile_scale(amax);
+  return fmaxf(__fdiv_rn(amax, 57344.0f), 1e-12f);
+}
+
+// e4m3x2_neg_quot for either format.  The E5M2 claim (the code of -t equals
+// the code of fl32(x / s)) was checked by the same exhaustive walk, with
+// s = max(fl32(amax / 57344), fl32(1e-12)): no mismatch.
+template <int kFmt>
+__device__ __forceinline__ uint32_t fp8x2_neg_quot(float x0, float x1, float nr0, float nr1, float s0, float s1) {
+  if (kFmt == kFmtE4M3) return e4m3x2_neg_quot(x0, x1, nr0, nr1, s0, s1);
+  const float2 x = make_float2(x0, x1), nr = make_float2(nr0, nr1);
+  const float2 n = fmul2(x, nr);
+  const float2 e = ffma2(n, make_float2(s0, s1), x);
+  const float2 t = ffma2(e, nr, n);
+  return cvt_e5m2x2(t.x, t.y);
 }
 
 }  // namespace fp8q

@@ -29,6 +29,8 @@ struct DeviceInfo {
   int sm_count = 0;
   bool gemm_attr[2][2][3] = {};   // [grouped][row mode][output mode]
   bool q2_attr = false;
+  bool rq_attr = false;
+  int rq_per_sm = 0;
   bool pair_attr[2][3] = {};       // [row mode][output mode]
   bool pt_attr[2] = {};            // per-tensor GEMM [output mode]
   int pt_clusters[2] = {};
@@ -37,6 +39,9 @@ struct DeviceInfo {
   int q1g_per_sm = 0;
   int q1s_per_sm = 0;
   int q1p_per_sm = 0;
+  int q1e5_per_sm = 0;
+  int q2e5_per_sm = 0;
+  bool q2e5_attr = false;
   int pt_amax_per_sm = 0;
   int pt_cast_per_sm = 0;
   int q2_per_sm = 0;
@@ -277,7 +282,7 @@ fp8q_status dense_launch(DeviceInfo* dev, bool pair, int out, const CUtensorMap&
 // (d = E4M3 codes [M][ldd], sfd[(n/128) * ld_sfd + m] the scales of their 1x128 tiles).
 fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* b, int64_t ldb,
                        const float* sfb, int64_t ld_sfb, int sfb_mode, void* d, int64_t ldd, int out, float* sfd,
-                       int64_t ld_sfd, int64_t M, int64_t N, int64_t K, void* stream) {
+                       int64_t ld_sfd, int64_t M, int64_t N, int64_t K, void* stream, uint32_t idesc_fmt = 0) {
   const int64_t kIntMax = 0x7FFFFFFF;
   if (M < 1 || N < 128 || K < 128 || N % 128 != 0 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
   if (M > kIntMax || N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
@@ -332,6 +337,7 @@ fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_
   args.num_m_tiles = static_cast<int>((M + fp8q::BM - 1) / fp8q::BM);
   args.group_offsets = nullptr;
   args.G = 1;
+  args.idesc_fmt = idesc_fmt;
   const int64_t tiles = static_cast<int64_t>(args.num_m_tiles) * args.num_n_tiles;
   if (tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
@@ -396,6 +402,59 @@ fp8q_status gemm_grouped(const void* a, int64_t lda, const float* sfa, int64_t l
 
 }  // namespace
 
+// Body of the 1x128 quantizer entries, for either FP8 format.
+template <int kFmt>
+fp8q_status quant_1x128_impl(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq, float* sf,
+                             int64_t ld_sf, void* stream) {
+  if (M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  const int per_sm = blocks_per_sm(kFmt == fp8q::kFmtE4M3 ? &dev->q1_per_sm : &dev->q1e5_per_sm, fp8q::quant_act_1x128_kernel<false, kFmt>, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  fp8q::quant_act_1x128_kernel<false, kFmt><<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, nullptr, M);
+  return launch_status();
+}
+
+// Body of the 128x1 quantizer entries, for either FP8 format.
+template <int kFmt>
+fp8q_status quant_128x1_impl(const void* x, int64_t T, int64_t C, int64_t ldx, void* qt, int64_t ldqt, float* sf,
+                             int64_t ld_sf, void* stream) {
+  if (T < 0 || C < 0 || T % 128 != 0 || C % 8 != 0 || ldx < C || ldqt < T || ld_sf < C) return FP8Q_ERR_INVALID_ARG;
+  if (T == 0 || C == 0) return FP8Q_OK;
+  if (x == nullptr || qt == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(qt, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldqt % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    bool& attr = kFmt == fp8q::kFmtE4M3 ? dev->q2_attr : dev->q2e5_attr;
+    if (!attr) {
+      if (cudaFuncSetAttribute(fp8q::quant_act_128x1_kernel<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fp8q::kQTSmem) != cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      attr = true;
+    }
+  }
+  const int64_t items = (T / 128) * ((C + fp8q::kQTCols - 1) / fp8q::kQTCols);
+  const int per_sm = blocks_per_sm(kFmt == fp8q::kFmtE4M3 ? &dev->q2_per_sm : &dev->q2e5_per_sm,
+                                   fp8q::quant_act_128x1_kernel<kFmt>, fp8q::kQTThreads, fp8q::kQTSmem);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  fp8q::quant_act_128x1_kernel<kFmt><<<static_cast<unsigned>(grid), fp8q::kQTThreads, fp8q::kQTSmem,
+                                 static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(x), T, C, ldx,
+                                                                      static_cast<uint8_t*>(qt), ldqt, sf, ld_sf);
+  return launch_status();
+}
+
 extern "C" {
 
 int fp8q_version(void) { return 100; }
@@ -428,21 +487,12 @@ fp8q_status fp8q_device_status(void* stream, int* out_code) {
 
 fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
                                  float* sf, int64_t ld_sf, void* stream) {
-  if (M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M) return FP8Q_ERR_INVALID_ARG;
-  if (M == 0 || K == 0) return FP8Q_OK;
-  if (x == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldq % 16 != 0)
-    return FP8Q_ERR_ALIGNMENT;
-  DeviceInfo* dev = nullptr;
-  fp8q_status st = device_info(&dev);
-  if (st != FP8Q_OK) return st;
-  const int64_t KB = K / 128;
-  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
-  const int per_sm = blocks_per_sm(&dev->q1_per_sm, fp8q::quant_act_1x128_kernel<false>, fp8q::kQ1Threads, 0);
-  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
-  fp8q::quant_act_1x128_kernel<false><<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, nullptr, M);
-  return launch_status();
+  return quant_1x128_impl<fp8q::kFmtE4M3>(x, M, K, ldx, q, ldq, sf, ld_sf, stream);
+}
+
+fp8q_status fp8q_quant_act_1x128_e5m2(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
+                                      float* sf, int64_t ld_sf, void* stream) {
+  return quant_1x128_impl<fp8q::kFmtE5M2>(x, M, K, ldx, q, ldq, sf, ld_sf, stream);
 }
 
 fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K, int64_t ldx, const int32_t* rows,
@@ -596,32 +646,46 @@ fp8q_status fp8q_scale_history_update(int policy, float alpha, const float* amax
   return launch_status();
 }
 
-fp8q_status fp8q_quant_act_128x1(const void* x, int64_t T, int64_t C, int64_t ldx, void* qt, int64_t ldqt,
-                                 float* sf, int64_t ld_sf, void* stream) {
-  if (T < 0 || C < 0 || T % 128 != 0 || C % 8 != 0 || ldx < C || ldqt < T || ld_sf < C) return FP8Q_ERR_INVALID_ARG;
+fp8q_status fp8q_requant_1x128_to_128x1(const void* q, int64_t T, int64_t C, int64_t ldq, const float* sf_in,
+                                        int64_t ld_sf_in, void* qt, int64_t ldqt, float* sf, int64_t ld_sf,
+                                        void* stream) {
+  if (T < 0 || C < 0 || T % 128 != 0 || C % 128 != 0 || ldq < C || ld_sf_in < T || ldqt < T || ld_sf < C)
+    return FP8Q_ERR_INVALID_ARG;
   if (T == 0 || C == 0) return FP8Q_OK;
-  if (x == nullptr || qt == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(qt, 16) || !aligned(sf, 4) || ldx % 8 != 0 || ldqt % 16 != 0)
+  if (q == nullptr || sf_in == nullptr || qt == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(sf_in, 16) || !aligned(qt, 16) || !aligned(sf, 4) || ldq % 16 != 0 ||
+      ld_sf_in % 4 != 0 || ldqt % 16 != 0)
     return FP8Q_ERR_ALIGNMENT;
   DeviceInfo* dev = nullptr;
   fp8q_status st = device_info(&dev);
   if (st != FP8Q_OK) return st;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!dev->q2_attr) {
-      if (cudaFuncSetAttribute(fp8q::quant_act_128x1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fp8q::kQTSmem) != cudaSuccess)
+    if (!dev->rq_attr) {
+      if (cudaFuncSetAttribute(fp8q::requant_1x128_to_128x1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fp8q::kRQSmem) != cudaSuccess)
         return FP8Q_ERR_CUDA;
-      dev->q2_attr = true;
+      dev->rq_attr = true;
     }
   }
-  const int64_t items = (T / 128) * ((C + fp8q::kQTCols - 1) / fp8q::kQTCols);
-  const int per_sm = blocks_per_sm(&dev->q2_per_sm, fp8q::quant_act_128x1_kernel, fp8q::kQTThreads, fp8q::kQTSmem);
+  const int64_t items = (T / 128) * (C / 128);
+  const int per_sm =
+      blocks_per_sm(&dev->rq_per_sm, fp8q::requant_1x128_to_128x1_kernel, fp8q::kQTThreads, fp8q::kRQSmem);
   const int64_t grid = grid_for(items, dev->sm_count, per_sm);
-  fp8q::quant_act_128x1_kernel<<<static_cast<unsigned>(grid), fp8q::kQTThreads, fp8q::kQTSmem,
-                                 static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(x), T, C, ldx,
-                                                                      static_cast<uint8_t*>(qt), ldqt, sf, ld_sf);
+  fp8q::requant_1x128_to_128x1_kernel<<<static_cast<unsigned>(grid), fp8q::kQTThreads, fp8q::kRQSmem,
+                                        static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(q), T, C, ldq, sf_in, ld_sf_in, static_cast<uint8_t*>(qt), ldqt, sf, ld_sf);
   return launch_status();
+}
+
+fp8q_status fp8q_quant_act_128x1(const void* x, int64_t T, int64_t C, int64_t ldx, void* qt, int64_t ldqt,
+                                 float* sf, int64_t ld_sf, void* stream) {
+  return quant_128x1_impl<fp8q::kFmtE4M3>(x, T, C, ldx, qt, ldqt, sf, ld_sf, stream);
+}
+
+fp8q_status fp8q_quant_act_128x1_e5m2(const void* x, int64_t T, int64_t C, int64_t ldx, void* qt, int64_t ldqt,
+                                      float* sf, int64_t ld_sf, void* stream) {
+  return quant_128x1_impl<fp8q::kFmtE5M2>(x, T, C, ldx, qt, ldqt, sf, ld_sf, stream);
 }
 
 fp8q_status fp8q_quant_w_128x128(const void* w, int64_t N, int64_t K, int64_t ldw, void* q, int64_t ldq, float* sf,
@@ -654,6 +718,18 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
   if (d_dtype != FP8Q_OUT_BF16 && d_dtype != FP8Q_OUT_F32) return FP8Q_ERR_INVALID_ARG;
   return gemm_dense(a, lda, sfa, ld_sfa, b, ldb, sfb, ld_sfb, sfb_mode, d, ldd,
                     d_dtype == FP8Q_OUT_F32 ? fp8q::kOutF32 : fp8q::kOutBf16, nullptr, 0, M, N, K, stream);
+}
+
+fp8q_status fp8q_gemm_blockscaled_fmt(const void* a, int a_fmt, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                      const void* b, int b_fmt, int64_t ldb, const float* sfb, int64_t ld_sfb,
+                                      int sfb_mode, void* d, int64_t ldd, int d_dtype, int64_t M, int64_t N, int64_t K,
+                                      void* stream) {
+  if (d_dtype != FP8Q_OUT_BF16 && d_dtype != FP8Q_OUT_F32) return FP8Q_ERR_INVALID_ARG;
+  if ((a_fmt != FP8Q_FMT_E4M3 && a_fmt != FP8Q_FMT_E5M2) || (b_fmt != FP8Q_FMT_E4M3 && b_fmt != FP8Q_FMT_E5M2))
+    return FP8Q_ERR_INVALID_ARG;
+  return gemm_dense(a, lda, sfa, ld_sfa, b, ldb, sfb, ld_sfb, sfb_mode, d, ldd,
+                    d_dtype == FP8Q_OUT_F32 ? fp8q::kOutF32 : fp8q::kOutBf16, nullptr, 0, M, N, K, stream,
+                    fp8q::umma_idesc_formats(static_cast<uint32_t>(a_fmt), static_cast<uint32_t>(b_fmt)));
 }
 
 fp8q_status fp8q_gemm_blockscaled_q1x128(const void* a, int64_t lda, const float* sfa, int64_t ld_sfa, const void* b,

@@ -94,6 +94,7 @@ struct GemmArgs {
   const int32_t* group_offsets;  // grouped only
   int G;
   int group_m;           // pair kernel: 256-row tiles per L2 group (tiles run m-fastest within a group)
+  uint32_t idesc_fmt;    // operand formats OR-ed into the MMA instruction descriptor (0: both E4M3)
 };
 
 // Which output tile a linear tile id denotes.
@@ -460,7 +461,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
     } else if (warp == 9) {
       // ---------------- MMA issuer (one lane) ----------------
       if (lane == 0) {
-        const uint32_t idesc = umma_idesc_e4m3_f32(BM, BN);
+        const uint32_t idesc = umma_idesc_e4m3_f32(BM, BN) | p.idesc_fmt;
         const int total_chunks = ((total_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                                   static_cast<int>(gridDim.x)) * nk;
         bool ok = true;

@@ -197,7 +197,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     } else if (warp == 9 && rank == 0) {
       // ---------------- MMA issuer (leader CTA, one lane) ----------------
       if (lane == 0) {
-        const uint32_t idesc = umma_idesc_e4m3_f32(2 * BM, BN);
+        const uint32_t idesc = umma_idesc_e4m3_f32(2 * BM, BN) | p.idesc_fmt;
         const int total_chunks =
             ((total_tiles - cluster + nclusters - 1) / nclusters) * nk;
         bool ok = true;

@@ -29,9 +29,10 @@ __device__ __forceinline__ float amax2_value(uint32_t m) { return fmaxf(bf16lo(m
 // order: q = e4m3(fl32(x / s)), with nr = -fl32(1/s) (see e4m3x2_neg_quot,
 // which returns the codes with inverted signs; one XOR flips all four back).
 constexpr uint32_t kFlipSigns = 0x80808080u;
+template <int kFmt = kFmtE4M3>
 __device__ __forceinline__ uint32_t quant_words(uint32_t w0, uint32_t w1, float nr, float s) {
-  const uint32_t c0 = e4m3x2_neg_quot(bf16lo(w0), bf16hi(w0), nr, nr, s, s);
-  const uint32_t c1 = e4m3x2_neg_quot(bf16lo(w1), bf16hi(w1), nr, nr, s, s);
+  const uint32_t c0 = fp8x2_neg_quot<kFmt>(bf16lo(w0), bf16hi(w0), nr, nr, s, s);
+  const uint32_t c1 = fp8x2_neg_quot<kFmt>(bf16lo(w1), bf16hi(w1), nr, nr, s, s);
   return (c0 | (c1 << 16)) ^ kFlipSigns;
 }
 
@@ -86,7 +87,7 @@ __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restr
   }
 }
 
-template <bool kGather>
+template <bool kGather, int kFmt = kFmtE4M3>
 __global__ void __launch_bounds__(kQ1Threads)
 quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
                        uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
@@ -115,15 +116,15 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
     float m = amax2_value(m2);
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    const float s = tile_scale(m);
+    const float s = tile_scale_fmt<kFmt>(m);
     const float nr = -__frcp_rn(s);
     if (row < M) {
       uint8_t* dst = q + row * ldq + kb * 128 + sub * 8;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint2 o;
-        o.x = quant_words(cur.v[i].x, cur.v[i].y, nr, s);
-        o.y = quant_words(cur.v[i].z, cur.v[i].w, nr, s);
+        o.x = quant_words<kFmt>(cur.v[i].x, cur.v[i].y, nr, s);
+        o.y = quant_words<kFmt>(cur.v[i].z, cur.v[i].w, nr, s);
         if (kGather)
           __stcs(reinterpret_cast<uint2*>(dst + 32 * i), o);   // evict-first: leave the L2 to the source rows
         else
@@ -372,15 +373,106 @@ __device__ __forceinline__ void qt_stage(uint32_t* tile, const __nv_bfloat16* __
   cp_async_commit();
 }
 
+// Write the 128x1 codes of a 128-token x ncols tile transposed (qt rows c0 +
+// c, columns tb*128 ..), through 16 KB of shared memory that every thread has
+// finished reading.  Thread (p = tid % 64, r = tid / 64) holds channel 2p's
+// tokens 32r .. +15 and +16 .. +31 in codes[0], codes[1], and channel 2p+1's
+// in codes[2], codes[3].  Channel row c keeps its 16-byte chunk j at slot
+// j ^ ((c / 2) % 8), so the 8 lanes of a wavefront hit 8 different bank
+// groups both when the rows are written and when they are read back; each
+// warp store instruction then writes 4 whole 128-byte rows of qt.
+__device__ __forceinline__ void qt_store_transposed(uint8_t* smem16k, const uint4 (&codes)[4], bool active,
+                                                    int64_t tb, int64_t c0, int64_t ncols,
+                                                    uint8_t* __restrict__ qt, int64_t ldqt, int tid) {
+  const int p = tid & 63;
+  const int r = tid >> 6;
+  __syncthreads();
+  uint4* crows = reinterpret_cast<uint4*>(smem16k);
+  if (active) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 2 * r + h;
+      crows[(2 * p) * 8 + (j ^ (p & 7))] = codes[h];
+      crows[(2 * p + 1) * 8 + (j ^ (p & 7))] = codes[2 + h];
+    }
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int row = 4 * warp + (lane >> 3); row < ncols; row += 4 * (kQTThreads / 32)) {
+    const int j = lane & 7;
+    *reinterpret_cast<uint4*>(qt + (c0 + row) * ldqt + tb * 128 + 16 * j) = crows[row * 8 + (j ^ ((row >> 1) & 7))];
+  }
+}
+
+// Cast one staged BF16 tile -- 128 tokens x ncols (<= 128) channels, row t
+// at tile_bytes + 256 t -- as 128x1 tiles: each channel's maximum over the
+// 128 tokens (the four token quarters combine through qmax), its scale into
+// sf[tb * ld_sf + c0 + c], and its 128 codes transposed into row c0 + c of
+// qt.  The staged tile is overwritten by the transposed codes.  Every thread
+// of the block calls it (it synchronizes the block).
+template <int kFmt = kFmtE4M3>
+__device__ __forceinline__ void qt_cast_staged(uint8_t* tile_bytes, float* qmax, int64_t tb, int64_t c0,
+                                               int64_t ncols, uint8_t* __restrict__ qt, int64_t ldqt,
+                                               float* __restrict__ sf, int64_t ld_sf, int tid) {
+  const int p = tid & 63;          // channel pair
+  const int r = tid >> 6;          // token quarter
+  constexpr int kWords = kQTCols / 2;   // 64 words per staged row
+  const uint32_t* tile = reinterpret_cast<const uint32_t*>(tile_bytes);
+  const bool active = 2 * p < ncols;
+  uint4 codes[4];                  // channel 2p: tokens 32r .. +15, +16 .. +31; then channel 2p+1
+  float ma = 0.0f, mb = 0.0f;
+  if (active) {
+    uint32_t m2 = 0;   // channel 2p in the low half, 2p+1 in the high half
+#pragma unroll 8
+    for (int t = 32 * r; t < 32 * r + 32; ++t) m2 = amax2(m2, tile[t * kWords + p]);
+    ma = bf16lo(m2);
+    mb = bf16hi(m2);
+  }
+  qmax[r * kQTCols + 2 * p] = ma;
+  qmax[r * kQTCols + 2 * p + 1] = mb;
+  __syncthreads();
+  if (active) {
+    ma = fmaxf(fmaxf(qmax[2 * p], qmax[kQTCols + 2 * p]), fmaxf(qmax[2 * kQTCols + 2 * p], qmax[3 * kQTCols + 2 * p]));
+    mb = fmaxf(fmaxf(qmax[2 * p + 1], qmax[kQTCols + 2 * p + 1]),
+               fmaxf(qmax[2 * kQTCols + 2 * p + 1], qmax[3 * kQTCols + 2 * p + 1]));
+    const float sa = tile_scale_fmt<kFmt>(ma), sb = tile_scale_fmt<kFmt>(mb);
+    const float nra = -__frcp_rn(sa), nrb = -__frcp_rn(sb);
+    const int64_t ca = c0 + 2 * p;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t oa[4], ob[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t a4 = 0, b4 = 0;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 32 * r + 16 * h + 4 * j + 2 * e;
+          const uint32_t w0 = tile[t * kWords + p];
+          const uint32_t w1 = tile[(t + 1) * kWords + p];
+          a4 |= fp8x2_neg_quot<kFmt>(bf16lo(w0), bf16lo(w1), nra, nra, sa, sa) << (16 * e);
+          b4 |= fp8x2_neg_quot<kFmt>(bf16hi(w0), bf16hi(w1), nrb, nrb, sb, sb) << (16 * e);
+        }
+        oa[j] = a4 ^ kFlipSigns;
+        ob[j] = b4 ^ kFlipSigns;
+      }
+      codes[h] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+      codes[2 + h] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+    if (r == 0) {
+      sf[tb * ld_sf + ca] = sa;
+      sf[tb * ld_sf + ca + 1] = sb;
+    }
+  }
+  qt_store_transposed(tile_bytes, codes, active, tb, c0, ncols, qt, ldqt, tid);
+}
+
+template <int kFmt = kFmtE4M3>
 __global__ void __launch_bounds__(kQTThreads)
 quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C, int64_t ldx,
                        uint8_t* __restrict__ qt, int64_t ldqt, float* __restrict__ sf, int64_t ld_sf) {
   extern __shared__ __align__(128) uint8_t q2_smem[];
   float* qmax = reinterpret_cast<float*>(q2_smem + 2 * kQTTileBytes);   // [4 quarters][128 channels]
   const int tid = threadIdx.x;
-  const int p = tid & 63;          // channel pair
-  const int r = tid >> 6;          // token quarter
-  constexpr int kWords = kQTCols / 2;   // 64 words per staged row
   const int64_t col_blocks = (C + kQTCols - 1) / kQTCols;
   const int64_t items = (T / 128) * col_blocks;
   int64_t it = blockIdx.x;
@@ -397,77 +489,153 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
       cp_async_wait<0>();
     }
     __syncthreads();
-    const uint32_t* tile = reinterpret_cast<const uint32_t*>(q2_smem + buf * kQTTileBytes);
     const int64_t tb = it / col_blocks;
     const int64_t c0 = (it - tb * col_blocks) * kQTCols;
     const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;
-    const bool active = 2 * p < ncols;
-    uint4 codes[4];                  // channel 2p: tokens 32r .. +15, +16 .. +31; then channel 2p+1
-    float ma = 0.0f, mb = 0.0f;
-    if (active) {
-      uint32_t m2 = 0;   // channel 2p in the low half, 2p+1 in the high half
-#pragma unroll 8
-      for (int t = 32 * r; t < 32 * r + 32; ++t) m2 = amax2(m2, tile[t * kWords + p]);
-      ma = bf16lo(m2);
-      mb = bf16hi(m2);
-    }
-    qmax[r * kQTCols + 2 * p] = ma;
-    qmax[r * kQTCols + 2 * p + 1] = mb;
-    __syncthreads();
-    if (active) {
-      ma = fmaxf(fmaxf(qmax[2 * p], qmax[kQTCols + 2 * p]), fmaxf(qmax[2 * kQTCols + 2 * p], qmax[3 * kQTCols + 2 * p]));
-      mb = fmaxf(fmaxf(qmax[2 * p + 1], qmax[kQTCols + 2 * p + 1]),
-                 fmaxf(qmax[2 * kQTCols + 2 * p + 1], qmax[3 * kQTCols + 2 * p + 1]));
-      const float sa = tile_scale(ma), sb = tile_scale(mb);
-      const float nra = -__frcp_rn(sa), nrb = -__frcp_rn(sb);
-      const int64_t ca = c0 + 2 * p;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t oa[4], ob[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t a4 = 0, b4 = 0;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = 32 * r + 16 * h + 4 * j + 2 * e;
-            const uint32_t w0 = tile[t * kWords + p];
-            const uint32_t w1 = tile[(t + 1) * kWords + p];
-            a4 |= e4m3x2_neg_quot(bf16lo(w0), bf16lo(w1), nra, nra, sa, sa) << (16 * e);
-            b4 |= e4m3x2_neg_quot(bf16hi(w0), bf16hi(w1), nrb, nrb, sb, sb) << (16 * e);
-          }
-          oa[j] = a4 ^ kFlipSigns;
-          ob[j] = b4 ^ kFlipSigns;
-        }
-        codes[h] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        codes[2 + h] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-      }
-      if (r == 0) {
-        sf[tb * ld_sf + ca] = sa;
-        sf[tb * ld_sf + ca + 1] = sb;
-      }
-    }
-    // Transpose the codes through the staged tile (every read of it is done):
-    // channel row c holds its 128 token codes, 16-byte chunk j at slot
-    // j ^ ((c / 2) % 8), so the 8 lanes of a wavefront hit 8 different bank
-    // groups both when the rows are written and when they are read back; each
-    // warp store instruction then writes 4 whole 128-byte rows of qt.
-    __syncthreads();
-    uint4* crows = reinterpret_cast<uint4*>(q2_smem + buf * kQTTileBytes);
-    if (active) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = 2 * r + h;
-        crows[(2 * p) * 8 + (j ^ (p & 7))] = codes[h];
-        crows[(2 * p + 1) * 8 + (j ^ (p & 7))] = codes[2 + h];
-      }
-    }
-    __syncthreads();
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int row = 4 * warp + (lane >> 3); row < ncols; row += 4 * (kQTThreads / 32)) {
-      const int j = lane & 7;
-      *reinterpret_cast<uint4*>(qt + (c0 + row) * ldqt + tb * 128 + 16 * j) = crows[row * 8 + (j ^ ((row >> 1) & 7))];
-    }
+    qt_cast_staged<kFmt>(q2_smem + buf * kQTTileBytes, qmax, tb, c0, ncols, qt, ldqt, sf, ld_sf, tid);
     __syncthreads();   // this buffer is refilled two items later; the maxima are reused next item
+  }
+}
+
+// ---------------------------------------------------------------------------
+// FP8 activation caching ("FP8 Mixed Precision: DeepSeek-V3 Training
+// Architecture", section 4: activations are cached in FP8 for the backward
+// pass, halving their memory).  The forward pass keeps only the 1x128-tile
+// codes and scales it already made for Fprop; Wgrad needs the activation in
+// 128x1 tiles along tokens, transposed.  This kernel rebuilds that operand
+// from the cache: each element is dequantized to BF16, xh = RN_bf16(e4m3(q) *
+// s) (the exact product rounded once), and the BF16 tile is quantized 128x1
+// exactly as quant_act_128x1_kernel quantizes a BF16 activation.
+//
+// A 256-thread block handles 128 tokens x 128 channels (one 1x128 tile column
+// kb, so one scale per token): the codes (16 KB) and the 128 token scales are
+// staged with cp.async, double-buffered.  Thread (p, r) dequantizes channels
+// 2p, 2p+1 of tokens 32r .. +31 into registers as BF16 pairs, the four token
+// quarters combine their channel maxima through shared memory, and the codes
+// leave transposed through the stage's code buffer (qt_store_transposed).
+// ---------------------------------------------------------------------------
+constexpr int kRQCodeBytes = 128 * 128;
+constexpr int kRQStageBytes = kRQCodeBytes + 128 * 4;
+constexpr int kRQSmem = 2 * kRQStageBytes + 4 * kQTCols * 4;
+
+__device__ __forceinline__ void rq_stage(uint8_t* st, const uint8_t* __restrict__ q, int64_t ldq,
+                                         const float* __restrict__ sf, int64_t ld_sf, int64_t col_blocks, int64_t it,
+                                         int tid) {
+  const int64_t tb = it / col_blocks;
+  const int64_t kb = it - tb * col_blocks;
+  for (int i = tid; i < 128 * 8; i += kQTThreads) {
+    const int rr = i >> 3, cc = i & 7;
+    cp_async16(st + rr * 128 + cc * 16, q + (tb * 128 + rr) * ldq + kb * 128 + cc * 16);
+  }
+  if (tid < 32) cp_async16(st + kRQCodeBytes + 16 * tid, sf + kb * ld_sf + tb * 128 + 4 * tid);
+  cp_async_commit();
+}
+
+// The BF16 bits of the exact product c * s, rounded once to nearest-even,
+// from p = fl32(c * s) and its exact error e = c * s - p: p rounds like the
+// exact product unless p is itself a BF16 midpoint and e != 0, in which case
+// the sign of e says on which side of the midpoint the product lies.
+__device__ __forceinline__ uint32_t bf16_at_midpoint(float p, float e, uint32_t rne) {
+  const uint32_t u = __float_as_uint(p);
+  if ((u & 0xFFFFu) != 0x8000u || e == 0.0f) return rne;
+  return (u >> 16) + (((e > 0.0f) == (p > 0.0f)) ? 1u : 0u);
+}
+
+// Two E4M3 codes (low byte first) -> the BF16 pair RN_bf16(code * s), low
+// first.  Decoding: an E4M3 code's 7 magnitude bits shifted left by 20, read
+// as FP32, are exactly 2^-120 times its value -- the 4 exponent bits land in
+// the float's exponent field and the subnormal codes on FP32 subnormals with
+// the same ratio -- so one exact multiply by 2^120 decodes two codes at once.
+// The common case rounds both products with one packed conversion; the rare
+// product that float32 rounding put on a BF16 midpoint is fixed by its error.
+__device__ __forceinline__ uint32_t dequant_bf16x2(uint32_t c2, float s) {
+  const uint32_t b0 = ((c2 & 0x7Fu) << 20) | ((c2 & 0x80u) << 24);
+  const uint32_t b1 = ((c2 & 0x7F00u) << 12) | ((c2 & 0x8000u) << 16);
+  const float2 v = fmul2(f2u(b0, b1), f2(0x1p120f));
+  const float2 sv = f2(s);
+  const float2 p = fmul2(v, sv);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(p.x, p.y);
+  uint32_t r = *reinterpret_cast<const uint32_t*>(&h);
+  const uint32_t u0 = __float_as_uint(p.x), u1 = __float_as_uint(p.y);
+  if (((u0 & 0xFFFFu) == 0x8000u) | ((u1 & 0xFFFFu) == 0x8000u)) {
+    const float2 e = ffma2(v, sv, make_float2(-p.x, -p.y));
+    r = bf16_at_midpoint(p.x, e.x, r & 0xFFFFu) | (bf16_at_midpoint(p.y, e.y, r >> 16) << 16);
+  }
+  return r;
+}
+
+__global__ void __launch_bounds__(kQTThreads)
+requant_1x128_to_128x1_kernel(const uint8_t* __restrict__ q, int64_t T, int64_t C, int64_t ldq,
+                              const float* __restrict__ sf_in, int64_t ld_sf_in, uint8_t* __restrict__ qt,
+                              int64_t ldqt, float* __restrict__ sf, int64_t ld_sf) {
+  extern __shared__ __align__(128) uint8_t rq_smem[];
+  float* qmax = reinterpret_cast<float*>(rq_smem + 2 * kRQStageBytes);   // [4 quarters][128 channels]
+  const int tid = threadIdx.x;
+  const int p = tid & 63;          // channel pair
+  const int r = tid >> 6;          // token quarter
+  const int64_t col_blocks = C / 128;
+  const int64_t items = (T / 128) * col_blocks;
+  int64_t it = blockIdx.x;
+  if (it >= items) return;
+  int buf = 0;
+  rq_stage(rq_smem, q, ldq, sf_in, ld_sf_in, col_blocks, it, tid);
+  for (; it < items; it += gridDim.x, buf ^= 1) {
+    const int64_t next = it + gridDim.x;
+    if (next < items) {
+      rq_stage(rq_smem + (buf ^ 1) * kRQStageBytes, q, ldq, sf_in, ld_sf_in, col_blocks, next, tid);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    uint8_t* st = rq_smem + buf * kRQStageBytes;
+    const float* tok_scale = reinterpret_cast<const float*>(st + kRQCodeBytes);
+    // channels 2p, 2p+1 of tokens 32r .. 32r+31, dequantized to BF16 pairs
+    uint32_t w[32];
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = 32 * r + i;
+      const uint32_t c2 = *reinterpret_cast<const uint16_t*>(st + t * 128 + 2 * p);
+      w[i] = dequant_bf16x2(c2, tok_scale[t]);
+      m2 = amax2(m2, w[i]);
+    }
+    qmax[r * kQTCols + 2 * p] = bf16lo(m2);
+    qmax[r * kQTCols + 2 * p + 1] = bf16hi(m2);
+    __syncthreads();
+    const float ma = fmaxf(fmaxf(qmax[2 * p], qmax[kQTCols + 2 * p]),
+                           fmaxf(qmax[2 * kQTCols + 2 * p], qmax[3 * kQTCols + 2 * p]));
+    const float mb = fmaxf(fmaxf(qmax[2 * p + 1], qmax[kQTCols + 2 * p + 1]),
+                           fmaxf(qmax[2 * kQTCols + 2 * p + 1], qmax[3 * kQTCols + 2 * p + 1]));
+    const float sa = tile_scale(ma), sb = tile_scale(mb);
+    const float nra = -__frcp_rn(sa), nrb = -__frcp_rn(sb);
+    uint4 codes[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t oa[4], ob[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t a4 = 0, b4 = 0;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 16 * h + 4 * j + 2 * e;
+          a4 |= e4m3x2_neg_quot(bf16lo(w[i]), bf16lo(w[i + 1]), nra, nra, sa, sa) << (16 * e);
+          b4 |= e4m3x2_neg_quot(bf16hi(w[i]), bf16hi(w[i + 1]), nrb, nrb, sb, sb) << (16 * e);
+        }
+        oa[j] = a4 ^ kFlipSigns;
+        ob[j] = b4 ^ kFlipSigns;
+      }
+      codes[h] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+      codes[2 + h] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+    const int64_t tb = it / col_blocks;
+    const int64_t c0 = (it - tb * col_blocks) * kQTCols;
+    if (r == 0) {
+      sf[tb * ld_sf + c0 + 2 * p] = sa;
+      sf[tb * ld_sf + c0 + 2 * p + 1] = sb;
+    }
+    qt_store_transposed(st, codes, true, tb, c0, kQTCols, qt, ldqt, tid);
+    __syncthreads();   // this stage buffer is refilled next item; the maxima are reused
   }
 }
 

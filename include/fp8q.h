@@ -66,6 +66,13 @@ enum {
   FP8Q_OUT_F32 = 1   /* FP32 */
 };
 
+/* FP8 operand formats (the method uses E4M3 everywhere; E5M2 is the gradient
+ * variant of conventional FP8 recipes). */
+enum {
+  FP8Q_FMT_E4M3 = 0, /* 1-4-3, max 448 */
+  FP8Q_FMT_E5M2 = 1  /* 1-5-2, max 57344 */
+};
+
 /* Library version (major*10000 + minor*100 + patch). */
 int fp8q_version(void);
 
@@ -200,6 +207,39 @@ fp8q_status fp8q_quant_act_128x1(const void* x, int64_t T, int64_t C, int64_t ld
                                  void* stream);
 
 /*
+ * E5M2 gradient variant of fp8q_quant_act_1x128 and fp8q_quant_act_128x1
+ * ("FP8 Mixed Precision: DeepSeek-V3 Training Architecture", "2. Universal
+ * E4M3": conventional recipes keep gradients in E5M2, which DeepSeek replaces
+ * with E4M3; "Introduction to LLM Quantization", "E4M3 vs E5M2").  The same
+ * tile rule with the E5M2 maximum: s = max(fl32(amax / 57344), fl32(1e-12)),
+ * q = e5m2(fl32(x / s)), round-to-nearest-even, saturating at +-57344.
+ * Arguments, layouts and requirements as the E4M3 calls.
+ */
+fp8q_status fp8q_quant_act_1x128_e5m2(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                      void* q, int64_t ldq, float* sf, int64_t ld_sf, void* stream);
+fp8q_status fp8q_quant_act_128x1_e5m2(const void* x, int64_t T, int64_t C, int64_t ldx,
+                                      void* qt, int64_t ldqt, float* sf, int64_t ld_sf, void* stream);
+
+/*
+ * FP8 activation caching: rebuild Wgrad's 128x1 transposed operand from the
+ * 1x128 FP8 copy the forward pass made ("FP8 Mixed Precision: DeepSeek-V3
+ * Training Architecture", section 4: activations cached in FP8 for the
+ * backward pass), so the BF16 activation need not be kept.
+ *   xh[t][c] = RN_bf16(e4m3(q[t][c]) * s[t][c/128])   (exact product, rounded once)
+ *   then exactly fp8q_quant_act_128x1 of xh.
+ *
+ *   q     : E4M3 [T][ldq], as fp8q_quant_act_1x128 wrote it (no NaN codes).
+ *   sf_in : its scales, sf_in[(c/128) * ld_sf_in + t], ld_sf_in >= T.
+ *   qt, sf: as fp8q_quant_act_128x1 (qt [C][ldqt], sf[(t/128) * ld_sf + c]).
+ * Requirements: T % 128 == 0, C % 128 == 0, ldq >= C, ldqt >= T, ld_sf >= C;
+ * q, qt 16-byte aligned, ldq % 16 == 0, ldqt % 16 == 0; sf_in 16-byte aligned
+ * with ld_sf_in % 4 == 0; sf 4-byte aligned.
+ */
+fp8q_status fp8q_requant_1x128_to_128x1(const void* q, int64_t T, int64_t C, int64_t ldq,
+                                        const float* sf_in, int64_t ld_sf_in,
+                                        void* qt, int64_t ldqt, float* sf, int64_t ld_sf, void* stream);
+
+/*
  * 128x128 weight block quantization ("Fine-Grained FP8 Quantization in
  * DeepSeek", section 3 "Weights use 128x128 blocks"; "FP8 Mixed Precision",
  * eq. s_W = max|W_block| / 448).  Run once per optimizer step; the result is
@@ -244,6 +284,19 @@ fp8q_status fp8q_gemm_blockscaled(const void* a, int64_t lda, const float* sfa, 
                                   const void* b, int64_t ldb, const float* sfb, int64_t ld_sfb,
                                   int sfb_mode, void* d, int64_t ldd, int d_dtype,
                                   int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * fp8q_gemm_blockscaled with the operands' FP8 formats given (FP8Q_FMT_E4M3
+ * or FP8Q_FMT_E5M2 each): the E5M2 gradient variant runs Dgrad as
+ * dY (E5M2) x W^T (E4M3) and Wgrad as dY^T (E5M2) x X^T (E4M3).  The tensor
+ * cores take both formats in one instruction kind; nothing else changes.
+ * Other arguments and requirements as fp8q_gemm_blockscaled; a format outside
+ * the two is FP8Q_ERR_INVALID_ARG.
+ */
+fp8q_status fp8q_gemm_blockscaled_fmt(const void* a, int a_fmt, int64_t lda, const float* sfa, int64_t ld_sfa,
+                                      const void* b, int b_fmt, int64_t ldb, const float* sfb, int64_t ld_sfb,
+                                      int sfb_mode, void* d, int64_t ldd, int d_dtype,
+                                      int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
  * fp8q_gemm_blockscaled (FP8Q_SFB_BLOCK128) whose output is the next layer's

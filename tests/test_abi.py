@@ -98,6 +98,23 @@ def test_scale_policy_validation(fp8q):
     assert qp(K=200) == INV and qp(ld_sf=4) == INV and qp(ldq=128) == INV and qp(sf=None) == INV
     assert qp(ldq=264) == ALN and qp(clipped=FAKE + 4) == ALN and qp(sf=FAKE + 2) == ALN
     assert qp(M=0, q=None, sf=None, ld_sf=0) == 0
+    assert L.fp8q_quant_act_1x128_e5m2(FAKE, 4, 200, 256, FAKE, 256, FAKE, 4, None) == INV     # K % 128
+    assert L.fp8q_quant_act_1x128_e5m2(FAKE, 4, 256, 256, FAKE, 264, FAKE, 4, None) == ALN     # ldq % 16
+    assert L.fp8q_quant_act_128x1_e5m2(FAKE, 100, 8, 8, FAKE, 128, FAKE, 8, None) == INV       # T % 128
+    assert L.fp8q_quant_act_128x1_e5m2(FAKE, 0, 8, 8, None, 128, None, 8, None) == 0
+    F = L.fp8q_gemm_blockscaled_fmt
+    assert F(FAKE, 2, 256, FAKE, 256, FAKE, 0, 256, FAKE, 2, 0, FAKE, 256, 0, 256, 256, 256, None) == INV   # a_fmt
+    assert F(FAKE, 1, 256, FAKE, 256, FAKE, -1, 256, FAKE, 2, 0, FAKE, 256, 0, 256, 256, 256, None) == INV  # b_fmt
+    assert F(FAKE, 1, 256, FAKE, 256, FAKE, 0, 256, FAKE, 2, 0, FAKE, 256, 3, 256, 256, 256, None) == INV   # dtype
+    assert F(FAKE, 1, 256, FAKE, 256, FAKE, 0, 256, FAKE, 2, 0, FAKE, 256, 0, 256, 200, 256, None) == INV   # N % 128
+    R = L.fp8q_requant_1x128_to_128x1
+    assert R(FAKE, 100, 256, 256, FAKE, 128, FAKE, 128, FAKE, 256, None) == INV     # T % 128
+    assert R(FAKE, 128, 200, 256, FAKE, 128, FAKE, 128, FAKE, 256, None) == INV     # C % 128
+    assert R(FAKE, 128, 256, 256, FAKE, 64, FAKE, 128, FAKE, 256, None) == INV      # ld_sf_in < T
+    assert R(FAKE, 128, 256, 256, FAKE + 4, 128, FAKE, 128, FAKE, 256, None) == ALN  # sf_in 16-byte
+    assert R(FAKE, 128, 256, 256, FAKE, 130, FAKE, 128, FAKE, 256, None) == ALN     # ld_sf_in % 4
+    assert R(FAKE, 128, 256, 264, FAKE, 128, FAKE, 128, FAKE, 256, None) == ALN     # ldq % 16
+    assert R(FAKE, 0, 256, 256, None, 0, None, 0, None, 256, None) == 0
     P = L.fp8q_quant_pertensor
     assert P(FAKE, 4, 100, 128, FAKE, 128, FAKE, None) == INV                       # K % 8
     assert P(FAKE, 4, 128, 120, FAKE, 128, FAKE, None) == INV                       # ldx < K
