@@ -648,7 +648,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -677,6 +677,34 @@ def run_single(args):
         amax_scale = torch.empty(2, dtype=f32, device=dev)
         fn = lambda: fp8q.fp8q_quant_pertensor(x, q, amax_scale)
         work = ("bytes", T * HID * 3)
+    elif name in ("moe_dispatch", "moe_dispatch_nccl", "moe_layout"):
+        # FP8 MoE dispatch on one GPU: without a process group (layout + gather-quantize
+        # into the grouped GEMM's input), through a one-rank NCCL group (layout, host sync
+        # for the split sizes, gather-quantize, all_to_all_single, regroup), or the layout alone
+        from fine_grained_fp8_x128_b200.moe_dispatch import dispatch
+        moe_tokens = MOE_TOK if T == TOK else T
+        xm = randn(moe_tokens, HID)
+        ids = torch.from_numpy(W.moe_routing(tokens=moe_tokens, experts=MOE_E, top_k=MOE_K, seed=0).expert_ids
+                               .astype(np.int32)).to(dev)
+        if name == "moe_layout":
+            fn = lambda: fp8q.moe_dispatch_layout(ids, MOE_E)
+            work = ("bytes", moe_tokens * MOE_K * 4 * 4)
+        else:
+            if name == "moe_dispatch_nccl":
+                import socket
+                import torch.distributed as dist
+                sock = socket.socket()
+                sock.bind(("127.0.0.1", 0))
+                os.environ["MASTER_ADDR"] = "127.0.0.1"
+                os.environ["MASTER_PORT"] = str(sock.getsockname()[1])
+                sock.close()
+                dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device(dev))
+            fn = lambda: dispatch(xm, ids, MOE_E)
+            rows_out = moe_tokens * MOE_K
+            # tokens read once (repeats hit the L2), codes and scales written; the exchange path
+            # also reads and writes them again (all_to_all_single) and once more (regroup)
+            passes = 1 if name == "moe_dispatch" else 5
+            work = ("bytes", moe_tokens * HID * 2 + passes * (rows_out * HID + rows_out * (HID // 128) * 4))
     elif name == "quant_dy_e5m2":
         # E5M2 gradient variant of the dY quantizer (1x128, s = amax / 57344)
         dy = randn(T, OUT, sigma=1e-3)
@@ -799,6 +827,9 @@ def run_single(args):
     else:
         out["TFLOPs"] = round(work[1] / t / 1e12, 1)
     print(json.dumps(out), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
     if code != 0:
         raise SystemExit(1)
 

@@ -49,6 +49,8 @@ EXPORTS = (
     "fp8q_grouped_gemm_blockscaled", "fp8q_grouped_gemm_blockscaled_q1x128",
     "fp8q_quant_pertensor", "fp8q_gemm_pertensor", "fp8q_requant_1x128_to_128x1",
     "fp8q_quant_act_1x128_e5m2", "fp8q_quant_act_128x1_e5m2", "fp8q_gemm_blockscaled_fmt",
+    "fp8q_moe_dispatch_layout_workspace", "fp8q_moe_dispatch_layout", "fp8q_quant_act_1x128_gather_rowscales",
+    "fp8q_gather_rows_fp8",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
 )
 
@@ -67,6 +69,11 @@ _lib.fp8q_quant_act_1x128_e5m2.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_128x1_e5m2.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_gemm_blockscaled_fmt.argtypes = [_P, ctypes.c_int, _I, _P, _I, _P, ctypes.c_int, _I, _P, _I, ctypes.c_int,
                                            _P, _I, ctypes.c_int, _I, _I, _I, _P]
+_lib.fp8q_moe_dispatch_layout_workspace.argtypes = [_I, ctypes.c_int]
+_lib.fp8q_moe_dispatch_layout_workspace.restype = ctypes.c_int64
+_lib.fp8q_moe_dispatch_layout.argtypes = [_P, _I, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _I, _P]
+_lib.fp8q_quant_act_1x128_gather_rowscales.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_gather_rows_fp8.argtypes = [_P, _I, _P, _I, _I, _P, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_pertensor.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_pertensor.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_int, _I, _I, _I, _P]
 _lib.fp8q_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, _P, _P, _P, _I, _P]
@@ -232,6 +239,44 @@ def fp8q_gemm_blockscaled_fmt(a, a_fmt, sfa, b, b_fmt, sfb, sfb_mode, d, stream=
     _check(_lib.fp8q_gemm_blockscaled_fmt(_ptr(a), int(a_fmt), _ld(a), _ptr(sfa), _ld(sfa), _ptr(b), int(b_fmt), _ld(b),
                                           _ptr(sfb), _ld(sfb), int(sfb_mode), _ptr(d), _ld(d), dt, M, N, K,
                                           _stream(stream)), "fp8q_gemm_blockscaled_fmt")
+
+
+def fp8q_moe_dispatch_layout(expert_ids, num_experts, rows, pos, offsets, workspace, stream=None):
+    """Stable counting sort of the (token, slot) entries by expert (expert_ids int32 [T][k])."""
+    T, k = expert_ids.shape
+    _check(_lib.fp8q_moe_dispatch_layout(_ptr(expert_ids), T * k, k, int(num_experts), _ptr(rows), _ptr(pos),
+                                         _ptr(offsets), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fp8q_moe_dispatch_layout")
+
+
+def moe_dispatch_layout(expert_ids, num_experts, stream=None):
+    """Returns (rows int32 [T*k], pos int32 [T][k], offsets int32 [E+1]) on expert_ids' device."""
+    T, k = expert_ids.shape
+    dev = expert_ids.device
+    rows = torch.empty(T * k, dtype=torch.int32, device=dev)
+    pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(1, _lib.fp8q_moe_dispatch_layout_workspace(T * k, int(num_experts))), dtype=torch.int32,
+                     device=dev)
+    fp8q_moe_dispatch_layout(expert_ids, num_experts, rows, pos, offsets, ws, stream)
+    return rows, pos, offsets
+
+
+def fp8q_quant_act_1x128_gather_rowscales(x, rows, q, sf, stream=None):
+    """Gather-quantize: q row m = 1x128 FP8 of x row rows[m]; sf row-major [M][ld >= K/128]."""
+    M_src, K = x.shape
+    M = rows.numel()
+    _check(_lib.fp8q_quant_act_1x128_gather_rowscales(_ptr(x), M_src, K, _ld(x), _ptr(rows), M, _ptr(q), _ld(q),
+                                                      _ptr(sf), _ld(sf), _stream(stream)),
+           "fp8q_quant_act_1x128_gather_rowscales")
+
+
+def fp8q_gather_rows_fp8(q_in, sf_in, rows, q_out, sf_out, stream=None):
+    """q_out row m = q_in row rows[m]; scales row-major in, [K/128][ld >= M_out] out."""
+    M_in, K = q_in.shape
+    _check(_lib.fp8q_gather_rows_fp8(_ptr(q_in), _ld(q_in), _ptr(sf_in), _ld(sf_in), M_in, _ptr(rows), rows.numel(), K,
+                                     _ptr(q_out), _ld(q_out), _ptr(sf_out), _ld(sf_out), _stream(stream)),
+           "fp8q_gather_rows_fp8")
 
 
 def fp8q_quant_pertensor(x, q, amax_scale, stream=None):

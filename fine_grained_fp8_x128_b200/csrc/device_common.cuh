@@ -30,6 +30,7 @@ enum : uint32_t {
   WAIT_DEBUG = 6,
   BAD_GROUP_OFFSETS = 7,
   BAD_ROW_INDEX = 8,
+  BAD_EXPERT_ID = 9,
 };
 
 __device__ __forceinline__ void report_status(uint32_t code, uint32_t where) {

@@ -40,6 +40,7 @@ struct DeviceInfo {
   int q1s_per_sm = 0;
   int q1p_per_sm = 0;
   int q1e5_per_sm = 0;
+  int q1gr_per_sm = 0;
   int q2e5_per_sm = 0;
   bool q2e5_attr = false;
   int pt_amax_per_sm = 0;
@@ -230,6 +231,13 @@ fp8q_status launch_gemm_pertensor(DeviceInfo* dev, const CUtensorMap& ta, const 
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args, sa, sb) != cudaSuccess) return FP8Q_ERR_CUDA;
   return launch_status();
+}
+
+// Chunks of the dispatch layout's counting sort: about 256 entries each, at
+// most 512 (a fixed rule, so the workspace size needs no device query).
+int64_t layout_chunks(int64_t n) {
+  int64_t c = (n + 255) / 256;
+  return c < 1 ? 1 : (c > 512 ? 512 : c);
 }
 
 // L2 tile order of the pair kernel: tiles run through groups of group_m
@@ -511,6 +519,92 @@ fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K,
   const int64_t grid = grid_for(items, dev->sm_count, per_sm);
   fp8q::quant_act_1x128_kernel<true><<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, rows, M_src);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_act_1x128_gather_rowscales(const void* x, int64_t M_src, int64_t K, int64_t ldx,
+                                                  const int32_t* rows, int64_t M, void* q, int64_t ldq, float* sf,
+                                                  int64_t ld_sf, void* stream) {
+  if (M_src < 0 || M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < K / 128)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || rows == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || !aligned(rows, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  auto kern = fp8q::quant_act_1x128_kernel<true, fp8q::kFmtE4M3, true>;
+  const int per_sm = blocks_per_sm(&dev->q1gr_per_sm, kern, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  kern<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf, rows, M_src);
+  return launch_status();
+}
+
+int64_t fp8q_moe_dispatch_layout_workspace(int64_t n_entries, int num_experts) {
+  if (n_entries <= 0 || num_experts <= 0) return 0;
+  const int64_t chunks = layout_chunks(n_entries);
+  return 2 * chunks * num_experts;
+}
+
+fp8q_status fp8q_moe_dispatch_layout(const int32_t* expert_ids, int64_t n_entries, int k, int num_experts,
+                                     int32_t* rows, int32_t* pos, int32_t* offsets, int32_t* workspace,
+                                     int64_t workspace_len, void* stream) {
+  if (n_entries < 0 || k < 1 || num_experts < 1 || num_experts > fp8q::kLayoutMaxExperts || n_entries % k != 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (n_entries > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+  if (offsets == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (n_entries > 0 && (expert_ids == nullptr || rows == nullptr || pos == nullptr || workspace == nullptr))
+    return FP8Q_ERR_INVALID_ARG;
+  if (workspace_len < fp8q_moe_dispatch_layout_workspace(n_entries, num_experts)) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(offsets, 4) || (n_entries > 0 && (!aligned(expert_ids, 4) || !aligned(rows, 4) ||
+                                                 !aligned(pos, 4) || !aligned(workspace, 4))))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_entries == 0) {
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (num_experts + 1), s) != cudaSuccess) return FP8Q_ERR_CUDA;
+    return FP8Q_OK;
+  }
+  const int64_t chunks = layout_chunks(n_entries);
+  const int64_t chunk = (n_entries + chunks - 1) / chunks;
+  int32_t* hist = workspace;
+  int32_t* starts = workspace + chunks * num_experts;
+  fp8q::moe_layout_hist_kernel<<<static_cast<unsigned>(chunks), 256, 0, s>>>(expert_ids, n_entries, num_experts, chunk,
+                                                                            hist);
+  if ((st = launch_status()) != FP8Q_OK) return st;
+  fp8q::moe_layout_scan_kernel<<<1, fp8q::kLayoutMaxExperts, 0, s>>>(hist, static_cast<int>(chunks), num_experts,
+                                                                    offsets, starts);
+  if ((st = launch_status()) != FP8Q_OK) return st;
+  fp8q::moe_layout_scatter_kernel<<<static_cast<unsigned>(chunks), 32, 0, s>>>(expert_ids, n_entries, k, num_experts,
+                                                                               chunk, starts, rows, pos);
+  return launch_status();
+}
+
+fp8q_status fp8q_gather_rows_fp8(const void* q_in, int64_t ldq_in, const float* sf_in, int64_t ld_sf_in, int64_t M_in,
+                                 const int32_t* rows, int64_t M_out, int64_t K, void* q_out, int64_t ldq_out,
+                                 float* sf_out, int64_t ld_sf_out, void* stream) {
+  if (M_in < 0 || M_out < 0 || K < 0 || K % 128 != 0 || ldq_in < K || ldq_out < K || ld_sf_in < K / 128 ||
+      ld_sf_out < M_out)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M_out == 0 || K == 0) return FP8Q_OK;
+  if (q_in == nullptr || sf_in == nullptr || rows == nullptr || q_out == nullptr || sf_out == nullptr)
+    return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(q_in, 16) || !aligned(q_out, 16) || ldq_in % 16 != 0 || ldq_out % 16 != 0 || !aligned(sf_in, 4) ||
+      !aligned(sf_out, 4) || !aligned(rows, 4))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t grid = grid_for((M_out + 7) / 8, dev->sm_count, 8);
+  fp8q::gather_rows_fp8_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(q_in), ldq_in, sf_in, ld_sf_in, M_in, rows, M_out, K, static_cast<uint8_t*>(q_out),
+      ldq_out, sf_out, ld_sf_out);
   return launch_status();
 }
 

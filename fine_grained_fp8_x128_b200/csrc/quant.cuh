@@ -47,6 +47,8 @@ __device__ __forceinline__ uint32_t quant_words(uint32_t w0, uint32_t w1, float 
 // With a row map (rows != nullptr) output row m is the quantization of source
 // row rows[m] -- the gather of MoE dispatch fused into the quantizer; an index
 // outside [0, M_src) gives the all-zero tile and records FP8Q_ERR_INVALID_ARG.
+// kRowScales writes the scales row-major, sf[m * ld_sf + kb], the layout in
+// which each row's scales travel with its codes through the dispatch exchange.
 // ---------------------------------------------------------------------------
 constexpr int kQ1Threads = 256;
 constexpr int kQ1Rows = 64;
@@ -87,7 +89,7 @@ __device__ __forceinline__ void q1_load(Q1Slice& d, const __nv_bfloat16* __restr
   }
 }
 
-template <bool kGather, int kFmt = kFmtE4M3>
+template <bool kGather, int kFmt = kFmtE4M3, bool kRowScales = false>
 __global__ void __launch_bounds__(kQ1Threads)
 quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
                        uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sf, int64_t ld_sf,
@@ -130,7 +132,12 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
         else
           *reinterpret_cast<uint2*>(dst + 32 * i) = o;
       }
-      if (sub == 0) sf[kb * ld_sf + row] = s;
+      if (sub == 0) {
+        if (kRowScales)
+          sf[row * ld_sf + kb] = s;      // row-major [M][ld_sf >= K/128]: a row's scales travel with it
+        else
+          sf[kb * ld_sf + row] = s;
+      }
     }
     cur = nxt;
   }
@@ -762,6 +769,126 @@ __global__ void wait_timeout_kernel(long long budget) {
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, WAIT_DEBUG, budget);
   __syncthreads();
+}
+
+}  // namespace fp8q
+
+namespace fp8q {
+
+// ---------------------------------------------------------------------------
+// MoE dispatch ("FP8 Mixed Precision: DeepSeek-V3 Training Architecture",
+// section 4: tokens sent to their experts' GPUs are quantized to FP8 on the
+// fly, halving the all-to-all's bytes).
+//
+// Layout: the (token, slot) entries i = t * k + j with expert ids[i] are put
+// in expert-major order, ties in entry order (a stable counting sort): rows[m]
+// is the token of output row m, pos[i] the output row of entry i, and
+// offsets[e] .. offsets[e+1] the rows of expert e.  Experts are assigned to
+// ranks in contiguous ranges, so the order is also destination-rank-major.
+// Three launches, deterministic: per-chunk expert histograms, one block that
+// scans them, and one warp per chunk that places its entries in order (equal
+// experts within 32 entries are ranked with __match_any_sync).  An id outside
+// [0, E) records FP8Q_ERR_INVALID_ARG and its entry is dropped (pos = -1).
+// ---------------------------------------------------------------------------
+constexpr int kLayoutMaxExperts = 1024;
+
+__global__ void __launch_bounds__(256)
+moe_layout_hist_kernel(const int32_t* __restrict__ ids, int64_t n, int E, int64_t chunk, int32_t* __restrict__ hist) {
+  __shared__ int32_t cnt[kLayoutMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int64_t lo = blockIdx.x * chunk;
+  const int64_t hi = lo + chunk < n ? lo + chunk : n;
+  for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+    const int32_t e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else report_status(FP8Q_ERR_INVALID_ARG, BAD_EXPERT_ID);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[static_cast<int64_t>(blockIdx.x) * E + e] = cnt[e];
+}
+
+// One block of kLayoutMaxExperts threads: offsets[e] = sum of the counts of
+// experts < e; starts[b][e] = offsets[e] + the counts of expert e in chunks < b.
+__global__ void __launch_bounds__(kLayoutMaxExperts)
+moe_layout_scan_kernel(const int32_t* __restrict__ hist, int nchunks, int E, int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ starts) {
+  __shared__ int32_t tot[kLayoutMaxExperts];
+  const int e = threadIdx.x;
+  int32_t t = 0;
+  if (e < E)
+    for (int b = 0; b < nchunks; ++b) t += hist[static_cast<int64_t>(b) * E + e];
+  tot[e] = e < E ? t : 0;
+  __syncthreads();
+  // inclusive scan over the experts (Hillis-Steele in shared memory)
+  for (int d = 1; d < kLayoutMaxExperts; d <<= 1) {
+    const int32_t v = e >= d ? tot[e - d] : 0;
+    __syncthreads();
+    tot[e] += v;
+    __syncthreads();
+  }
+  if (e < E) {
+    int32_t base = tot[e] - t;                // exclusive
+    offsets[e] = base;
+    for (int b = 0; b < nchunks; ++b) {
+      starts[static_cast<int64_t>(b) * E + e] = base;
+      base += hist[static_cast<int64_t>(b) * E + e];
+    }
+    if (e == E - 1) offsets[E] = base;
+  }
+}
+
+__global__ void __launch_bounds__(32)
+moe_layout_scatter_kernel(const int32_t* __restrict__ ids, int64_t n, int k, int E, int64_t chunk,
+                          const int32_t* __restrict__ starts, int32_t* __restrict__ rows, int32_t* __restrict__ pos) {
+  __shared__ int32_t next[kLayoutMaxExperts];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) next[e] = starts[static_cast<int64_t>(blockIdx.x) * E + e];
+  __syncwarp();
+  const int64_t lo = blockIdx.x * chunk;
+  const int64_t hi = lo + chunk < n ? lo + chunk : n;
+  for (int64_t seg = lo; seg < hi; seg += 32) {
+    const int64_t i = seg + lane;
+    int32_t e = i < hi ? ids[i] : -1;
+    if (e >= E) e = -1;
+    const unsigned same = __match_any_sync(0xFFFFFFFFu, e);
+    const int before = __popc(same & ((1u << lane) - 1u));
+    int32_t p = -1;
+    if (e >= 0) p = next[e] + before;
+    __syncwarp();
+    if (e >= 0 && before == 0) next[e] += __popc(same);
+    __syncwarp();
+    if (i < hi) {
+      pos[i] = p;
+      if (p >= 0) rows[p] = static_cast<int32_t>(i / k);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Regroup of received FP8 rows: q_out row m = q_in row rows[m] (K bytes, 16-byte
+// copies), and its K/128 scales from the row-major receive layout into the
+// GEMM's K-chunk-major layout, sf_out[kb * ld_out + m].  One warp per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+gather_rows_fp8_kernel(const uint8_t* __restrict__ q_in, int64_t ldq_in, const float* __restrict__ sf_in,
+                       int64_t ld_sf_in, int64_t M_in, const int32_t* __restrict__ rows, int64_t M_out, int64_t K,
+                       uint8_t* __restrict__ q_out, int64_t ldq_out, float* __restrict__ sf_out, int64_t ld_sf_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t KB = K / 128;
+  for (int64_t m = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); m < M_out; m += warps) {
+    int64_t src = rows[m];
+    if (src < 0 || src >= M_in) {
+      if (lane == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_ROW_INDEX);
+      src = -1;
+    }
+    const uint4* in = reinterpret_cast<const uint4*>(q_in + (src < 0 ? 0 : src) * ldq_in);
+    uint4* out = reinterpret_cast<uint4*>(q_out + m * ldq_out);
+    for (int64_t c = lane; c < K / 16; c += 32) out[c] = src < 0 ? make_uint4(0, 0, 0, 0) : __ldcs(in + c);
+    for (int64_t kb = lane; kb < KB; kb += 32)
+      sf_out[kb * ld_sf_out + m] = src < 0 ? 1e-12f : sf_in[src * ld_sf_in + kb];
+  }
 }
 
 }  // namespace fp8q

@@ -1,0 +1,137 @@
+"""FP8 MoE dispatch across expert-parallel ranks.
+
+"FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 4: tokens
+sent to their experts' GPUs are quantized to FP8 on the fly, which halves the
+all-to-all traffic.  One process per GPU; the experts are split into equal
+contiguous ranges over the ranks of the process group.  One call:
+
+  1. layout (device): a stable counting sort of the (token, slot) entries by
+     expert, giving the send order -- expert-major, hence rank-major;
+  2. the expert offsets come to the host (one synchronisation: the collective
+     needs the split sizes; without a process group nothing is exchanged, the
+     gather quantizer writes the grouped GEMM's input directly and the host
+     never waits);
+  3. gather-quantize (device): each routed token's 1x128 FP8 codes and
+     row-major scales written straight into the send buffer;
+  4. all_to_all_single of the per-(rank, local expert) row counts, then of the
+     codes and of the scales (NCCL over NVLink on GPUs);
+  5. regroup (device): the received rows from (source, expert) order into
+     (expert, source) order, the scales into the grouped GEMM's K-chunk-major
+     layout, so that the grouped GEMM runs on the result directly.
+
+The device steps are this package's kernels (`CudaDispatchOps`).  The
+collectives are torch.distributed's.  The host part -- split sizes and the
+regroup order -- is plain index arithmetic on per-expert counts.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+
+class CudaDispatchOps:
+    """The device steps of a dispatch, on this package's CUDA kernels."""
+
+    def layout(self, expert_ids, num_experts):
+        from . import moe_dispatch_layout
+        return moe_dispatch_layout(expert_ids, num_experts)
+
+    def gather_quant(self, x, rows):
+        import torch
+        from . import fp8q_quant_act_1x128_gather_rowscales
+        M, K = rows.numel(), x.shape[1]
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+        sf = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+        if M > 0:
+            fp8q_quant_act_1x128_gather_rowscales(x, rows, q, sf)
+        return q, sf
+
+    def gather_quant_grouped(self, x, rows):
+        """Without an exchange: the grouped GEMM's input directly (scales K-chunk-major)."""
+        import torch
+        from . import fp8q_quant_act_1x128_gather, sf_ld
+        M, K = rows.numel(), x.shape[1]
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+        sf = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=x.device)
+        if M > 0:
+            fp8q_quant_act_1x128_gather(x, rows, q, sf)
+        return q, sf
+
+    def regroup(self, q, sf, rows):
+        import torch
+        from . import fp8q_gather_rows_fp8, sf_ld
+        M, K = rows.numel(), q.shape[1]
+        q_out = torch.empty((M, K), dtype=torch.uint8, device=q.device)
+        sf_out = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=q.device)
+        if M > 0:
+            fp8q_gather_rows_fp8(q, sf, rows, q_out, sf_out)
+        return q_out, sf_out
+
+
+def regroup_order(recv_counts: np.ndarray):
+    """Received rows arrive source-major, each source's rows expert-major.
+    Returns (rows, expert_offsets): the receive-buffer row of every output row
+    in (local expert, source) order, and the local experts' row ranges."""
+    recv_counts = np.asarray(recv_counts, np.int64)
+    world, el = recv_counts.shape
+    src_base = np.zeros(world + 1, np.int64)
+    src_base[1:] = np.cumsum(recv_counts.sum(axis=1))
+    within = np.zeros((world, el + 1), np.int64)
+    within[:, 1:] = np.cumsum(recv_counts, axis=1)
+    pieces = [src_base[s] + within[s, e] + np.arange(recv_counts[s, e], dtype=np.int64)
+              for e in range(el) for s in range(world)]
+    rows = np.concatenate(pieces).astype(np.int32) if pieces else np.zeros(0, np.int32)
+    offsets = np.zeros(el + 1, np.int32)
+    offsets[1:] = np.cumsum(recv_counts.sum(axis=0))
+    return rows, offsets
+
+
+@dataclass
+class DispatchResult:
+    q: object               # uint8 [M][H]: this rank's expert rows, expert-major then source rank
+    sf: object              # float32 [H/128][ld >= M]: their 1x128 scales (grouped GEMM layout)
+    expert_offsets: object  # int32 [E_local + 1] on the device: the grouped GEMM's group offsets
+    pos: object             # int32 [T][k]: where each local (token, slot) entry went in the send order
+    send_counts: np.ndarray  # int64 [world]: rows sent to each rank (None without a process group)
+    recv_counts: np.ndarray  # int64 [world][E_local]: rows received per source rank and local expert (idem)
+
+
+def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchResult:
+    """x: bf16 [T][H] (H % 128 == 0) on this rank's device; expert_ids: int32
+    [T][k] on the same device.  Collective over `group`: every rank calls it."""
+    import torch
+    import torch.distributed as dist
+    ops = ops or CudaDispatchOps()
+    collective = dist.is_initialized()
+    world = dist.get_world_size(group) if collective else 1
+    if num_experts % world != 0:
+        raise ValueError("num_experts must be a multiple of the group size")
+    el = num_experts // world
+    H = x.shape[1]
+    KB = H // 128
+    rows, pos, offsets = ops.layout(expert_ids, num_experts)
+    if not collective:
+        # one process, all experts local: the layout order is the grouped GEMM's
+        # order, so the gather quantizer writes its input directly, and nothing
+        # waits on the host
+        q, sf = ops.gather_quant_grouped(x, rows)
+        return DispatchResult(q=q, sf=sf, expert_offsets=offsets, pos=pos, send_counts=None, recv_counts=None)
+    off = offsets.cpu().numpy().astype(np.int64)                         # one host sync: the split sizes
+    per_expert = np.diff(off)
+    send_counts = per_expert.reshape(world, el).sum(axis=1)
+    q_send, sf_send = ops.gather_quant(x, rows)
+    counts_send = torch.from_numpy(per_expert.reshape(world, el).astype(np.int64)).to(x.device)
+    counts_recv = torch.empty_like(counts_send)
+    dist.all_to_all_single(counts_recv, counts_send, group=group)
+    recv_counts = counts_recv.cpu().numpy()
+    recv_rows = recv_counts.sum(axis=1)
+    M = int(recv_rows.sum())
+    q_recv = torch.empty((M, H), dtype=torch.uint8, device=x.device)
+    sf_recv = torch.empty((M, KB), dtype=torch.float32, device=x.device)
+    dist.all_to_all_single(q_recv, q_send, recv_rows.tolist(), send_counts.tolist(), group=group)
+    dist.all_to_all_single(sf_recv, sf_send, recv_rows.tolist(), send_counts.tolist(), group=group)
+    order, exp_off = regroup_order(recv_counts)
+    q, sf = ops.regroup(q_recv, sf_recv, torch.from_numpy(order).to(x.device))
+    return DispatchResult(q=q, sf=sf, expert_offsets=torch.from_numpy(exp_off).to(x.device), pos=pos,
+                          send_counts=send_counts, recv_counts=recv_counts)

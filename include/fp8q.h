@@ -130,6 +130,52 @@ fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K,
                                         void* stream);
 
 /*
+ * MoE dispatch in FP8 ("FP8 Mixed Precision: DeepSeek-V3 Training
+ * Architecture", section 4: tokens sent to their experts' GPUs are quantized
+ * to FP8 on the fly, which halves the all-to-all traffic).  The exchange
+ * itself is a collective (torch.distributed all_to_all_single over NCCL);
+ * these calls are its device steps.
+ *
+ * fp8q_moe_dispatch_layout: a stable counting sort of the (token, slot)
+ * entries i = t * k + j by expert id: output row m of the expert-major order
+ * holds token rows[m]; entry i lands on row pos[i]; expert e owns rows
+ * offsets[e] .. offsets[e+1] - 1.  Ties keep entry order.  With experts
+ * assigned to ranks in contiguous ranges the order is also rank-major.
+ *   expert_ids : device int32 [n_entries] (token-major, k per token).
+ *   rows, pos  : device int32 [n_entries]; offsets: device int32 [num_experts + 1].
+ *   workspace  : device int32, at least fp8q_moe_dispatch_layout_workspace(n_entries, num_experts).
+ * Requirements: 1 <= num_experts <= 1024, k >= 1, n_entries % k == 0.  An id
+ * outside [0, num_experts) drops its entry (pos = -1, no row) and records
+ * FP8Q_ERR_INVALID_ARG in the device status word.  Three launches.
+ */
+int64_t fp8q_moe_dispatch_layout_workspace(int64_t n_entries, int num_experts);
+fp8q_status fp8q_moe_dispatch_layout(const int32_t* expert_ids, int64_t n_entries, int k, int num_experts,
+                                     int32_t* rows, int32_t* pos, int32_t* offsets,
+                                     int32_t* workspace, int64_t workspace_len, void* stream);
+
+/*
+ * fp8q_quant_act_1x128_gather with the scales written row-major,
+ * sf[m * ld_sf + kb] (ld_sf >= K/128): the send layout of the dispatch
+ * exchange, in which a row's scales travel with its codes.
+ */
+fp8q_status fp8q_quant_act_1x128_gather_rowscales(const void* x, int64_t M_src, int64_t K, int64_t ldx,
+                                                  const int32_t* rows, int64_t M, void* q, int64_t ldq,
+                                                  float* sf, int64_t ld_sf, void* stream);
+
+/*
+ * Regroup of received FP8 rows into the grouped GEMM's layout: q_out row m =
+ * q_in row rows[m], and its scales from the row-major receive layout
+ * (sf_in[r * ld_sf_in + kb]) into sf_out[kb * ld_sf_out + m].  A row index
+ * outside [0, M_in) writes a zero row with scale 1e-12 and records
+ * FP8Q_ERR_INVALID_ARG.
+ * Requirements: K % 128 == 0, ldq_in >= K, ldq_out >= K (both % 16 == 0,
+ * q_in and q_out 16-byte aligned), ld_sf_in >= K/128, ld_sf_out >= M_out.
+ */
+fp8q_status fp8q_gather_rows_fp8(const void* q_in, int64_t ldq_in, const float* sf_in, int64_t ld_sf_in, int64_t M_in,
+                                 const int32_t* rows, int64_t M_out, int64_t K, void* q_out, int64_t ldq_out,
+                                 float* sf_out, int64_t ld_sf_out, void* stream);
+
+/*
  * 1x128 quantization with GIVEN tile scales -- a scale policy's (fixed
  * calibration, delayed, or a tile-maximum history) instead of the tiles' own
  * maxima.  "Online Quantization During Training", section 4 "Max scaling is

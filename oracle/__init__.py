@@ -396,6 +396,56 @@ def scale_policy_drift(tiles_bf16: np.ndarray, alpha: float = 0.9, percentile: f
     return out
 
 
+# ---------------------------------------------------------------- MoE dispatch
+def moe_layout(expert_ids: np.ndarray, num_experts: int):
+    """[P3] section 4, FP8 MoE dispatch: the (token, slot) entries i = t*k + j
+    in expert-major order, ties in entry order (a stable sort by expert id).
+    Returns (rows [n]: token of output row m, pos [T][k]: output row of each
+    entry, offsets [E+1]: the rows of expert e are offsets[e] .. offsets[e+1]-1)."""
+    ids = np.ascontiguousarray(expert_ids, np.int64)
+    T, k = ids.shape
+    flat = ids.reshape(-1)
+    assert np.all((flat >= 0) & (flat < num_experts))
+    order = np.argsort(flat, kind="stable")
+    rows = (order // k).astype(np.int32)
+    pos = np.empty(flat.size, np.int32)
+    pos[order] = np.arange(flat.size, dtype=np.int32)
+    offsets = np.zeros(num_experts + 1, np.int32)
+    offsets[1:] = np.cumsum(np.bincount(flat, minlength=num_experts))
+    return rows, pos.reshape(T, k), offsets
+
+
+def moe_dispatch_reference(xs, expert_ids_list, num_experts: int):
+    """What each rank holds after an FP8 MoE dispatch over len(xs) ranks with
+    experts split into equal contiguous ranges: for every local expert (in
+    order), the rows from every source rank (in rank order), each source's
+    rows in entry order -- every row the 1x128 FP8 quantization of its token.
+    xs[s]: bf16 bits [T_s][H]; expert_ids_list[s]: int [T_s][k].
+    Returns per rank (q [M][H], sf [M][H/128], expert offsets [E_local+1])."""
+    world = len(xs)
+    assert num_experts % world == 0
+    el = num_experts // world
+    quant = [quant_act_1x128(x) for x in xs]
+    out = []
+    for r in range(world):
+        q_rows, s_rows, counts = [], [], np.zeros(el, np.int64)
+        for e in range(r * el, (r + 1) * el):
+            for s_ in range(world):
+                ids = np.asarray(expert_ids_list[s_])
+                ent = np.nonzero(ids.reshape(-1) == e)[0]
+                toks = ent // ids.shape[1]
+                q_rows.append(quant[s_][0][toks])
+                s_rows.append(quant[s_][1][toks])
+                counts[e - r * el] += toks.size
+        H = xs[0].shape[1]
+        q = np.concatenate(q_rows) if q_rows else np.zeros((0, H), np.uint8)
+        sf = np.concatenate(s_rows) if s_rows else np.zeros((0, H // 128), np.float32)
+        off = np.zeros(el + 1, np.int32)
+        off[1:] = np.cumsum(counts)
+        out.append((q, sf, off))
+    return out
+
+
 # ---------------------------------------------------------------- GEMMs
 SFB_BLOCK128 = 0
 SFB_ROW = 1

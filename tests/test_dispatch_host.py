@@ -1,0 +1,105 @@
+"""Host logic of the FP8 MoE dispatch ("FP8 Mixed Precision: DeepSeek-V3
+Training Architecture", section 4: FP8 all-to-all dispatch), on the CPU: the
+regroup order from per-expert counts, and the whole dispatch over two gloo
+ranks with the device steps done by the oracle, compared with the oracle's
+definition of what each rank must hold afterwards.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from fine_grained_fp8_x128_b200.moe_dispatch import dispatch, regroup_order
+
+
+def test_regroup_order_small():
+    # 2 sources x 3 local experts; receive buffer: source 0 rows (e0: 2, e1: 0, e2: 1), source 1 rows (e0: 1, e1: 2, e2: 0)
+    rows, off = regroup_order(np.array([[2, 0, 1], [1, 2, 0]]))
+    # expected output order: e0 (s0 rows 0,1; s1 row 3), e1 (s1 rows 4,5), e2 (s0 row 2)
+    assert rows.tolist() == [0, 1, 3, 4, 5, 2]
+    assert off.tolist() == [0, 3, 5, 6]
+
+
+def test_regroup_order_is_a_permutation():
+    rng = np.random.default_rng(0)
+    counts = rng.integers(0, 5, (4, 8))
+    counts[1, :] = 0                                  # a source that sends nothing
+    counts[:, 3] = 0                                  # an expert that receives nothing
+    rows, off = regroup_order(counts)
+    assert np.array_equal(np.sort(rows), np.arange(counts.sum()))
+    assert off[-1] == counts.sum() and np.array_equal(np.diff(off), counts.sum(axis=0))
+
+
+class OracleOps:
+    """The dispatch's device steps done by the oracle, on CPU tensors."""
+
+    def layout(self, expert_ids, num_experts):
+        import torch
+        rows, pos, off = oracle.moe_layout(expert_ids.numpy(), num_experts)
+        return torch.from_numpy(rows), torch.from_numpy(pos), torch.from_numpy(off)
+
+    def gather_quant(self, x, rows):
+        import torch
+        q, sf = oracle.quant_act_1x128(x.numpy()[rows.numpy()])
+        return torch.from_numpy(q), torch.from_numpy(sf)
+
+    def regroup(self, q, sf, rows):
+        import torch
+        r = rows.numpy()
+        return torch.from_numpy(q.numpy()[r]), torch.from_numpy(np.ascontiguousarray(sf.numpy()[r].T))
+
+
+def _inputs(rank, T, H, k, E):
+    x = W.activations_with_outliers(T, H, seed=100 + rank, channel_frac=2 / H, elem_frac=1e-3)
+    ids = W.moe_routing(T, E, k, n_forced_empty=1, seed=200 + rank).expert_ids
+    return x, ids
+
+
+def _rank_main(rank, world, port, T_list, H, k, E, result_q):
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x, ids = _inputs(rank, T_list[rank], H, k, E)
+        res = dispatch(torch.from_numpy(x), torch.from_numpy(ids.astype(np.int32)), E, ops=OracleOps())
+        ref = oracle.moe_dispatch_reference([_inputs(r, T_list[r], H, k, E)[0] for r in range(world)],
+                                            [_inputs(r, T_list[r], H, k, E)[1] for r in range(world)], E)[rank]
+        ok = (np.array_equal(res.q.numpy(), ref[0]) and np.array_equal(res.sf.numpy().T, ref[1])
+              and np.array_equal(res.expert_offsets.numpy(), ref[2]))
+        result_q.put((rank, ok, int(res.q.shape[0]), res.send_counts.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+@pytest.mark.parametrize("T_list", [(64, 64), (96, 40)])
+def test_dispatch_two_gloo_ranks(T_list):
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world, H, k, E = 2, 256, 4, 8
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, T_list, H, k, E, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    codes = [p.exitcode for p in procs]
+    results = sorted(q.get(timeout=5) for _ in range(world))
+    assert codes == [0, 0], codes
+    assert all(ok for _, ok, _, _ in results), results
+    # every routed entry was sent and received exactly once
+    total_sent = sum(sum(s) for _, _, _, s in results)
+    assert total_sent == sum(T_list) * k == sum(m for _, _, m, _ in results)

@@ -140,6 +140,7 @@ class Routing:
     token_of_row: np.ndarray  # int64 [T*top_k]
     counts: np.ndarray       # int64 [G]
     empty_experts: np.ndarray
+    expert_ids: np.ndarray = None   # int64 [T][top_k]: each token's experts, in its pick order
 
 
 def moe_routing(tokens: int = 4096, experts: int = 256, top_k: int = 8, zipf_s: float = 1.1,
@@ -164,7 +165,8 @@ def moe_routing(tokens: int = 4096, experts: int = 256, top_k: int = 8, zipf_s: 
     counts = np.bincount(exp, minlength=experts).astype(np.int64)
     offsets = np.zeros(experts + 1, np.int64)
     offsets[1:] = np.cumsum(counts)
-    return Routing(offsets=offsets, token_of_row=tok[order], counts=counts, empty_experts=empty)
+    return Routing(offsets=offsets, token_of_row=tok[order], counts=counts, empty_experts=empty,
+                   expert_ids=choice.astype(np.int64))
 
 
 def expert_weights(G: int, N: int, K: int, seed: int = 0, sigma: float = 0.02,
