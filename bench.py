@@ -35,6 +35,7 @@ import time
 import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+LOG_DIR = os.environ.get("FP8Q_BENCH_LOG_DIR", os.path.join(ROOT, "bench_logs"))   # nvidia-smi clock samples
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
@@ -123,7 +124,7 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank_gpu{gpu_index}.csv")
+        self.path = os.path.join(LOG_DIR, f"clocks_rank_gpu{gpu_index}.csv")
 
     def start(self):
         try:
@@ -515,7 +516,7 @@ def run_fp8q(args):
     # ---- device-resident timed region
     uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     clocks = ClockSampler(uuid)
-    clocks.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+    clocks.path = os.path.join(LOG_DIR, f"clocks_rank{rank}.csv")
     barrier(world, device)
     torch.cuda.synchronize()
     clocks.start()
