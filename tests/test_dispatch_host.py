@@ -84,12 +84,13 @@ def _free_port():
     return port
 
 
-@pytest.mark.parametrize("T_list", [(64, 64), (96, 40)])
-def test_dispatch_two_gloo_ranks(T_list):
+@pytest.mark.parametrize("T_list", [(64, 64), (96, 40), (50, 0, 70, 33)])
+def test_dispatch_gloo_ranks(T_list):
+    """Two and four ranks; one rank of four has no tokens at all."""
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    world, H, k, E = 2, 256, 4, 8
+    world, H, k, E = len(T_list), 256, 4, 8
     port = _free_port()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, T_list, H, k, E, q)) for r in range(world)]
     for p in procs:
@@ -98,7 +99,7 @@ def test_dispatch_two_gloo_ranks(T_list):
         p.join(timeout=120)
     codes = [p.exitcode for p in procs]
     results = sorted(q.get(timeout=5) for _ in range(world))
-    assert codes == [0, 0], codes
+    assert codes == [0] * world, codes
     assert all(ok for _, ok, _, _ in results), results
     # every routed entry was sent and received exactly once
     total_sent = sum(sum(s) for _, _, _, s in results)
