@@ -8,7 +8,7 @@ seeded, outlier-injected input:
     quant_act_1x128(dY) -> Dgrad  dX = dY W           (BF16 out)
     quant_act_128x1(dY), quant_act_128x1(X) -> Wgrad dW = dY^T X   (FP32 out)
   MoE layer, 4096 tokens, top-8 of 256 experts (Zipf 1.1), hidden 7168, expert 2048:
-    quant_act_1x128 over the dispatch gather (tokens -> expert rows)
+    quant_act_1x128 of each token once, scattered to its 8 expert rows (the dispatch)
     grouped up-projection, epilogue emitting H as 1x128 FP8 tiles
     grouped down-projection (BF16 out)
 Expert weights are resident FP8 (quantized once at set-up); the dense weight is
@@ -308,13 +308,13 @@ class DeviceStep:
         self.mt = int(route.offsets[-1])
         xt = W.activations_with_outliers(MOE_TOK, HID, seed=seed, tid=W.TID_MISC)
         self.h_xm = torch.from_numpy(xt.view(np.int16)).view(bf).pin_memory()       # MoE tokens, token order
-        self.h_rows = torch.from_numpy(route.token_of_row.astype(np.int32)).pin_memory()   # expert row -> token
+        self.h_pos = torch.from_numpy(route.entry_row.astype(np.int32)).pin_memory()   # (token, pick) -> expert row
         self.h_off = torch.from_numpy(route.offsets.astype(np.int32)).pin_memory()
         self.w = dev_bf16(W.weights(OUT, HID, seed=seed))                      # model state, resident
         self.x = torch.empty((TOK, HID), dtype=bf, device=device)
         self.dy = torch.empty((TOK, OUT), dtype=bf, device=device)
         self.xm = torch.empty((MOE_TOK, HID), dtype=bf, device=device)
-        self.rows = torch.empty((self.mt,), dtype=torch.int32, device=device)
+        self.pos = torch.empty((MOE_TOK, MOE_K), dtype=torch.int32, device=device)
         self.off = torch.empty((MOE_E + 1,), dtype=torch.int32, device=device)
         self.upload()
         # quantized operands and outputs
@@ -360,7 +360,7 @@ class DeviceStep:
         self.slots.append({k: torch.empty_like(v) for k, v in self.slots[0].items()})
         torch.cuda.synchronize()
 
-    _SLOT = ("x", "dy", "xm", "rows", "off", "y", "dx", "dw", "out")
+    _SLOT = ("x", "dy", "xm", "pos", "off", "y", "dx", "dw", "out")
 
     def _slot_tensors(self):
         return {k: getattr(self, k) for k in self._SLOT}
@@ -370,7 +370,7 @@ class DeviceStep:
             setattr(self, k, v)
 
     def h2d_bytes(self):
-        return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_dy, self.h_xm, self.h_rows, self.h_off))
+        return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_dy, self.h_xm, self.h_pos, self.h_off))
 
     def d2h_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.h_y, self.h_dx, self.h_dw, self.h_out))
@@ -379,7 +379,7 @@ class DeviceStep:
         self.x.copy_(self.h_x, non_blocking=True)
         self.dy.copy_(self.h_dy, non_blocking=True)
         self.xm.copy_(self.h_xm, non_blocking=True)
-        self.rows.copy_(self.h_rows, non_blocking=True)
+        self.pos.copy_(self.h_pos, non_blocking=True)
         self.off.copy_(self.h_off, non_blocking=True)
 
     def download(self):
@@ -403,7 +403,7 @@ class DeviceStep:
             ("quant_x_t", lambda: f.fp8q_quant_act_128x1(self.x, self.xqt, self.sxt)),
             ("wgrad", lambda: f.fp8q_gemm_blockscaled(self.dyqt, self.sdyt, self.xqt, self.sxt, f.FP8Q_SFB_ROW,
                                                       self.dw)),
-            ("quant_moe_x", lambda: f.fp8q_quant_act_1x128_gather(self.xm, self.rows, self.xpq, self.sxp)),
+            ("quant_moe_x", lambda: f.fp8q_quant_act_1x128_scatter(self.xm, self.pos, self.xpq, self.sxp)),
             ("moe_up", lambda: f.fp8q_grouped_gemm_blockscaled_q1x128(self.xpq, self.sxp, self.wup_q, self.wup_s,
                                                                       self.off, self.hq, self.sh)),
             ("moe_down", lambda: f.fp8q_grouped_gemm_blockscaled(self.hq, self.sh, self.wdn_q, self.wdn_s, self.off,
@@ -649,7 +649,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "quant_moe_x_gather", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -780,16 +780,20 @@ def run_single(args):
             mode = fp8q.FP8Q_SFB_BLOCK128
         fn = lambda: fp8q.fp8q_gemm_blockscaled(qa, sa, qb, sb, mode, d)
         work = ("flops", 2.0 * M * N * K)
-    elif name in ("quant_moe_x", "moe_up", "moe_up_q", "moe_down"):
+    elif name in ("quant_moe_x", "quant_moe_x_gather", "moe_up", "moe_up_q", "moe_down"):
         moe_tokens = MOE_TOK if T == TOK else T          # --tokens counts MoE tokens before top-k
         route = W.moe_routing(tokens=moe_tokens, experts=MOE_E, top_k=MOE_K, seed=0)
         mt = int(route.offsets[-1])
-        if name == "quant_moe_x":
+        if name in ("quant_moe_x", "quant_moe_x_gather"):
             xm = randn(moe_tokens, HID)
-            rows = torch.from_numpy(route.token_of_row.astype(np.int32)).to(dev)
             q = torch.empty((mt, HID), dtype=u8, device=dev)
             sf = torch.empty((HID // 128, ld(mt)), dtype=f32, device=dev)
-            fn = lambda: fp8q.fp8q_quant_act_1x128_gather(xm, rows, q, sf)
+            if name == "quant_moe_x":       # each token quantized once, scattered to its expert rows
+                pos = torch.from_numpy(route.entry_row.astype(np.int32)).to(dev)
+                fn = lambda: fp8q.fp8q_quant_act_1x128_scatter(xm, pos, q, sf)
+            else:                           # each expert row gathers and quantizes its token
+                rows = torch.from_numpy(route.token_of_row.astype(np.int32)).to(dev)
+                fn = lambda: fp8q.fp8q_quant_act_1x128_gather(xm, rows, q, sf)
             work = ("bytes", moe_tokens * HID * 2 + mt * HID + mt * HID // 128 * 4)
         else:
             K, N = (MOE_FF, HID) if name == "moe_down" else (HID, MOE_FF)

@@ -50,7 +50,7 @@ EXPORTS = (
     "fp8q_quant_pertensor", "fp8q_gemm_pertensor", "fp8q_requant_1x128_to_128x1",
     "fp8q_quant_act_1x128_e5m2", "fp8q_quant_act_128x1_e5m2", "fp8q_gemm_blockscaled_fmt",
     "fp8q_moe_dispatch_layout_workspace", "fp8q_moe_dispatch_layout", "fp8q_quant_act_1x128_gather_rowscales",
-    "fp8q_gather_rows_fp8",
+    "fp8q_gather_rows_fp8", "fp8q_quant_act_1x128_scatter",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
 )
 
@@ -73,6 +73,7 @@ _lib.fp8q_moe_dispatch_layout_workspace.argtypes = [_I, ctypes.c_int]
 _lib.fp8q_moe_dispatch_layout_workspace.restype = ctypes.c_int64
 _lib.fp8q_moe_dispatch_layout.argtypes = [_P, _I, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_gather_rowscales.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_1x128_scatter.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_gather_rows_fp8.argtypes = [_P, _I, _P, _I, _I, _P, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_pertensor.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_pertensor.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_int, _I, _I, _I, _P]
@@ -269,6 +270,14 @@ def fp8q_quant_act_1x128_gather_rowscales(x, rows, q, sf, stream=None):
     _check(_lib.fp8q_quant_act_1x128_gather_rowscales(_ptr(x), M_src, K, _ld(x), _ptr(rows), M, _ptr(q), _ld(q),
                                                       _ptr(sf), _ld(sf), _stream(stream)),
            "fp8q_quant_act_1x128_gather_rowscales")
+
+
+def fp8q_quant_act_1x128_scatter(x, pos, q, sf, stream=None):
+    """Quantize each row of x once and write it to output rows pos[row][j] (pos int32 [M_src][k])."""
+    M_src, K = x.shape
+    k = pos.shape[1]
+    _check(_lib.fp8q_quant_act_1x128_scatter(_ptr(x), M_src, K, _ld(x), _ptr(pos), k, q.shape[0], _ptr(q), _ld(q),
+                                             _ptr(sf), _ld(sf), _stream(stream)), "fp8q_quant_act_1x128_scatter")
 
 
 def fp8q_gather_rows_fp8(q_in, sf_in, rows, q_out, sf_out, stream=None):

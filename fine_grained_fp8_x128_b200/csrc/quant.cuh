@@ -144,6 +144,70 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
 }
 
 // ---------------------------------------------------------------------------
+// Quantize once, scatter k times: the MoE dispatch from the token side.  Each
+// source row's 1x128 tiles are quantized once (tiling and loads as above) and
+// written to the k output rows pos[row * k + j] it is routed to, so that the
+// same token is not re-read and re-quantized per routed copy.  A negative
+// position (a dropped entry) is skipped; one at or above M_out records
+// FP8Q_ERR_INVALID_ARG and is skipped.  Output rows no entry maps to are not
+// written.
+// ---------------------------------------------------------------------------
+constexpr int kScatterMaxK = 64;
+
+__global__ void __launch_bounds__(kQ1Threads)
+quant_act_1x128_scatter_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
+                               const int32_t* __restrict__ pos, int k, int64_t M_out, uint8_t* __restrict__ q,
+                               int64_t ldq, float* __restrict__ sf, int64_t ld_sf) {
+  const int tid = threadIdx.x;
+  const int sub = tid & 3;
+  const int tile = tid >> 2;
+  const int64_t items = ((M + kQ1Rows - 1) / kQ1Rows) * KB;
+  int64_t it = blockIdx.x;
+  if (it >= items) return;
+  Q1Slice cur, nxt;
+  q1_load<false>(cur, x, M, KB, ldx, nullptr, 0, it, tile, sub);
+  for (; it < items; it += gridDim.x) {
+    const int64_t it_next = it + gridDim.x;
+    if (it_next < items) q1_load<false>(nxt, x, M, KB, ldx, nullptr, 0, it_next, tile, sub);
+    const int64_t rb = it / KB;
+    const int64_t kb = it - rb * KB;
+    const int64_t row = rb * kQ1Rows + tile;
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m2 = amax2(m2, cur.v[i].x); m2 = amax2(m2, cur.v[i].y);
+      m2 = amax2(m2, cur.v[i].z); m2 = amax2(m2, cur.v[i].w);
+    }
+    float m = amax2_value(m2);
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    const float s = tile_scale(m);
+    const float nr = -__frcp_rn(s);
+    if (row < M) {
+      uint2 o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[i].x = quant_words(cur.v[i].x, cur.v[i].y, nr, s);
+        o[i].y = quant_words(cur.v[i].z, cur.v[i].w, nr, s);
+      }
+      for (int j = 0; j < k; ++j) {
+        const int64_t dst = __ldg(pos + row * k + j);
+        if (dst < 0) continue;
+        if (dst >= M_out) {
+          if (sub == 0 && kb == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_ROW_INDEX);
+          continue;
+        }
+        uint8_t* d = q + dst * ldq + kb * 128 + sub * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) __stcs(reinterpret_cast<uint2*>(d + 32 * i), o[i]);
+        if (sub == 0) sf[kb * ld_sf + dst] = s;
+      }
+    }
+    cur = nxt;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Scale policies ("Online Quantization During Training", section 4 and its
 // worked example; "Introduction to LLM Quantization", "5) Online Quantization",
 // delayed quantization): 1x128 tiles cast with GIVEN scales (a policy's, e.g.

@@ -8,9 +8,9 @@ contiguous ranges over the ranks of the process group.  One call:
   1. layout (device): a stable counting sort of the (token, slot) entries by
      expert, giving the send order -- expert-major, hence rank-major;
   2. the expert offsets come to the host (one synchronisation: the collective
-     needs the split sizes; without a process group nothing is exchanged, the
-     gather quantizer writes the grouped GEMM's input directly and the host
-     never waits);
+     needs the split sizes; without a process group nothing is exchanged: each
+     token is quantized once and scattered to its rows of the grouped GEMM's
+     input, and the host never waits);
   3. gather-quantize (device): each routed token's 1x128 FP8 codes and
      row-major scales written straight into the send buffer;
   4. all_to_all_single of the per-(rank, local expert) row counts, then of the
@@ -47,15 +47,16 @@ class CudaDispatchOps:
             fp8q_quant_act_1x128_gather_rowscales(x, rows, q, sf)
         return q, sf
 
-    def gather_quant_grouped(self, x, rows):
-        """Without an exchange: the grouped GEMM's input directly (scales K-chunk-major)."""
+    def quant_grouped(self, x, pos, M):
+        """Without an exchange: the grouped GEMM's input directly (scales K-chunk-major),
+        each token quantized once and written to its M-row layout positions."""
         import torch
-        from . import fp8q_quant_act_1x128_gather, sf_ld
-        M, K = rows.numel(), x.shape[1]
+        from . import fp8q_quant_act_1x128_scatter, sf_ld
+        K = x.shape[1]
         q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
         sf = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=x.device)
-        if M > 0:
-            fp8q_quant_act_1x128_gather(x, rows, q, sf)
+        if M > 0 and x.shape[0] > 0:
+            fp8q_quant_act_1x128_scatter(x, pos, q, sf)
         return q, sf
 
     def regroup(self, q, sf, rows):
@@ -113,9 +114,9 @@ def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchR
     rows, pos, offsets = ops.layout(expert_ids, num_experts)
     if not collective:
         # one process, all experts local: the layout order is the grouped GEMM's
-        # order, so the gather quantizer writes its input directly, and nothing
-        # waits on the host
-        q, sf = ops.gather_quant_grouped(x, rows)
+        # order, so each token is quantized once and written to its rows of the
+        # GEMM input, and nothing waits on the host
+        q, sf = ops.quant_grouped(x, pos, expert_ids.numel())
         return DispatchResult(q=q, sf=sf, expert_offsets=offsets, pos=pos, send_counts=None, recv_counts=None)
     off = offsets.cpu().numpy().astype(np.int64)                         # one host sync: the split sizes
     per_expert = np.diff(off)

@@ -154,6 +154,23 @@ fp8q_status fp8q_moe_dispatch_layout(const int32_t* expert_ids, int64_t n_entrie
                                      int32_t* workspace, int64_t workspace_len, void* stream);
 
 /*
+ * The dispatch quantizer from the token side: each source row of x is
+ * quantized once (1x128 tiles, exactly as fp8q_quant_act_1x128) and its codes
+ * and scales are written to the k output rows pos[row * k + j] (j < k), the
+ * positions fp8q_moe_dispatch_layout returns.  Equal to
+ * fp8q_quant_act_1x128_gather over the inverse map, without quantizing a
+ * token once per routed copy.
+ *   x   : BF16 [M_src][ldx].   pos: device int32 [M_src][k]; a negative entry
+ *         is skipped (a dropped entry), one >= M_out is skipped and records
+ *         FP8Q_ERR_INVALID_ARG.  Output rows that no entry names are left as they are.
+ *   q, sf: as fp8q_quant_act_1x128 with M_out output rows.
+ * Requirements: as fp8q_quant_act_1x128_gather, plus 1 <= k <= 64, pos 4-byte aligned.
+ */
+fp8q_status fp8q_quant_act_1x128_scatter(const void* x, int64_t M_src, int64_t K, int64_t ldx,
+                                         const int32_t* pos, int k, int64_t M_out,
+                                         void* q, int64_t ldq, float* sf, int64_t ld_sf, void* stream);
+
+/*
  * fp8q_quant_act_1x128_gather with the scales written row-major,
  * sf[m * ld_sf + kb] (ld_sf >= K/128): the send layout of the dispatch
  * exchange, in which a row's scales travel with its codes.

@@ -1,9 +1,10 @@
 """GPU parity of the FP8 MoE dispatch's device steps against the oracle
 ("FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 4: FP8
 all-to-all dispatch): the layout kernel (a stable counting sort by expert, bit
-for bit), the gather quantizer with row-major scales, the regroup of received
-FP8 rows, and the whole dispatch on one GPU -- without a process group, and
-through a one-rank NCCL group (the all_to_all_single path).
+for bit), the gather quantizer with row-major scales, the quantize-once scatter
+quantizer, the regroup of received FP8 rows, and the whole dispatch on one GPU
+-- without a process group, and through a one-rank NCCL group (the
+all_to_all_single path).
 """
 import os
 import socket
@@ -131,3 +132,32 @@ def test_dispatch_through_a_one_rank_nccl_group(fp8q):
         _check_dispatch(res, x, ids, 64)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T,k,E,H", [(4096, 8, 256, 7168), (300, 3, 7, 384), (1, 1, 1, 128)])
+def test_scatter_quantizer_matches_oracle(fp8q, T, k, E, H):
+    """Each token quantized once and written to its k layout rows: equal to the
+    oracle's 1x128 quantization of the token for every row, rows untouched
+    elsewhere, dropped entries (position -1) skipped."""
+    import torch
+    x = W.activations_with_outliers(T, H, seed=T + k, channel_frac=2 / H, elem_frac=1e-3)
+    ids = W.moe_routing(T, E, k, n_forced_empty=min(2, E - k), seed=T).expert_ids
+    rows, pos, off = oracle.moe_layout(ids, E)
+    pos = pos.copy()
+    if T > 1:
+        pos[0, 0] = -1                                    # a dropped entry: its row stays untouched
+    M = rows.size + 3                                     # three rows that no entry names
+    q = torch.full((M, H + 16), 0x5A, dtype=torch.uint8, device="cuda")
+    ld = (M + 3) // 4 * 4
+    sf = torch.full((H // 128, ld), -1.0, dtype=torch.float32, device="cuda")
+    fp8q.fp8q_quant_act_1x128_scatter(to_dev_bf16(x), torch.from_numpy(pos.astype(np.int32)).cuda(), q[:, :H], sf)
+    assert fp8q.fp8q_device_status() == 0
+    oq, osf = oracle.quant_act_1x128(x)
+    qh, sh = q.cpu().numpy(), sf.cpu().numpy()
+    written = np.zeros(M, bool)
+    written[pos[pos >= 0]] = True
+    tok_of = np.full(M, -1)
+    tok_of[pos[pos >= 0]] = np.nonzero(pos >= 0)[0]
+    assert np.array_equal(qh[written, :H], oq[tok_of[written]])
+    assert np.array_equal(sh[:, :M][:, written], osf[tok_of[written]].T)
+    assert np.all(qh[~written] == 0x5A) and np.all(sh[:, :M][:, ~written] == -1.0) and np.all(qh[:, H:] == 0x5A)

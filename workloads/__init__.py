@@ -141,6 +141,7 @@ class Routing:
     counts: np.ndarray       # int64 [G]
     empty_experts: np.ndarray
     expert_ids: np.ndarray = None   # int64 [T][top_k]: each token's experts, in its pick order
+    entry_row: np.ndarray = None    # int64 [T][top_k]: the packed row of each (token, pick)
 
 
 def moe_routing(tokens: int = 4096, experts: int = 256, top_k: int = 8, zipf_s: float = 1.1,
@@ -165,8 +166,10 @@ def moe_routing(tokens: int = 4096, experts: int = 256, top_k: int = 8, zipf_s: 
     counts = np.bincount(exp, minlength=experts).astype(np.int64)
     offsets = np.zeros(experts + 1, np.int64)
     offsets[1:] = np.cumsum(counts)
+    entry_row = np.empty(tok.size, np.int64)
+    entry_row[order] = np.arange(tok.size, dtype=np.int64)
     return Routing(offsets=offsets, token_of_row=tok[order], counts=counts, empty_experts=empty,
-                   expert_ids=choice.astype(np.int64))
+                   expert_ids=choice.astype(np.int64), entry_row=entry_row.reshape(tokens, top_k))
 
 
 def expert_weights(G: int, N: int, K: int, seed: int = 0, sigma: float = 0.02,
