@@ -50,7 +50,7 @@ EXPORTS = (
     "fp8q_quant_pertensor", "fp8q_gemm_pertensor", "fp8q_requant_1x128_to_128x1",
     "fp8q_quant_act_1x128_e5m2", "fp8q_quant_act_128x1_e5m2", "fp8q_gemm_blockscaled_fmt",
     "fp8q_moe_dispatch_layout_workspace", "fp8q_moe_dispatch_layout", "fp8q_quant_act_1x128_gather_rowscales",
-    "fp8q_gather_rows_fp8", "fp8q_quant_act_1x128_scatter",
+    "fp8q_gather_rows_fp8", "fp8q_quant_act_1x128_scatter", "fp8q_quant_act_1x128_scatter_rowscales",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
 )
 
@@ -74,6 +74,7 @@ _lib.fp8q_moe_dispatch_layout_workspace.restype = ctypes.c_int64
 _lib.fp8q_moe_dispatch_layout.argtypes = [_P, _I, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_gather_rowscales.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scatter.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_quant_act_1x128_scatter_rowscales.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_gather_rows_fp8.argtypes = [_P, _I, _P, _I, _I, _P, _I, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_pertensor.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_pertensor.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_int, _I, _I, _I, _P]
@@ -278,6 +279,15 @@ def fp8q_quant_act_1x128_scatter(x, pos, q, sf, stream=None):
     k = pos.shape[1]
     _check(_lib.fp8q_quant_act_1x128_scatter(_ptr(x), M_src, K, _ld(x), _ptr(pos), k, q.shape[0], _ptr(q), _ld(q),
                                              _ptr(sf), _ld(sf), _stream(stream)), "fp8q_quant_act_1x128_scatter")
+
+
+def fp8q_quant_act_1x128_scatter_rowscales(x, pos, q, sf, stream=None):
+    """fp8q_quant_act_1x128_scatter with row-major scales sf [M_out][ld >= K/128]."""
+    M_src, K = x.shape
+    k = pos.shape[1]
+    _check(_lib.fp8q_quant_act_1x128_scatter_rowscales(_ptr(x), M_src, K, _ld(x), _ptr(pos), k, q.shape[0], _ptr(q),
+                                                       _ld(q), _ptr(sf), _ld(sf), _stream(stream)),
+           "fp8q_quant_act_1x128_scatter_rowscales")
 
 
 def fp8q_gather_rows_fp8(q_in, sf_in, rows, q_out, sf_out, stream=None):

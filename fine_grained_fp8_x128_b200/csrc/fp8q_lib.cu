@@ -42,6 +42,7 @@ struct DeviceInfo {
   int q1e5_per_sm = 0;
   int q1gr_per_sm = 0;
   int q1sc_per_sm = 0;
+  int q1scr_per_sm = 0;
   int q2e5_per_sm = 0;
   bool q2e5_attr = false;
   int pt_amax_per_sm = 0;
@@ -464,6 +465,30 @@ fp8q_status quant_128x1_impl(const void* x, int64_t T, int64_t C, int64_t ldx, v
   return launch_status();
 }
 
+// Body of both scatter quantizer entries.
+template <bool kRowScales>
+fp8q_status quant_scatter_impl(const void* x, int64_t M_src, int64_t K, int64_t ldx, const int32_t* pos, int k,
+                               int64_t M_out, void* q, int64_t ldq, float* sf, int64_t ld_sf, void* stream) {
+  if (M_src < 0 || M_out < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < (kRowScales ? K / 128 : M_out) || k < 1 ||
+      k > fp8q::kScatterMaxK)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M_src == 0 || M_out == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || pos == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || !aligned(pos, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M_src + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
+  auto kern = fp8q::quant_act_1x128_scatter_kernel<kRowScales>;
+  const int per_sm = blocks_per_sm(kRowScales ? &dev->q1scr_per_sm : &dev->q1sc_per_sm, kern, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  kern<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M_src, KB, ldx, pos, k, M_out, static_cast<uint8_t*>(q), ldq, sf, ld_sf);
+  return launch_status();
+}
+
 extern "C" {
 
 int fp8q_version(void) { return 100; }
@@ -526,24 +551,13 @@ fp8q_status fp8q_quant_act_1x128_gather(const void* x, int64_t M_src, int64_t K,
 fp8q_status fp8q_quant_act_1x128_scatter(const void* x, int64_t M_src, int64_t K, int64_t ldx, const int32_t* pos,
                                          int k, int64_t M_out, void* q, int64_t ldq, float* sf, int64_t ld_sf,
                                          void* stream) {
-  if (M_src < 0 || M_out < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K || ld_sf < M_out || k < 1 ||
-      k > fp8q::kScatterMaxK)
-    return FP8Q_ERR_INVALID_ARG;
-  if (M_src == 0 || M_out == 0 || K == 0) return FP8Q_OK;
-  if (x == nullptr || pos == nullptr || q == nullptr || sf == nullptr) return FP8Q_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf, 4) || !aligned(pos, 4) || ldx % 8 != 0 || ldq % 16 != 0)
-    return FP8Q_ERR_ALIGNMENT;
-  DeviceInfo* dev = nullptr;
-  fp8q_status st = device_info(&dev);
-  if (st != FP8Q_OK) return st;
-  const int64_t KB = K / 128;
-  const int64_t items = ((M_src + fp8q::kQ1Rows - 1) / fp8q::kQ1Rows) * KB;
-  const int per_sm = blocks_per_sm(&dev->q1sc_per_sm, fp8q::quant_act_1x128_scatter_kernel, fp8q::kQ1Threads, 0);
-  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
-  fp8q::quant_act_1x128_scatter_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0,
-                                         static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x), M_src, KB, ldx, pos, k, M_out, static_cast<uint8_t*>(q), ldq, sf, ld_sf);
-  return launch_status();
+  return quant_scatter_impl<false>(x, M_src, K, ldx, pos, k, M_out, q, ldq, sf, ld_sf, stream);
+}
+
+fp8q_status fp8q_quant_act_1x128_scatter_rowscales(const void* x, int64_t M_src, int64_t K, int64_t ldx,
+                                                   const int32_t* pos, int k, int64_t M_out, void* q, int64_t ldq,
+                                                   float* sf, int64_t ld_sf, void* stream) {
+  return quant_scatter_impl<true>(x, M_src, K, ldx, pos, k, M_out, q, ldq, sf, ld_sf, stream);
 }
 
 fp8q_status fp8q_quant_act_1x128_gather_rowscales(const void* x, int64_t M_src, int64_t K, int64_t ldx,

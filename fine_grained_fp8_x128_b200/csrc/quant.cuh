@@ -150,10 +150,11 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
 // same token is not re-read and re-quantized per routed copy.  A negative
 // position (a dropped entry) is skipped; one at or above M_out records
 // FP8Q_ERR_INVALID_ARG and is skipped.  Output rows no entry maps to are not
-// written.
+// written.  kRowScales writes the scales row-major (the exchange's send layout).
 // ---------------------------------------------------------------------------
 constexpr int kScatterMaxK = 64;
 
+template <bool kRowScales = false>
 __global__ void __launch_bounds__(kQ1Threads)
 quant_act_1x128_scatter_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t KB, int64_t ldx,
                                const int32_t* __restrict__ pos, int k, int64_t M_out, uint8_t* __restrict__ q,
@@ -200,7 +201,12 @@ quant_act_1x128_scatter_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, i
         uint8_t* d = q + dst * ldq + kb * 128 + sub * 8;
 #pragma unroll
         for (int i = 0; i < 4; ++i) __stcs(reinterpret_cast<uint2*>(d + 32 * i), o[i]);
-        if (sub == 0) sf[kb * ld_sf + dst] = s;
+        if (sub == 0) {
+          if (kRowScales)
+            sf[dst * ld_sf + kb] = s;
+          else
+            sf[kb * ld_sf + dst] = s;
+        }
       }
     }
     cur = nxt;

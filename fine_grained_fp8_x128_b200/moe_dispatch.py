@@ -11,8 +11,8 @@ contiguous ranges over the ranks of the process group.  One call:
      needs the split sizes; without a process group nothing is exchanged: each
      token is quantized once and scattered to its rows of the grouped GEMM's
      input, and the host never waits);
-  3. gather-quantize (device): each routed token's 1x128 FP8 codes and
-     row-major scales written straight into the send buffer;
+  3. quantize (device): each token's 1x128 FP8 codes and row-major scales,
+     computed once and written straight to its rows of the send buffer;
   4. all_to_all_single of the per-(rank, local expert) row counts, then of the
      codes and of the scales (NCCL over NVLink on GPUs);
   5. regroup (device): the received rows from (source, expert) order into
@@ -37,14 +37,16 @@ class CudaDispatchOps:
         from . import moe_dispatch_layout
         return moe_dispatch_layout(expert_ids, num_experts)
 
-    def gather_quant(self, x, rows):
+    def quant_send(self, x, pos, M):
+        """The send buffer: each token quantized once and written to its M-row
+        layout positions, scales row-major so that they travel with their rows."""
         import torch
-        from . import fp8q_quant_act_1x128_gather_rowscales
-        M, K = rows.numel(), x.shape[1]
+        from . import fp8q_quant_act_1x128_scatter_rowscales
+        K = x.shape[1]
         q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
         sf = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
-        if M > 0:
-            fp8q_quant_act_1x128_gather_rowscales(x, rows, q, sf)
+        if M > 0 and x.shape[0] > 0:
+            fp8q_quant_act_1x128_scatter_rowscales(x, pos, q, sf)
         return q, sf
 
     def quant_grouped(self, x, pos, M):
@@ -121,7 +123,7 @@ def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchR
     off = offsets.cpu().numpy().astype(np.int64)                         # one host sync: the split sizes
     per_expert = np.diff(off)
     send_counts = per_expert.reshape(world, el).sum(axis=1)
-    q_send, sf_send = ops.gather_quant(x, rows)
+    q_send, sf_send = ops.quant_send(x, pos, expert_ids.numel())
     counts_send = torch.from_numpy(per_expert.reshape(world, el).astype(np.int64)).to(x.device)
     counts_recv = torch.empty_like(counts_send)
     dist.all_to_all_single(counts_recv, counts_send, group=group)

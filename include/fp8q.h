@@ -169,6 +169,11 @@ fp8q_status fp8q_moe_dispatch_layout(const int32_t* expert_ids, int64_t n_entrie
 fp8q_status fp8q_quant_act_1x128_scatter(const void* x, int64_t M_src, int64_t K, int64_t ldx,
                                          const int32_t* pos, int k, int64_t M_out,
                                          void* q, int64_t ldq, float* sf, int64_t ld_sf, void* stream);
+/* The same with the scales written row-major, sf[m * ld_sf + kb] (ld_sf >=
+ * K/128): the exchange's send layout. */
+fp8q_status fp8q_quant_act_1x128_scatter_rowscales(const void* x, int64_t M_src, int64_t K, int64_t ldx,
+                                                   const int32_t* pos, int k, int64_t M_out,
+                                                   void* q, int64_t ldq, float* sf, int64_t ld_sf, void* stream);
 
 /*
  * fp8q_quant_act_1x128_gather with the scales written row-major,

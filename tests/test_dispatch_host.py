@@ -41,9 +41,15 @@ class OracleOps:
         rows, pos, off = oracle.moe_layout(expert_ids.numpy(), num_experts)
         return torch.from_numpy(rows), torch.from_numpy(pos), torch.from_numpy(off)
 
-    def gather_quant(self, x, rows):
+    def quant_send(self, x, pos, M):
         import torch
-        q, sf = oracle.quant_act_1x128(x.numpy()[rows.numpy()])
+        qx, sx = oracle.quant_act_1x128(x.numpy())
+        p = pos.numpy()
+        tok = np.nonzero(p >= 0)[0]
+        q = np.zeros((M, qx.shape[1]), np.uint8)
+        sf = np.zeros((M, sx.shape[1]), np.float32)
+        q[p[p >= 0]] = qx[tok]
+        sf[p[p >= 0]] = sx[tok]
         return torch.from_numpy(q), torch.from_numpy(sf)
 
     def regroup(self, q, sf, rows):

@@ -161,3 +161,22 @@ def test_scatter_quantizer_matches_oracle(fp8q, T, k, E, H):
     assert np.array_equal(qh[written, :H], oq[tok_of[written]])
     assert np.array_equal(sh[:, :M][:, written], osf[tok_of[written]].T)
     assert np.all(qh[~written] == 0x5A) and np.all(sh[:, :M][:, ~written] == -1.0) and np.all(qh[:, H:] == 0x5A)
+
+
+def test_scatter_rowscales_matches_oracle(fp8q):
+    """The send-buffer form: scales row-major, sf[row][kb]."""
+    import torch
+    T, k, E, H = 500, 4, 16, 512
+    x = W.activations_with_outliers(T, H, seed=7, channel_frac=2 / H, elem_frac=1e-3)
+    ids = W.moe_routing(T, E, k, n_forced_empty=2, seed=7).expert_ids
+    rows, pos, off = oracle.moe_layout(ids, E)
+    M = rows.size
+    q = torch.full((M, H), 0x5A, dtype=torch.uint8, device="cuda")
+    sf = torch.full((M, H // 128 + 2), -1.0, dtype=torch.float32, device="cuda")
+    fp8q.fp8q_quant_act_1x128_scatter_rowscales(to_dev_bf16(x), torch.from_numpy(pos.astype(np.int32)).cuda(), q,
+                                                sf[:, :H // 128])
+    assert fp8q.fp8q_device_status() == 0
+    oq, osf = oracle.quant_act_1x128(x)
+    sh = sf.cpu().numpy()
+    assert np.array_equal(q.cpu().numpy(), oq[rows])
+    assert np.array_equal(sh[:, :H // 128], osf[rows]) and np.all(sh[:, H // 128:] == -1.0)
