@@ -82,9 +82,15 @@ def regroup_order(recv_counts: np.ndarray):
     src_base[1:] = np.cumsum(recv_counts.sum(axis=1))
     within = np.zeros((world, el + 1), np.int64)
     within[:, 1:] = np.cumsum(recv_counts, axis=1)
-    pieces = [src_base[s] + within[s, e] + np.arange(recv_counts[s, e], dtype=np.int64)
-              for e in range(el) for s in range(world)]
-    rows = np.concatenate(pieces).astype(np.int32) if pieces else np.zeros(0, np.int32)
+    # piece (e, s) -- expert-major, source-minor -- is a run of receive rows
+    # starting at src_base[s] + within[s, e]; output row i of a piece that
+    # begins at output row o maps to its start + (i - o)
+    cnt = recv_counts.T.reshape(-1)
+    start = (src_base[:world, None] + within[:, :el]).T.reshape(-1)
+    out_start = np.zeros(cnt.size, np.int64)
+    out_start[1:] = np.cumsum(cnt)[:-1]
+    total = int(cnt.sum())
+    rows = (np.repeat(start - out_start, cnt) + np.arange(total, dtype=np.int64)).astype(np.int32)
     offsets = np.zeros(el + 1, np.int32)
     offsets[1:] = np.cumsum(recv_counts.sum(axis=0))
     return rows, offsets

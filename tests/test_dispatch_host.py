@@ -33,6 +33,25 @@ def test_regroup_order_is_a_permutation():
     assert off[-1] == counts.sum() and np.array_equal(np.diff(off), counts.sum(axis=0))
 
 
+def test_regroup_order_against_a_loop():
+    """Random count tables (empty sources and experts included) against the
+    order written out piece by piece."""
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        world, el = int(rng.integers(1, 9)), int(rng.integers(1, 40))
+        counts = rng.integers(0, 6, (world, el))
+        counts[rng.random((world, el)) < 0.3] = 0
+        base = np.concatenate([[0], np.cumsum(counts.sum(axis=1))])
+        want = []
+        for e in range(el):
+            for s in range(world):
+                first = base[s] + counts[s, :e].sum()
+                want.extend(range(first, first + counts[s, e]))
+        rows, off = regroup_order(counts)
+        assert rows.tolist() == want
+        assert off.tolist() == [0] + np.cumsum(counts.sum(axis=0)).tolist()
+
+
 class OracleOps:
     """The dispatch's device steps done by the oracle, on CPU tensors."""
 
