@@ -76,6 +76,23 @@ class OracleOps:
         r = rows.numpy()
         return torch.from_numpy(q.numpy()[r]), torch.from_numpy(np.ascontiguousarray(sf.numpy()[r].T))
 
+    def quant_grouped(self, x, pos, M):
+        import torch
+        q, sf = self.quant_send(x, pos, M)
+        return q, torch.from_numpy(np.ascontiguousarray(sf.numpy().T))
+
+
+def test_dispatch_without_a_process_group():
+    """One process, all experts local: no exchange, the layout order is the
+    grouped GEMM's, and the result equals the one-rank reference."""
+    import torch
+    x, ids = _inputs(0, 80, 256, 4, 8)
+    res = dispatch(torch.from_numpy(x), torch.from_numpy(ids.astype(np.int32)), 8, ops=OracleOps())
+    (q, sf, off), = oracle.moe_dispatch_reference([x], [ids], 8)
+    assert np.array_equal(res.q.numpy(), q) and np.array_equal(res.sf.numpy().T, sf)
+    assert np.array_equal(res.expert_offsets.numpy(), off)
+    assert res.send_counts is None and res.recv_counts is None
+
 
 def _inputs(rank, T, H, k, E):
     x = W.activations_with_outliers(T, H, seed=100 + rank, channel_frac=2 / H, elem_frac=1e-3)
