@@ -73,6 +73,57 @@ def test_history_update_special_cases():
     assert np.all(he >= lo * (1 - 2 ** -22)) and np.all(he <= hi * (1 + 2 ** -22))
 
 
+ALPHAS = (0.1, 0.37, 0.9, 0.999)
+
+
+def _ema_pairs(seed, n=4096):
+    rng = np.random.default_rng(seed)
+    a = np.exp(rng.uniform(-8, 6, n)).astype(np.float32)
+    h = np.exp(rng.uniform(-8, 6, n)).astype(np.float32)
+    return a, h
+
+
+@pytest.mark.parametrize("alpha", ALPHAS)
+def test_ema_history_bit_exact_against_numpy_float32(alpha):
+    """The exponential history rounds every operation to FP32 on its own:
+    beta = fl32(1 - alpha), h' = fl32(fl32(alpha * h) + fl32(beta * a))
+    ("Online Quantization During Training", section 4 and its worked example:
+    an exponential moving history of the tile maxima).  NumPy float32
+    arithmetic rounds each operation once, so it states the same value
+    independently of the oracle's C++."""
+    a, h = _ema_pairs(seed=int(alpha * 1000))
+    got, sf = oracle.scale_history_update(oracle.POLICY_EMA, alpha, a, h)
+    al = np.float32(alpha)
+    beta = np.float32(np.float32(1.0) - al)
+    want = (np.float32(al * h) + np.float32(beta * a)).astype(np.float32)
+    assert want.dtype == np.float32
+    assert np.array_equal(got, want)
+    tile = np.vectorize(oracle.tile_scale, otypes=[np.float32])
+    assert np.array_equal(sf, tile(want))
+
+
+def test_ema_pin_separates_plausible_variants():
+    """The pin above would catch the plausible mistakes: a fused multiply-add
+    (one rounding of alpha*h + r), beta = 1 - alpha kept in double, or the
+    whole update in double and rounded once.  Each of them differs from the
+    oracle on some of the same inputs."""
+    fma_diff = dbl_beta_diff = all_dbl_diff = 0
+    for alpha in ALPHAS:
+        a, h = _ema_pairs(seed=int(alpha * 1000))
+        got, _ = oracle.scale_history_update(oracle.POLICY_EMA, alpha, a, h)
+        al = np.float32(alpha)
+        beta = np.float32(np.float32(1.0) - al)
+        r = (beta * a).astype(np.float32)
+        fma = (np.float64(al) * h.astype(np.float64) + r.astype(np.float64)).astype(np.float32)
+        beta64 = np.float64(1.0) - np.float64(al)
+        dbl_beta = (np.float32(al * h) + (beta64 * a.astype(np.float64)).astype(np.float32)).astype(np.float32)
+        all_dbl = (np.float64(al) * h.astype(np.float64) + beta64 * a.astype(np.float64)).astype(np.float32)
+        fma_diff += int((fma != got).sum())
+        dbl_beta_diff += int((dbl_beta != got).sum())
+        all_dbl_diff += int((all_dbl != got).sum())
+    assert fma_diff > 0 and dbl_beta_diff > 0 and all_dbl_diff > 0, (fma_diff, dbl_beta_diff, all_dbl_diff)
+
+
 def test_bad_policy_is_rejected():
     with pytest.raises(Exception):
         oracle.scale_history_update(3, 0.5, np.ones(4, np.float32), np.ones(4, np.float32))
