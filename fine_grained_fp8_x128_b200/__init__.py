@@ -40,6 +40,9 @@ FP8Q_OUT_BF16 = 0
 FP8Q_OUT_F32 = 1
 FP8Q_FMT_E4M3 = 0
 FP8Q_FMT_E5M2 = 1
+FP8Q_DENSE_AUTO = 0
+FP8Q_DENSE_SINGLE = 1
+FP8Q_DENSE_PAIR = 2
 
 EXPORTS = (
     "fp8q_version", "fp8q_status_string", "fp8q_device_status",
@@ -51,7 +54,7 @@ EXPORTS = (
     "fp8q_quant_act_1x128_e5m2", "fp8q_quant_act_128x1_e5m2", "fp8q_gemm_blockscaled_fmt",
     "fp8q_moe_dispatch_layout_workspace", "fp8q_moe_dispatch_layout", "fp8q_quant_act_1x128_gather_rowscales",
     "fp8q_gather_rows_fp8", "fp8q_quant_act_1x128_scatter", "fp8q_quant_act_1x128_scatter_rowscales",
-    "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout",
+    "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
 )
 
 _P = ctypes.c_void_p
@@ -89,6 +92,7 @@ _lib.fp8q_grouped_gemm_blockscaled_q1x128.argtypes = [_P, _I, _P, _I, _P, _P, _P
                                                       _P]
 _lib.fp8q_debug_cast_e4m3_bits.argtypes = [ctypes.c_uint32, _I, _P, _P]
 _lib.fp8q_debug_wait_timeout.argtypes = [_I, _P]
+_lib.fp8q_debug_force_dense_kernel.argtypes = [ctypes.c_int]
 for _n in EXPORTS[2:]:
     getattr(_lib, _n).restype = ctypes.c_int
 
@@ -139,7 +143,7 @@ def fp8q_device_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word (0 = clean)."""
     code = ctypes.c_int(0)
     rc = _lib.fp8q_device_status(_stream(stream), ctypes.byref(code))
-    if rc not in (FP8Q_OK, FP8Q_ERR_TIMEOUT):
+    if rc not in (FP8Q_OK, FP8Q_ERR_TIMEOUT, FP8Q_ERR_INVALID_ARG):
         raise FP8QError(rc, "fp8q_device_status")
     return code.value
 
@@ -345,6 +349,11 @@ def fp8q_grouped_gemm_blockscaled_q1x128(a, sfa, w, sfw, group_offsets, dq, sfd,
 def fp8q_debug_cast_e4m3_bits(start: int, count: int, out, stream=None):
     _check(_lib.fp8q_debug_cast_e4m3_bits(ctypes.c_uint32(start & 0xFFFFFFFF), count, _ptr(out), _stream(stream)),
            "fp8q_debug_cast_e4m3_bits")
+
+
+def fp8q_debug_force_dense_kernel(choice: int):
+    """FP8Q_DENSE_AUTO / FP8Q_DENSE_SINGLE / FP8Q_DENSE_PAIR for later dense GEMM calls."""
+    _check(_lib.fp8q_debug_force_dense_kernel(int(choice)), "fp8q_debug_force_dense_kernel")
 
 
 def fp8q_debug_wait_timeout(budget_cycles: int, stream=None):

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -255,18 +256,22 @@ int64_t pair_group_m(int64_t m_pairs, int64_t a_bytes, int64_t b_bytes) {
   return m_pairs < 8 ? m_pairs : 8;
 }
 
+// Dense kernel choice set by fp8q_debug_force_dense_kernel (a test hook):
+// FP8Q_DENSE_AUTO, FP8Q_DENSE_SINGLE or FP8Q_DENSE_PAIR.
+std::atomic<int> g_dense_choice{FP8Q_DENSE_AUTO};
+
 // Which dense kernel runs: the CTA-pair kernel (256 x 256 tiles) when A has
 // more than one 128-row tile (the faster of the two on B200, both in short
 // bursts and under the power cap), else the one-CTA kernel (128 x 256 tiles),
 // which wastes no tensor-core rows on a short A.  The pair kernel TMA-loads
 // the scale factors, so it also needs both scale arrays 16-byte aligned with
-// leading dimensions that are multiples of 4 floats.  FP8Q_DENSE_KERNEL=single
-// or =pair forces one of them where it applies (the tests run both).
+// leading dimensions that are multiples of 4 floats.  A forced choice applies
+// where the kernel can run (the tests run both).
 bool use_pair_kernel(int64_t M, const float* sfa, int64_t ld_sfa, const float* sfb, int64_t ld_sfb) {
   const bool fits = aligned(sfa, 16) && aligned(sfb, 16) && ld_sfa % 4 == 0 && ld_sfb % 4 == 0;
-  const char* e = std::getenv("FP8Q_DENSE_KERNEL");
-  if (!fits || (e != nullptr && std::strcmp(e, "single") == 0)) return false;
-  if (e != nullptr && std::strcmp(e, "pair") == 0) return true;
+  const int choice = g_dense_choice.load(std::memory_order_relaxed);
+  if (!fits || choice == FP8Q_DENSE_SINGLE) return false;
+  if (choice == FP8Q_DENSE_PAIR) return true;
   return M > fp8q::BM;
 }
 
@@ -516,7 +521,11 @@ fp8q_status fp8q_device_status(void* stream, int* out_code) {
     return FP8Q_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return FP8Q_ERR_CUDA;
   *out_code = static_cast<int>(word);
-  return word == 0 ? FP8Q_OK : FP8Q_ERR_TIMEOUT;
+  if (word == 0) return FP8Q_OK;
+  // bits 0-7 hold the FP8Q_ERR_* code of the first report
+  const unsigned int code = word & 0xFFu;
+  return code == FP8Q_ERR_INVALID_ARG || code == FP8Q_ERR_TIMEOUT ? static_cast<fp8q_status>(code)
+                                                                  : FP8Q_ERR_CUDA;
 }
 
 fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
@@ -898,6 +907,13 @@ fp8q_status fp8q_debug_cast_e4m3_bits(uint32_t start, int64_t count, void* out, 
   fp8q::cast_e4m3_bits_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       start, count, static_cast<uint8_t*>(out));
   return launch_status();
+}
+
+fp8q_status fp8q_debug_force_dense_kernel(int choice) {
+  if (choice != FP8Q_DENSE_AUTO && choice != FP8Q_DENSE_SINGLE && choice != FP8Q_DENSE_PAIR)
+    return FP8Q_ERR_INVALID_ARG;
+  g_dense_choice.store(choice, std::memory_order_relaxed);
+  return FP8Q_OK;
 }
 
 fp8q_status fp8q_debug_wait_timeout(int64_t budget_cycles, void* stream) {

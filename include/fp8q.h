@@ -20,7 +20,10 @@
  *  - Outputs are written entirely (no accumulation into an existing output).
  *    Inputs and outputs must not overlap.
  *  - Inputs are finite BF16 values; behaviour for Inf/NaN inputs is unspecified.
- *  - The library allocates no per-call memory and no workspace.
+ *  - The library allocates no per-call memory.  Its only state is one
+ *    device-side status word per device.  One call needs scratch space, and
+ *    the caller passes it: fp8q_moe_dispatch_layout takes a workspace sized
+ *    by fp8q_moe_dispatch_layout_workspace.
  *  - E4M3 is the OCP "E4M3FN" encoding (bias 7, max 448, no infinities).
  *    The cast is round-to-nearest-even with saturation to +-448.
  *  - Tile scale: s = max(fl32(amax / 448), fl32(1e-12)), IEEE FP32 division;
@@ -82,9 +85,12 @@ const char* fp8q_status_string(fp8q_status s);
 /*
  * Synchronise `stream`, then read and clear this device's sticky device-side
  * status word.  *out_code receives the raw word: 0 when no kernel reported a
- * problem; otherwise bits 0-7 hold an FP8Q_ERR_* code and bits 8-31 say which
- * wait gave up.  Returns FP8Q_OK, FP8Q_ERR_TIMEOUT when the word was non-zero,
- * or FP8Q_ERR_CUDA.
+ * problem; otherwise bits 0-7 hold the FP8Q_ERR_* code of the first report and
+ * bits 8-31 say where it happened (which wait gave up, or which input check
+ * failed).  Returns FP8Q_OK for a clean word, else the code in bits 0-7:
+ * FP8Q_ERR_TIMEOUT (a bounded wait gave up) or FP8Q_ERR_INVALID_ARG (a
+ * device-side input check failed: group offsets, a row index or an expert id
+ * out of range).  FP8Q_ERR_CUDA if reading the word failed.
  */
 fp8q_status fp8q_device_status(void* stream, int* out_code);
 
@@ -466,6 +472,20 @@ fp8q_status fp8q_gemm_pertensor(const void* a, int64_t lda, const float* scale_a
  * with an independent encoder over every FP32 input.  count <= 2^32.
  */
 fp8q_status fp8q_debug_cast_e4m3_bits(uint32_t start, int64_t count, void* out, void* stream);
+
+/*
+ * Force which dense GEMM kernel fp8q_gemm_blockscaled and its variants use,
+ * where it can run: FP8Q_DENSE_AUTO (the default: the CTA-pair kernel when
+ * M > 128), FP8Q_DENSE_SINGLE (the one-CTA kernel) or FP8Q_DENSE_PAIR.  Both
+ * kernels compute the same result; the tests run each.  Process-wide, takes
+ * effect for later calls.  FP8Q_ERR_INVALID_ARG for another value.
+ */
+enum {
+  FP8Q_DENSE_AUTO = 0,
+  FP8Q_DENSE_SINGLE = 1,
+  FP8Q_DENSE_PAIR = 2
+};
+fp8q_status fp8q_debug_force_dense_kernel(int choice);
 
 /*
  * Launch one block that waits on a barrier no thread ever completes, with a

@@ -35,9 +35,11 @@ def fp8q():
 
 
 @pytest.fixture(params=["single", "pair"])
-def dense_kernel(request, monkeypatch):
-    monkeypatch.setenv("FP8Q_DENSE_KERNEL", request.param)
-    return request.param
+def dense_kernel(request, fp8q):
+    """Run a test on the one-CTA kernel and on the CTA-pair kernel."""
+    fp8q.fp8q_debug_force_dense_kernel(fp8q.FP8Q_DENSE_SINGLE if request.param == "single" else fp8q.FP8Q_DENSE_PAIR)
+    yield request.param
+    fp8q.fp8q_debug_force_dense_kernel(fp8q.FP8Q_DENSE_AUTO)
 
 
 def _sf_kmajor(sf_mk, ld=None):

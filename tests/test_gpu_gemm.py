@@ -95,10 +95,11 @@ def test_linear_y_wx_worked_example(fp8q):
 
 
 @pytest.fixture(params=["single", "pair"])
-def dense_kernel(request, monkeypatch):
+def dense_kernel(request, fp8q):
     """Run a test on the one-CTA kernel and on the CTA-pair kernel."""
-    monkeypatch.setenv("FP8Q_DENSE_KERNEL", request.param)
-    return request.param
+    fp8q.fp8q_debug_force_dense_kernel(fp8q.FP8Q_DENSE_SINGLE if request.param == "single" else fp8q.FP8Q_DENSE_PAIR)
+    yield request.param
+    fp8q.fp8q_debug_force_dense_kernel(fp8q.FP8Q_DENSE_AUTO)
 
 
 @pytest.mark.parametrize("M,N,K,mode,f32", [
@@ -200,6 +201,33 @@ def test_forward_gemm_full_size(fp8q):
     qa, sa = oracle.quant_act_1x128(x)
     qb, sb = oracle.quant_w_128x128(W.weights(18432, 7168, seed=0))
     _full_size_check(fp8q, qa, sa, qb, sb, BLK, False, seed=3)
+
+
+@pytest.mark.slow
+def test_forward_gemm_full_output(fp8q):
+    """Every output of the full-size Fprop (8192 x 18432 = 151 M values) against
+    the FP64 oracle, once, in blocks of 512 full rows: about 1.1e12 multiply-adds
+    of oracle work, a minute or two on the host cores."""
+    import torch
+    x = W.activations_with_outliers(8192, 7168, seed=0)
+    qa, sa = oracle.quant_act_1x128(x)
+    qb, sb = oracle.quant_w_128x128(W.weights(18432, 7168, seed=0))
+    M, N = qa.shape[0], qb.shape[0]
+    d = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    fp8q.fp8q_gemm_blockscaled(to_dev_u8(qa), sfa_dev(sa), to_dev_u8(qb), to_dev_f32(sb), BLK, d)
+    torch.cuda.synchronize()
+    assert fp8q.fp8q_device_status() == 0
+    got = d.float().cpu().numpy()
+    del d
+    num = den = 0.0
+    for r0 in range(0, M, 512):
+        rows = np.arange(r0, min(M, r0 + 512), dtype=np.int64)
+        ref = oracle.gemm_sampled(qa, sa, qb, sb, BLK, rows=rows)
+        blk = got[r0:r0 + len(rows)].astype(np.float64)
+        check_gemm(blk, ref, rounded(ref, False))
+        num += float(np.sum((blk - ref) ** 2))
+        den += float(np.sum(ref ** 2))
+    assert np.sqrt(num / den) <= 2e-3
 
 
 def test_backward_gemms_full_size(fp8q):
