@@ -78,8 +78,15 @@ def _load():
     lib.orc_tile_scale_e5m2.restype = ctypes.c_float
     lib.orc_gemm_sampled_fmt.argtypes = [P, I64, P, P, I64, P, ctypes.c_int, I64, I64, I64,
                                          P, I64, P, I64, ctypes.c_int, ctypes.c_int, P]
+    lib.orc_pow2_scale.argtypes = [ctypes.c_float]
+    lib.orc_pow2_scale.restype = ctypes.c_float
+    lib.orc_ue8m0_encode.argtypes = [ctypes.c_float]
+    lib.orc_ue8m0_encode.restype = ctypes.c_int
+    lib.orc_quant_act_1x128_pow2.argtypes = [P, I64, I64, I64, P, I64, P]
+    lib.orc_quant_w_128x128_pow2.argtypes = [P, I64, I64, I64, P, I64, P]
     for name in ("orc_quant_act_1x128", "orc_quant_act_128x1", "orc_quant_w_128x128",
-                 "orc_gemm_sampled", "orc_grouped_gemm_sampled"):
+                 "orc_gemm_sampled", "orc_grouped_gemm_sampled", "orc_quant_act_1x128_pow2",
+                 "orc_quant_w_128x128_pow2"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -234,6 +241,40 @@ def quant_w_128x128(w_bf16: np.ndarray):
     q = np.empty((N, K), np.uint8)
     sf = np.empty((N // 128, K // 128), np.float32)
     _check(_load().orc_quant_w_128x128(_p(w), N, K, K, _p(q), K, _p(sf)), "quant_w_128x128")
+    return q, sf
+
+
+# ---------------------------------------------------------------- power-of-two (UE8M0) scales
+# Not the pages' method (which fixes s = amax/448): a reading for the study of
+# hardware block scaling, which takes power-of-two scales.  The method's scale
+# is rounded up to the next power of two; the tiles stay 1x128 / 128x128.
+def pow2_scale(t: float) -> float:
+    """Smallest power of two >= t (t > 0, a float32 value)."""
+    return float(_load().orc_pow2_scale(float(t)))
+
+
+def ue8m0_encode(s: float) -> int:
+    """UE8M0 byte (biased exponent, 2^(b-127)) of a power of two; -1 otherwise."""
+    return int(_load().orc_ue8m0_encode(float(s)))
+
+
+def quant_act_1x128_pow2(x_bf16: np.ndarray):
+    """1x128 tiles, s2 = 2^ceil(log2 tile_scale(amax)): (q uint8 [M][K], sf float32 [M][K/128])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    sf = np.empty((M, K // 128), np.float32)
+    _check(_load().orc_quant_act_1x128_pow2(_p(x), M, K, K, _p(q), K, _p(sf)), "quant_act_1x128_pow2")
+    return q, sf
+
+
+def quant_w_128x128_pow2(w_bf16: np.ndarray):
+    """128x128 blocks with power-of-two scales: (q uint8 [N][K], sf float32 [N/128][K/128])."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    N, K = w.shape
+    q = np.empty((N, K), np.uint8)
+    sf = np.empty((N // 128, K // 128), np.float32)
+    _check(_load().orc_quant_w_128x128_pow2(_p(w), N, K, K, _p(q), K, _p(sf)), "quant_w_128x128_pow2")
     return q, sf
 
 

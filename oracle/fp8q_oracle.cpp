@@ -347,6 +347,74 @@ int orc_quant_w_128x128(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
   return 0;
 }
 
+// ---- power-of-two (UE8M0) scales: a throughput study beside the method ---------
+// The pages fix the scale as s = amax/448 ([P3] eq. s_W), a full FP32 value.
+// Block-scaled tensor-core MMAs take scales that are powers of two, stored as
+// UE8M0 bytes (an 8-bit biased exponent: byte b stands for 2^(b - 127)).  The
+// pages do not define such a scale; the reading taken here keeps the method's
+// tiles (1x128 activations, 128x128 weight blocks) and rounds the method's
+// scale UP to the next power of two, so no element saturates:
+//   t  = max(fl32(amax / 448), fl32(1e-12))      (the method's scale)
+//   s2 = 2^ceil(log2 t)                          (smallest power of two >= t)
+//   q  = e4m3(fl32(x / s2))
+// The GEMM over such operands is the block-scaled GEMM above with these scales.
+float orc_pow2_scale(float t) {
+  int e = 0;
+  const float m = std::frexp(t, &e);      // t = m * 2^e, 0.5 <= m < 1
+  return m == 0.5f ? t : std::ldexp(1.0f, e);
+}
+
+// UE8M0 byte of a power of two s = 2^p (p in [-127, 127]): p + 127.
+int orc_ue8m0_encode(float s) {
+  int e = 0;
+  const float m = std::frexp(s, &e);      // s = 0.5 * 2^e
+  if (m != 0.5f) return -1;               // not a power of two
+  const int b = (e - 1) + 127;
+  return (b < 0 || b > 254) ? -1 : b;
+}
+
+// 1x128 tiles with power-of-two scales.  x: bf16 [M][ldx]; q: [M][ldq];
+// sf: [M][K/128] row-major (the scale values s2).
+int orc_quant_act_1x128_pow2(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                             uint8_t* q, int64_t ldq, float* sf) {
+  if (K % 128 != 0 || ldx < K || ldq < K || M < 0) return 1;
+  const int64_t KB = K / 128;
+  parallel_for(M, [&](int64_t m) {
+    for (int64_t kb = 0; kb < KB; ++kb) {
+      const uint16_t* t = x + m * ldx + kb * 128;
+      float amax = 0.0f;
+      for (int i = 0; i < 128; ++i) amax = std::max(amax, std::fabs(bf16_to_float(t[i])));
+      const float s = orc_pow2_scale(orc_tile_scale(amax));
+      sf[m * KB + kb] = s;
+      for (int i = 0; i < 128; ++i) q[m * ldq + kb * 128 + i] = e4m3_encode(bf16_to_float(t[i]) / s);
+    }
+  });
+  return 0;
+}
+
+// 128x128 weight blocks with power-of-two scales.  w: bf16 [N][ldw];
+// q: [N][ldq]; sf: [N/128][K/128] row-major.
+int orc_quant_w_128x128_pow2(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                             uint8_t* q, int64_t ldq, float* sf) {
+  if (N % 128 != 0 || K % 128 != 0 || ldw < K || ldq < K) return 1;
+  const int64_t NB = N / 128, KB = K / 128;
+  parallel_for(NB * KB, [&](int64_t b) {
+    const int64_t nb = b / KB, kb = b % KB;
+    float amax = 0.0f;
+    for (int r = 0; r < 128; ++r)
+      for (int c = 0; c < 128; ++c)
+        amax = std::max(amax, std::fabs(bf16_to_float(w[(nb * 128 + r) * ldw + kb * 128 + c])));
+    const float s = orc_pow2_scale(orc_tile_scale(amax));
+    sf[nb * KB + kb] = s;
+    for (int r = 0; r < 128; ++r)
+      for (int c = 0; c < 128; ++c) {
+        const int64_t n = nb * 128 + r, k = kb * 128 + c;
+        q[n * ldq + k] = e4m3_encode(bf16_to_float(w[n * ldw + k]) / s);
+      }
+  });
+  return 0;
+}
+
 // ---- the [P3] listing's integer-grid simulation --------------------------------
 // [P3] "Step 1": q = clip(round(x/s), -448, 448) with numpy's round-half-even,
 // s = max(amax/448, 1e-12), here in double like the listing.  Groups are
