@@ -31,6 +31,8 @@ FP8Q_ERR_ALIGNMENT = 2
 FP8Q_ERR_UNSUPPORTED = 3
 FP8Q_ERR_CUDA = 4
 FP8Q_ERR_TIMEOUT = 5
+FP8Q_ERR_SCRATCH_LIMIT = 6
+FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS = 262144
 FP8Q_SFB_BLOCK128 = 0
 FP8Q_SFB_ROW = 1
 FP8Q_POLICY_PREVIOUS = 0
@@ -55,6 +57,7 @@ EXPORTS = (
     "fp8q_moe_dispatch_layout_workspace", "fp8q_moe_dispatch_layout", "fp8q_quant_act_1x128_gather_rowscales",
     "fp8q_gather_rows_fp8", "fp8q_quant_act_1x128_scatter", "fp8q_quant_act_1x128_scatter_rowscales",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
+    "fp8q_moe_dispatch_layout_noalloc",
 )
 
 _P = ctypes.c_void_p
@@ -75,6 +78,7 @@ _lib.fp8q_gemm_blockscaled_fmt.argtypes = [_P, ctypes.c_int, _I, _P, _I, _P, cty
 _lib.fp8q_moe_dispatch_layout_workspace.argtypes = [_I, ctypes.c_int]
 _lib.fp8q_moe_dispatch_layout_workspace.restype = ctypes.c_int64
 _lib.fp8q_moe_dispatch_layout.argtypes = [_P, _I, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _I, _P]
+_lib.fp8q_moe_dispatch_layout_noalloc.argtypes = [_P, _I, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P]
 _lib.fp8q_quant_act_1x128_gather_rowscales.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scatter.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scatter_rowscales.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
@@ -253,6 +257,17 @@ def fp8q_moe_dispatch_layout(expert_ids, num_experts, rows, pos, offsets, worksp
     _check(_lib.fp8q_moe_dispatch_layout(_ptr(expert_ids), T * k, k, int(num_experts), _ptr(rows), _ptr(pos),
                                          _ptr(offsets), _ptr(workspace), workspace.numel(), _stream(stream)),
            "fp8q_moe_dispatch_layout")
+
+
+def fp8q_moe_dispatch_layout_noalloc(expert_ids, num_experts, rows, pos, offsets, stream=None):
+    """fp8q_moe_dispatch_layout with no workspace argument: the library's fixed
+    scratch array (FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS int32) is used instead, so
+    the call allocates nothing.  For callers that cannot allocate device memory
+    when they call; calls that overlap on the GPU race on the shared array."""
+    T, k = expert_ids.shape
+    _check(_lib.fp8q_moe_dispatch_layout_noalloc(_ptr(expert_ids), T * k, k, int(num_experts), _ptr(rows), _ptr(pos),
+                                                 _ptr(offsets), _stream(stream)),
+           "fp8q_moe_dispatch_layout_noalloc")
 
 
 def moe_dispatch_layout(expert_ids, num_experts, stream=None):

@@ -506,6 +506,7 @@ const char* fp8q_status_string(fp8q_status s) {
     case FP8Q_ERR_UNSUPPORTED: return "unsupported configuration or device";
     case FP8Q_ERR_CUDA: return "CUDA error";
     case FP8Q_ERR_TIMEOUT: return "device-side bounded wait gave up";
+    case FP8Q_ERR_SCRATCH_LIMIT: return "request needs more scratch than the fixed no-allocation array holds";
     default: return "unknown status";
   }
 }
@@ -926,3 +927,77 @@ fp8q_status fp8q_debug_wait_timeout(int64_t budget_cycles, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fp8q_moe_dispatch_layout_noalloc: the dispatch layout with its scratch in a
+// fixed array of this library's device module instead of a caller workspace.
+// For callers that cannot allocate device memory at the time they call (see
+// the declaration in fp8q.h).  The array is FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS
+// int32 (1 MiB) and every device that loads the library holds it until the
+// process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t g_layout_scratch[FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS];
+
+namespace {
+
+int32_t* g_layout_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_layout_scratch on the current device.  In host code the
+// array's name stands for a host-side shadow, not device memory, so the
+// address is looked up once per device (with that device current) and kept.
+fp8q_status layout_scratch_address(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_layout_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr) return FP8Q_ERR_CUDA;
+    g_layout_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_layout_scratch_ptr[dev];
+  return FP8Q_OK;
+}
+
+}  // namespace
+
+extern "C" fp8q_status fp8q_moe_dispatch_layout_noalloc(const int32_t* expert_ids, int64_t n_entries, int k,
+                                                        int num_experts, int32_t* rows, int32_t* pos,
+                                                        int32_t* offsets, void* stream) {
+  if (n_entries < 0 || k < 1 || num_experts < 1 || num_experts > fp8q::kLayoutMaxExperts || n_entries % k != 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (n_entries > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+  // the scratch this request needs must fit the fixed array
+  if (fp8q_moe_dispatch_layout_workspace(n_entries, num_experts) > FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS)
+    return FP8Q_ERR_SCRATCH_LIMIT;
+  if (offsets == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (n_entries > 0 && (expert_ids == nullptr || rows == nullptr || pos == nullptr)) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(offsets, 4) ||
+      (n_entries > 0 && (!aligned(expert_ids, 4) || !aligned(rows, 4) || !aligned(pos, 4))))
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  int32_t* scratch = nullptr;
+  if ((st = layout_scratch_address(&scratch)) != FP8Q_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_entries == 0) {
+    // offsets are all zero; no kernel runs and the scratch is not touched
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (num_experts + 1), s) != cudaSuccess) return FP8Q_ERR_CUDA;
+    return FP8Q_OK;
+  }
+  // Every scratch word the kernels read is written earlier in the same call
+  // (per-chunk histograms, then per-chunk starts), so nothing needs clearing.
+  const int64_t chunks = layout_chunks(n_entries);
+  const int64_t chunk = (n_entries + chunks - 1) / chunks;
+  int32_t* hist = scratch;
+  int32_t* starts = scratch + chunks * num_experts;
+  fp8q::moe_layout_hist_kernel<<<static_cast<unsigned>(chunks), 256, 0, s>>>(expert_ids, n_entries, num_experts, chunk,
+                                                                            hist);
+  if ((st = launch_status()) != FP8Q_OK) return st;
+  fp8q::moe_layout_scan_kernel<<<1, fp8q::kLayoutMaxExperts, 0, s>>>(hist, static_cast<int>(chunks), num_experts,
+                                                                    offsets, starts);
+  if ((st = launch_status()) != FP8Q_OK) return st;
+  fp8q::moe_layout_scatter_kernel<<<static_cast<unsigned>(chunks), 32, 0, s>>>(expert_ids, n_entries, k, num_experts,
+                                                                               chunk, starts, rows, pos);
+  return launch_status();
+}

@@ -47,7 +47,8 @@ enum {
   FP8Q_ERR_ALIGNMENT = 2,    /* a pointer or leading dimension is misaligned    */
   FP8Q_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement     */
   FP8Q_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed     */
-  FP8Q_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (device status) */
+  FP8Q_ERR_TIMEOUT = 5,      /* a kernel gave up a bounded wait (device status) */
+  FP8Q_ERR_SCRATCH_LIMIT = 6 /* request exceeds a fixed no-allocation scratch     */
 };
 
 /* Scale layouts for operand B of fp8q_gemm_blockscaled. */
@@ -158,6 +159,37 @@ int64_t fp8q_moe_dispatch_layout_workspace(int64_t n_entries, int num_experts);
 fp8q_status fp8q_moe_dispatch_layout(const int32_t* expert_ids, int64_t n_entries, int k, int num_experts,
                                      int32_t* rows, int32_t* pos, int32_t* offsets,
                                      int32_t* workspace, int64_t workspace_len, void* stream);
+
+/*
+ * fp8q_moe_dispatch_layout for callers that cannot allocate device memory when
+ * they call.  Some callers have no allocator to use: a plugin that a host
+ * framework calls to enqueue work, where the framework owns all device memory
+ * and hands the plugin no workspace; a runtime that reserved its whole memory
+ * budget at start-up; a latency-critical path where cudaMalloc's implicit
+ * device synchronisation is not allowed.  This entry point takes no workspace
+ * and allocates nothing (no cudaMalloc, cudaFree or allocating library call):
+ * its scratch is a fixed array of FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS int32
+ * (1 MiB) in the library's device module, which every GPU that loads the
+ * library holds until the process exits.  The pages have no counterpart to
+ * this call; it is an interface for such callers only.
+ *   Arguments, results and device-side reports: as fp8q_moe_dispatch_layout
+ *   (rows, pos, offsets are caller-owned device buffers).
+ *   Limit: fp8q_moe_dispatch_layout_workspace(n_entries, num_experts) must not
+ *   exceed FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS (for 256 experts any n_entries; for
+ *   1024 experts up to 32768 entries); a larger request returns
+ *   FP8Q_ERR_SCRATCH_LIMIT and launches nothing.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *   first call before any stream capture.
+ *   Every call shares the one array and it keeps the last call's contents.
+ *   The call needs no cleared scratch: each word it reads it wrote earlier in
+ *   the same call.  Calls whose kernels overlap on the GPU (other streams, or
+ *   other host threads on the same device) race on the array: order them on
+ *   one stream or with events.
+ */
+enum { FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS = 262144 };
+fp8q_status fp8q_moe_dispatch_layout_noalloc(const int32_t* expert_ids, int64_t n_entries, int k, int num_experts,
+                                             int32_t* rows, int32_t* pos, int32_t* offsets, void* stream);
 
 /*
  * The dispatch quantizer from the token side: each source row of x is
