@@ -716,7 +716,7 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("linear_y_wx", "quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "quant_moe_x_gather", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("linear_y_wx", "mx_fprop", "fprop_single", "quant_x_ue8m0", "quant_w_ue8m0", "quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "quant_moe_x_gather", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -752,6 +752,28 @@ def run_single(args):
             fp8q.fp8q_quant_w_128x128(wd, qw, sw)
             fp8q.fp8q_gemm_blockscaled(qx, sx, qw, sw, fp8q.FP8Q_SFB_BLOCK128, y)
         work = ("flops", 2.0 * 256 * 128)
+    elif name == "mx_fprop":
+        # power-of-two (UE8M0) scale study: the Fprop shape on the block-scaled MMA, all of K in TMEM
+        M, N, K = T, OUT, HID
+        qa, sfa = fp8q.quant_act_1x128_ue8m0(randn(M, K))
+        qb, sfb = fp8q.quant_w_128x128_ue8m0(randn(N, K, sigma=0.02))
+        d = torch.empty((M, N), dtype=bf, device=dev)
+        fn = lambda: fp8q.fp8q_gemm_mxf8_ue8m0(qa, sfa, qb, sfb, d)
+        work = ("flops", 2.0 * M * N * K)
+    elif name in ("quant_x_ue8m0", "quant_w_ue8m0"):
+        # power-of-two (UE8M0) scale study: the quantizers writing scale atoms
+        if name == "quant_x_ue8m0":
+            x = randn(T, HID)
+            q = torch.empty((T, HID), dtype=u8, device=dev)
+            sf = torch.empty((HID // 128, (T + 127) // 128, 128), dtype=torch.int32, device=dev)
+            fn = lambda: fp8q.fp8q_quant_act_1x128_ue8m0(x, q, sf)
+            work = ("bytes", T * HID * 3 + T * HID // 128 * 4)
+        else:
+            w = randn(OUT, HID, sigma=0.02)
+            q = torch.empty((OUT, HID), dtype=u8, device=dev)
+            sf = torch.empty((HID // 128, OUT // 128, 128), dtype=torch.int32, device=dev)
+            fn = lambda: fp8q.fp8q_quant_w_128x128_ue8m0(w, q, sf)
+            work = ("bytes", OUT * HID * 3 + OUT * HID // 128 * 4)
     elif name == "quant_x_pt":
         # per-tensor baseline quantizer: amax pass + cast pass (reads x twice)
         x = randn(T, HID)
@@ -843,8 +865,11 @@ def run_single(args):
         q, sf, qt, sft = fp8q.quant_w_128x128(w, transposed=True)
         fn = lambda: fp8q.fp8q_quant_w_128x128(w, q, sf, qt, sft)
         work = ("bytes", OUT * HID * 4 + 2 * (OUT // 128) * (HID // 128) * 4)
-    elif name in ("fprop", "dgrad", "wgrad"):
-        if name == "fprop":
+    elif name in ("fprop", "fprop_single", "dgrad", "wgrad"):
+        if name == "fprop_single":
+            # the one-CTA (128 x 256 tile) kernel at the Fprop shape, beside the one-CTA UE8M0 kernel
+            fp8q.fp8q_debug_force_dense_kernel(fp8q.FP8Q_DENSE_SINGLE)
+        if name in ("fprop", "fprop_single"):
             M, N, K = T, OUT, HID
         elif name == "dgrad":
             M, N, K = T, HID, OUT

@@ -58,6 +58,7 @@ EXPORTS = (
     "fp8q_gather_rows_fp8", "fp8q_quant_act_1x128_scatter", "fp8q_quant_act_1x128_scatter_rowscales",
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
     "fp8q_moe_dispatch_layout_noalloc",
+    "fp8q_quant_act_1x128_ue8m0", "fp8q_quant_w_128x128_ue8m0", "fp8q_gemm_mxf8_ue8m0",
 )
 
 _P = ctypes.c_void_p
@@ -97,6 +98,9 @@ _lib.fp8q_grouped_gemm_blockscaled_q1x128.argtypes = [_P, _I, _P, _I, _P, _P, _P
 _lib.fp8q_debug_cast_e4m3_bits.argtypes = [ctypes.c_uint32, _I, _P, _P]
 _lib.fp8q_debug_wait_timeout.argtypes = [_I, _P]
 _lib.fp8q_debug_force_dense_kernel.argtypes = [ctypes.c_int]
+_lib.fp8q_quant_act_1x128_ue8m0.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
+_lib.fp8q_quant_w_128x128_ue8m0.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
+_lib.fp8q_gemm_mxf8_ue8m0.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P]
 for _n in EXPORTS[2:]:
     getattr(_lib, _n).restype = ctypes.c_int
 
@@ -366,6 +370,28 @@ def fp8q_debug_cast_e4m3_bits(start: int, count: int, out, stream=None):
            "fp8q_debug_cast_e4m3_bits")
 
 
+def fp8q_quant_act_1x128_ue8m0(x, q, sf_mx, stream=None):
+    """Power-of-two scale study: x bf16 [M][K] -> q uint8 [M][K], sf_mx int32 [K/128][ceil(M/128)][128] atoms."""
+    M, K = x.shape
+    _check(_lib.fp8q_quant_act_1x128_ue8m0(_ptr(x), M, K, _ld(x), _ptr(q), _ld(q), _ptr(sf_mx), _stream(stream)),
+           "fp8q_quant_act_1x128_ue8m0")
+
+
+def fp8q_quant_w_128x128_ue8m0(w, q, sf_mx, stream=None):
+    """Power-of-two scale study: w bf16 [N][K] -> q uint8 [N][K], sf_mx int32 [K/128][N/128][128] atoms."""
+    N, K = w.shape
+    _check(_lib.fp8q_quant_w_128x128_ue8m0(_ptr(w), N, K, _ld(w), _ptr(q), _ld(q), _ptr(sf_mx), _stream(stream)),
+           "fp8q_quant_w_128x128_ue8m0")
+
+
+def fp8q_gemm_mxf8_ue8m0(a, sfa_mx, b, sfb_mx, d, stream=None):
+    """d bf16 [M][N] = a . b^T on the block-scaled MMA with UE8M0 scale atoms (study)."""
+    M, K = a.shape
+    N = b.shape[0]
+    _check(_lib.fp8q_gemm_mxf8_ue8m0(_ptr(a), _ld(a), _ptr(sfa_mx), _ptr(b), _ld(b), _ptr(sfb_mx), _ptr(d), _ld(d),
+                                     M, N, K, _stream(stream)), "fp8q_gemm_mxf8_ue8m0")
+
+
 def fp8q_debug_force_dense_kernel(choice: int):
     """FP8Q_DENSE_AUTO / FP8Q_DENSE_SINGLE / FP8Q_DENSE_PAIR for later dense GEMM calls."""
     _check(_lib.fp8q_debug_force_dense_kernel(int(choice)), "fp8q_debug_force_dense_kernel")
@@ -386,6 +412,22 @@ def quant_act_1x128(x, stream=None):
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     sf = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=x.device)
     fp8q_quant_act_1x128(x, q, sf, stream)
+    return q, sf
+
+
+def quant_act_1x128_ue8m0(x, stream=None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((K // 128, (M + 127) // 128, 128), dtype=torch.int32, device=x.device)
+    fp8q_quant_act_1x128_ue8m0(x, q, sf, stream)
+    return q, sf
+
+
+def quant_w_128x128_ue8m0(w, stream=None):
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    sf = torch.empty((K // 128, N // 128, 128), dtype=torch.int32, device=w.device)
+    fp8q_quant_w_128x128_ue8m0(w, q, sf, stream)
     return q, sf
 
 

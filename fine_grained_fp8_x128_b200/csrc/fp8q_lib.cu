@@ -17,6 +17,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_pertensor.cuh"
+#include "mx.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -50,6 +51,9 @@ struct DeviceInfo {
   int pt_cast_per_sm = 0;
   int q2_per_sm = 0;
   int qw_per_sm = 0;
+  bool mx_attr = false;            // UE8M0 block-scaled GEMM (study)
+  int qmx_per_sm = 0;
+  int qwmx_per_sm = 0;
 };
 
 // Resident blocks per SM of a kernel (cached per device); at least 1.
@@ -999,5 +1003,96 @@ extern "C" fp8q_status fp8q_moe_dispatch_layout_noalloc(const int32_t* expert_id
   if ((st = launch_status()) != FP8Q_OK) return st;
   fp8q::moe_layout_scatter_kernel<<<static_cast<unsigned>(chunks), 32, 0, s>>>(expert_ids, n_entries, k, num_experts,
                                                                                chunk, starts, rows, pos);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Power-of-two (UE8M0) scales on the hardware block-scaled MMA: the
+// throughput study beside the method (mx.cuh).
+// ---------------------------------------------------------------------------
+extern "C" fp8q_status fp8q_quant_act_1x128_ue8m0(const void* x, int64_t M, int64_t K, int64_t ldx, void* q,
+                                                  int64_t ldq, uint32_t* sf_mx, void* stream) {
+  if (M < 0 || K < 0 || K % 128 != 0 || ldx < K || ldq < K) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8Q_OK;
+  if (x == nullptr || q == nullptr || sf_mx == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (M > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf_mx, 16) || ldx % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t KB = K / 128;
+  const int64_t items = ((M + 127) / 128) * (128 / fp8q::kQ1Rows) * KB;
+  const int per_sm = blocks_per_sm(&dev->qmx_per_sm, fp8q::quant_act_1x128_ue8m0_kernel, fp8q::kQ1Threads, 0);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  fp8q::quant_act_1x128_ue8m0_kernel<<<static_cast<unsigned>(grid), fp8q::kQ1Threads, 0,
+                                       static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), M, KB, ldx, static_cast<uint8_t*>(q), ldq, sf_mx);
+  return launch_status();
+}
+
+extern "C" fp8q_status fp8q_quant_w_128x128_ue8m0(const void* w, int64_t N, int64_t K, int64_t ldw, void* q,
+                                                  int64_t ldq, uint32_t* sf_mx, void* stream) {
+  if (N < 0 || K < 0 || N % 128 != 0 || K % 128 != 0 || ldw < K || ldq < K) return FP8Q_ERR_INVALID_ARG;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (w == nullptr || q == nullptr || sf_mx == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(sf_mx, 16) || ldw % 8 != 0 || ldq % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t NB = N / 128, KB = K / 128;
+  const int per_sm = blocks_per_sm(&dev->qwmx_per_sm, fp8q::quant_w_128x128_ue8m0_kernel, fp8q::kQWThreads, 0);
+  const int64_t grid = grid_for(NB * KB, dev->sm_count, per_sm);
+  fp8q::quant_w_128x128_ue8m0_kernel<<<static_cast<unsigned>(grid), fp8q::kQWThreads, 0,
+                                       static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w), NB, KB, ldw, static_cast<uint8_t*>(q), ldq, sf_mx);
+  return launch_status();
+}
+
+extern "C" fp8q_status fp8q_gemm_mxf8_ue8m0(const void* a, int64_t lda, const uint32_t* sfa_mx, const void* b,
+                                            int64_t ldb, const uint32_t* sfb_mx, void* d, int64_t ldd, int64_t M,
+                                            int64_t N, int64_t K, void* stream) {
+  const int64_t kIntMax = 0x7FFFFFFF;
+  if (M < 1 || N < 256 || K < 128 || K % 128 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (N % 256 != 0) return FP8Q_ERR_UNSUPPORTED;   // whole 256-column tiles only (the study's shapes)
+  if (M > kIntMax || N > kIntMax || K > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  if (lda < K || ldb < K || ldd < N) return FP8Q_ERR_INVALID_ARG;
+  if (a == nullptr || b == nullptr || sfa_mx == nullptr || sfb_mx == nullptr || d == nullptr)
+    return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa_mx, 16) || !aligned(sfb_mx, 16) ||
+      lda % 16 != 0 || ldb % 16 != 0 || (ldd * 2) % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
+  if ((st = make_tmap(&tb, b, K, N, ldb, fp8q::BN)) != FP8Q_OK) return st;
+  fp8q::MxArgs args{};
+  args.sfa = sfa_mx;
+  args.sfb = sfb_mx;
+  args.d = d;
+  args.ldd = ldd;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_m_tiles = static_cast<int>((M + fp8q::BM - 1) / fp8q::BM);
+  args.num_n_tiles = static_cast<int>(N / fp8q::BN);
+  args.num_k_chunks = static_cast<int>(K / fp8q::BK);
+  const int64_t tiles = static_cast<int64_t>(args.num_m_tiles) * args.num_n_tiles;
+  if (tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
+  const uint32_t smem = fp8q::MxSmemLayout::bytes + 1024;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!dev->mx_attr) {
+      if (cudaFuncSetAttribute(fp8q::gemm_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      dev->mx_attr = true;
+    }
+  }
+  const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
+  fp8q::gemm_mx_kernel<<<grid, fp8q::kGemmThreads, smem, static_cast<cudaStream_t>(stream)>>>(ta, tb, args);
   return launch_status();
 }

@@ -495,6 +495,58 @@ fp8q_status fp8q_gemm_pertensor(const void* a, int64_t lda, const float* scale_a
                                 const float* scale_b, void* d, int64_t ldd, int d_dtype,
                                 int64_t M, int64_t N, int64_t K, void* stream);
 
+/* ---- power-of-two (UE8M0) scales on the block-scaled MMA: a study ------------
+ * Not the pages' method.  The pages fix s = amax/448 ("FP8 Mixed Precision:
+ * DeepSeek-V3 Training Architecture", section 1, eq. s_W), a full FP32 scale,
+ * which is why fp8q_gemm_blockscaled promotes every 128-wide K chunk on the
+ * CUDA cores.  The tensor core's block-scaled MMA (tcgen05.mma
+ * kind::mxf8f6f4) applies scales itself but only powers of two (UE8M0: byte b
+ * stands for 2^(b - 127)), one per 32 elements of K.  These calls keep the
+ * method's tiles and round each scale UP to a power of two,
+ *   s2 = 2^ceil(log2 t),  t = max(fl32(amax / 448), fl32(1e-12)),
+ *   q  = e4m3(fl32(x / s2))   (no element saturates),
+ * so that the GEMM can accumulate all of K in the tensor core: they measure
+ * what the method's non-power-of-two scales cost.
+ *
+ * Scale layout ("scale atoms", the tensor core's scale-factor layout): one
+ * 512-byte atom of 128 uint32 words per (128-row block rb, K chunk kb); row
+ * r = 128 rb + r0 + 32 r1 (r0 < 32, r1 < 4) has word 4 r0 + r1, whose four
+ * bytes are the UE8M0 scales of its four 32-wide K-blocks (all equal here):
+ *   sf_mx[(kb * row_blocks + r / 128) * 128 + 4 * (r % 32) + (r % 128) / 32].
+ * Arrays are 16-byte aligned, row_blocks = ceil(rows / 128).
+ */
+
+/*
+ * 1x128 tiles with power-of-two scales.  x: BF16 [M][ldx]; q: E4M3 [M][ldq];
+ * sf_mx: uint32 [K/128][ceil(M/128)][128] scale atoms (rows M .. up to the
+ * next multiple of 128 get the word of 1.0).  Requirements as
+ * fp8q_quant_act_1x128, plus sf_mx 16-byte aligned.
+ */
+fp8q_status fp8q_quant_act_1x128_ue8m0(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,
+                                       uint32_t* sf_mx, void* stream);
+
+/*
+ * 128x128 weight blocks with power-of-two scales.  w: BF16 [N][ldw];
+ * q: E4M3 [N][ldq]; sf_mx: uint32 [K/128][N/128][128] scale atoms (every row
+ * of a block carries the block's scale).  N % 128 == 0, K % 128 == 0.
+ */
+fp8q_status fp8q_quant_w_128x128_ue8m0(const void* w, int64_t N, int64_t K, int64_t ldw, void* q, int64_t ldq,
+                                       uint32_t* sf_mx, void* stream);
+
+/*
+ * D = A . B^T on the block-scaled MMA with the scale atoms above, FP32
+ * accumulation of all of K in tensor memory, BF16 out (RNE):
+ *   D[m,n] = sum_k (qa[m,k] * sa2[m, k/128]) * (qb[n,k] * sb2[n, k/128]).
+ *   a: E4M3 [M][lda] K-major, sfa_mx [K/128][ceil(M/128)][128];
+ *   b: E4M3 [N][ldb] K-major, sfb_mx [K/128][N/128][128];  d: BF16 [M][ldd].
+ * Requirements: M >= 1, K % 128 == 0, N % 256 == 0 (else FP8Q_ERR_UNSUPPORTED),
+ * lda >= K, ldb >= K, ldd >= N; a, b, d, sfa_mx, sfb_mx 16-byte aligned,
+ * lda % 16 == 0, ldb % 16 == 0, ldd % 8 == 0.
+ */
+fp8q_status fp8q_gemm_mxf8_ue8m0(const void* a, int64_t lda, const uint32_t* sfa_mx, const void* b, int64_t ldb,
+                                 const uint32_t* sfb_mx, void* d, int64_t ldd, int64_t M, int64_t N, int64_t K,
+                                 void* stream);
+
 /* ---- diagnostics (used by the test suite; not on the hot path) ---------- */
 
 /*
