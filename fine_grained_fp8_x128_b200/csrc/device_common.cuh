@@ -485,3 +485,20 @@ __device__ __forceinline__ void tmem_ld_32x32b_x64_sync(uint32_t taddr, uint32_t
       : "memory");
 }
 }  // namespace fp8q
+
+// ---------------------------------------------------------------------------
+// TMA stores (shared -> global, bulk async-group completion).  The issuing
+// thread commits the group and waits on it: .read returns once the shared
+// memory source may be reused; the global writes complete on their own.
+// ---------------------------------------------------------------------------
+namespace fp8q {
+__device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+}  // namespace fp8q

@@ -150,9 +150,49 @@ fp8q_status make_tmap_f32(CUtensorMap* map, const float* base, int64_t inner, in
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
+// Output matrix [rows][ld] of BF16 (esz 2) or FP32 (esz 4) for the pair
+// kernel's tile-end tensor stores: box {128 bytes, 32 rows}, 128-byte swizzle
+// (the layout of the epilogue's staging buffer).
+fp8q_status make_tmap_out(CUtensorMap* map, void* base, int64_t cols, int64_t rows, int64_t ld, int esz) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  fp8q_status st = encoder(&enc);
+  if (st != FP8Q_OK) return st;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esz)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
+// The same for the one-CTA kernel: box {64 bytes, 32 rows} with the 64-byte
+// swizzle of its 2 KB staging buffers; esz 1 (E4M3 codes), 2 (BF16) or 4 (FP32).
+fp8q_status make_tmap_out64(CUtensorMap* map, void* base, int64_t cols, int64_t rows, int64_t ld, int esz) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  fp8q_status st = encoder(&enc);
+  if (st != FP8Q_OK) return st;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esz)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / esz), 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapDataType dt = esz == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+
 template <bool G, int MODE, int OUT>
 fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const fp8q::GemmArgs& args,
                         int grid, cudaStream_t stream) {
+  // the output's tensor map for the tile-end stores of full 32-row boxes
+  CUtensorMap td;
+  const int esz = OUT == fp8q::kOutF32 ? 4 : (OUT == fp8q::kOutE4m3 ? 1 : 2);
+  fp8q_status st = make_tmap_out64(&td, args.d, args.N, args.M, args.ldd, esz);
+  if (st != FP8Q_OK) return st;
   const uint32_t smem = (G ? fp8q::GemmSmemLayout::bytes_grouped : fp8q::GemmSmemLayout::bytes_dense) + 1024;
   auto kern = fp8q::gemm_blockscaled_kernel<G, MODE, OUT>;
   bool& attr = dev->gemm_attr[G ? 1 : 0][MODE == FP8Q_SFB_ROW ? 1 : 0][OUT];
@@ -162,14 +202,14 @@ fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMa
       return FP8Q_ERR_CUDA;
     attr = true;
   }
-  kern<<<grid, fp8q::kGemmThreads, smem, stream>>>(ta, tb, args);
+  kern<<<grid, fp8q::kGemmThreads, smem, stream>>>(ta, tb, td, args);
   return launch_status();
 }
 
 template <int MODE, int OUT>
 fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
-                             const CUtensorMap& tsb, const fp8q::GemmArgs& args, int64_t pair_tiles,
-                             cudaStream_t stream) {
+                             const CUtensorMap& tsb, const CUtensorMap& td, const fp8q::GemmArgs& args,
+                             int64_t pair_tiles, cudaStream_t stream) {
   const uint32_t smem = fp8q::PairSmemLayout::bytes + 1024;
   auto kern = fp8q::gemm_pair_kernel<MODE, OUT>;
   const int mi = MODE == FP8Q_SFB_ROW ? 1 : 0, fi = OUT;
@@ -199,7 +239,7 @@ fp8q_status launch_gemm_pair(DeviceInfo* dev, const CUtensorMap& ta, const CUten
   }
   const int64_t clusters = pair_tiles < dev->pair_clusters[mi][fi] ? pair_tiles : dev->pair_clusters[mi][fi];
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, td, args) != cudaSuccess) return FP8Q_ERR_CUDA;
   return launch_status();
 }
 
@@ -283,17 +323,17 @@ bool use_pair_kernel(int64_t M, const float* sfa, int64_t ld_sfa, const float* s
 // the output mode (the FP8 output exists for 128x128-block B scales only).
 template <int MODE>
 fp8q_status dense_launch(DeviceInfo* dev, bool pair, int out, const CUtensorMap& ta, const CUtensorMap& tb,
-                         const CUtensorMap& tsa, const CUtensorMap& tsb, const fp8q::GemmArgs& args,
-                         int64_t pair_tiles, int grid, cudaStream_t s) {
+                         const CUtensorMap& tsa, const CUtensorMap& tsb, const CUtensorMap& td,
+                         const fp8q::GemmArgs& args, int64_t pair_tiles, int grid, cudaStream_t s) {
   if (out == fp8q::kOutF32)
-    return pair ? launch_gemm_pair<MODE, fp8q::kOutF32>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+    return pair ? launch_gemm_pair<MODE, fp8q::kOutF32>(dev, ta, tb, tsa, tsb, td, args, pair_tiles, s)
                 : launch_gemm<false, MODE, fp8q::kOutF32>(dev, ta, tb, args, grid, s);
   if constexpr (MODE == FP8Q_SFB_BLOCK128) {
     if (out == fp8q::kOutE4m3)
-      return pair ? launch_gemm_pair<MODE, fp8q::kOutE4m3>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+      return pair ? launch_gemm_pair<MODE, fp8q::kOutE4m3>(dev, ta, tb, tsa, tsb, td, args, pair_tiles, s)
                   : launch_gemm<false, MODE, fp8q::kOutE4m3>(dev, ta, tb, args, grid, s);
   }
-  return pair ? launch_gemm_pair<MODE, fp8q::kOutBf16>(dev, ta, tb, tsa, tsb, args, pair_tiles, s)
+  return pair ? launch_gemm_pair<MODE, fp8q::kOutBf16>(dev, ta, tb, tsa, tsb, td, args, pair_tiles, s)
               : launch_gemm<false, MODE, fp8q::kOutBf16>(dev, ta, tb, args, grid, s);
 }
 
@@ -324,7 +364,7 @@ fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_
   fp8q_status st = device_info(&dev);
   if (st != FP8Q_OK) return st;
   const bool pair = use_pair_kernel(M, sfa, ld_sfa, sfb, ld_sfb);
-  CUtensorMap ta, tb, tsa, tsb;
+  CUtensorMap ta, tb, tsa, tsb, td;
   if ((st = make_tmap(&ta, a, K, M, lda, fp8q::BM)) != FP8Q_OK) return st;
   if ((st = make_tmap(&tb, b, K, N, ldb, pair ? fp8q::BN / 2 : fp8q::BN)) != FP8Q_OK) return st;
   if (pair) {
@@ -335,9 +375,13 @@ fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_
     st = sfb_mode == FP8Q_SFB_ROW ? make_tmap_f32(&tsb, sfb, N, K / 128, ld_sfb, fp8q::BN, 1)
                                   : make_tmap_f32(&tsb, sfb, K / 128, N / 128, ld_sfb, 4, 2);
     if (st != FP8Q_OK) return st;
+    // the tile-end tensor stores (BF16 and FP32 outputs of the 128x128-block mode)
+    if (out == fp8q::kOutE4m3 || sfb_mode == FP8Q_SFB_ROW) td = tb;
+    else if ((st = make_tmap_out(&td, d, N, M, ldd, static_cast<int>(esz))) != FP8Q_OK) return st;
   } else {
     tsa = tb;   // not read by the one-CTA kernel
     tsb = tb;
+    td = tb;
   }
   fp8q::GemmArgs args{};
   args.sfa = sfa;
@@ -365,8 +409,8 @@ fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_
   args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return sfb_mode == FP8Q_SFB_BLOCK128
-             ? dense_launch<FP8Q_SFB_BLOCK128>(dev, pair, out, ta, tb, tsa, tsb, args, pair_tiles, grid, s)
-             : dense_launch<FP8Q_SFB_ROW>(dev, pair, out, ta, tb, tsa, tsb, args, pair_tiles, grid, s);
+             ? dense_launch<FP8Q_SFB_BLOCK128>(dev, pair, out, ta, tb, tsa, tsb, td, args, pair_tiles, grid, s)
+             : dense_launch<FP8Q_SFB_ROW>(dev, pair, out, ta, tb, tsa, tsb, td, args, pair_tiles, grid, s);
 }
 
 // Body of both grouped GEMM entry points (out: kOutBf16 or kOutE4m3).

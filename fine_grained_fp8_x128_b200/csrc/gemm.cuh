@@ -65,12 +65,12 @@ struct GemmSmemLayout {
   // offsets from the 1024-aligned base
   static constexpr uint32_t stages = 0;
   static constexpr uint32_t sb_ring = stages + kStages * kStageBytes;
-  static constexpr uint32_t bars = sb_ring + kSbRing * kSbBytes;
+  static constexpr uint32_t out_stage = sb_ring + kSbRing * kSbBytes;   // 8 epilogue warps x 2 KB, 1024-aligned
+  static constexpr uint32_t bars = out_stage + 8 * 2048;
   // barriers: go[S], done[S], sbfull[R], sbempty[R]
   static constexpr uint32_t nbars = 2 * kStages + 2 * kSbRing;
   static constexpr uint32_t misc = bars + nbars * 8;           // tmem base, abort flag
-  static constexpr uint32_t out_stage = misc + 16;             // 8 epilogue warps x 2 KB (staged stores)
-  static constexpr uint32_t prefix = out_stage + 8 * 2048;     // grouped: tile prefix [G+1]
+  static constexpr uint32_t prefix = misc + 16;                // grouped: tile prefix [G+1]
   static constexpr uint32_t offs = prefix + (kMaxGroups + 1) * 4;  // grouped: clamped offsets [G+1]
   static constexpr uint32_t bytes_dense = prefix;
   static constexpr uint32_t bytes_grouped = offs + (kMaxGroups + 1) * 4;
@@ -189,6 +189,86 @@ __device__ __forceinline__ void stage_store_pass4(uint4* stage, const uint4 (&ch
     if (r < rows_valid) *reinterpret_cast<uint4*>(gbase + r * ld_bytes + 16 * c) = val;
   }
   __syncwarp();
+}
+
+// One pass of a tile-end tensor store: the warp's shared buffer (written in
+// the tensor map's swizzled layout) is stored as one box at (x, y) by lane 0,
+// which waits only until the buffer has been read; the global writes finish
+// in the background.
+__device__ __forceinline__ void tma_store_pass(uint8_t* buf, const CUtensorMap* tmap_d, int x, int y, int lane) {
+  fence_proxy_async_shared();   // the buffer's generic-proxy writes, before the async-proxy read
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmap_d, buf, x, y);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncwarp();
+}
+
+// store_rows128_staged4 for a warp whose 32 rows are all valid, through
+// tensor stores: each pass's 32 rows x 64 bytes go into the 2 KB buffer in
+// the 64-byte-swizzled layout of stage_store_pass4 (chunk j of row r at
+// j ^ ((r / 2) % 4), the tensor map's SWIZZLE_64B pattern) and leave as one
+// box.  kOutE4m3 also writes the row's tile scale, as the staged version does.
+template <int kOut>
+__device__ __forceinline__ void store_rows128_tma64(const float2* acc, int lane, int row0, int ncol0,
+                                                    const GemmArgs& p, const CUtensorMap* tmap_d, uint8_t* buf) {
+  uint4* stage = reinterpret_cast<uint4*>(buf);
+  auto put = [&](const uint4(&chunk)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) stage[lane * 4 + (j ^ ((lane >> 1) & 3))] = chunk[j];
+  };
+  uint4 chunk[4];
+  if (kOut == kOutF32) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 a = acc[8 * h + 2 * j], b = acc[8 * h + 2 * j + 1];
+        chunk[j] = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
+      }
+      put(chunk);
+      tma_store_pass(buf, tmap_d, ncol0 + 16 * h, row0, lane);
+    }
+  } else {
+    uint32_t w[64];   // BF16 pairs
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+      const __nv_bfloat162 h = __float22bfloat162_rn(acc[j]);
+      w[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    if (kOut == kOutBf16) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          chunk[j] = make_uint4(w[16 * h + 4 * j], w[16 * h + 4 * j + 1], w[16 * h + 4 * j + 2], w[16 * h + 4 * j + 3]);
+        put(chunk);
+        tma_store_pass(buf, tmap_d, ncol0 + 32 * h, row0, lane);
+      }
+    } else {
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
+      const float s = tile_scale(amax2_value(m2));
+      const float nr = -__frcp_rn(s);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t c[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            c[j] = quant_words(w[32 * h + 8 * i + 2 * j], w[32 * h + 8 * i + 2 * j + 1], nr, s);
+          chunk[i] = make_uint4(c[0], c[1], c[2], c[3]);
+        }
+        put(chunk);
+        tma_store_pass(buf, tmap_d, ncol0 + 64 * h, row0, lane);
+      }
+      p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
+    }
+  }
 }
 
 // store_rows128_staged through a 2 KB buffer: 8 passes of 16 FP32 columns, 4
@@ -388,7 +468,7 @@ __device__ __forceinline__ void build_group_prefix(const GemmArgs& p, int* offs,
 template <bool kGrouped, int kSfbMode, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                        const GemmArgs p) {
+                        const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
   extern __shared__ uint8_t gemm_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmemLayout::bars);
@@ -561,11 +641,17 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
       if (vcol) {   // warp-uniform
         const int row0 = c.a_row0 + quad * 32;
         const int rows_valid = min(32, c.row_end - row0);
-        if (rows_valid > 0)
-          store_rows128_staged4<kOut>(acc, lane, row0, rows_valid, ncol0, p,
-                                      reinterpret_cast<uint4*>(smem + GemmSmemLayout::out_stage + warp * 2048));
+        uint8_t* out_buf = smem + GemmSmemLayout::out_stage + warp * 2048;
+        // a box of 32 full rows leaves as tensor stores; a part-filled box (the
+        // last rows of an expert or of M) keeps the per-row staged stores, so
+        // nothing is written past the expert's rows
+        if (rows_valid == 32)
+          store_rows128_tma64<kOut>(acc, lane, row0, ncol0, p, &tmap_d, out_buf);
+        else if (rows_valid > 0)
+          store_rows128_staged4<kOut>(acc, lane, row0, rows_valid, ncol0, p, reinterpret_cast<uint4*>(out_buf));
       }
     }
+    if (lane == 0) bulk_wait_group0();   // this warp's tensor stores are complete before the CTA exits
   }
 
   tc_fence_before();

@@ -30,9 +30,12 @@
 // c + kPairScaleSlots - S - 2 >= c + 1, issued after the warp's last read of
 // slot c; a proxy fence before each release orders those reads before the
 // refill.
-// At the end of a tile each epilogue warp writes its 32 rows through a 4 KB
-// shared buffer (stage_store_pass) so that the global stores cover whole
-// 128-byte row segments.
+// At the end of a tile each epilogue warp writes its 32 rows x 128 columns
+// through a 4 KB shared buffer with TMA tensor stores (store_rows128_tma), so
+// the global writes complete in the background while the warp returns to the
+// next tile's chunks.  The FP8 output keeps the staged 16-byte stores of
+// stage_store_pass (with its scales), and the FP8Q_SFB_ROW mode's 16x256b
+// fragments are stored directly.
 #pragma once
 
 #include "gemm.cuh"
@@ -102,11 +105,56 @@ __device__ __forceinline__ void promote_rows16(float2* acc, const uint32_t (&v)[
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tile-end stores through TMA.  A warp's 32 rows x 128 columns leave in passes
+// of 32 rows x 128 bytes: the warp writes the pass into its 4 KB shared buffer
+// in the TMA's 128-byte-swizzled layout (16-byte chunk j of row r at chunk
+// j ^ (r % 8)), one lane issues a tensor store of the box and waits only
+// until the buffer has been read; the global writes complete in the
+// background while the warp goes on (to the next pass, then to the next
+// tile's chunks).  Rows past M are clipped by the tensor map.  (tma_store_pass
+// is in gemm.cuh.)
+// ---------------------------------------------------------------------------
+// 32x32b fragments (thread = row `lane`, acc[j] = columns 2j, 2j+1 of the
+// warp's 128): BF16 in 2 passes of 64 columns, FP32 in 4 passes of 32.
+template <int kOut>
+__device__ __forceinline__ void store_rows128_tma(const float2* acc, int lane, int row0, int ncol0,
+                                                  const CUtensorMap* tmap_d, uint8_t* buf) {
+  uint4* stage = reinterpret_cast<uint4*>(buf);
+  if (kOut == kOutF32) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 a = acc[16 * h + 2 * j], b = acc[16 * h + 2 * j + 1];
+        stage[lane * 8 + (j ^ (lane & 7))] =
+            make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
+      }
+      tma_store_pass(buf, tmap_d, ncol0 + 32 * h, row0, lane);
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 v = __float22bfloat162_rn(acc[32 * h + 4 * j + e]);
+          w[e] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+        stage[lane * 8 + (j ^ (lane & 7))] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      tma_store_pass(buf, tmap_d, ncol0 + 64 * h, row0, lane);
+    }
+  }
+}
+
 template <int kSfbMode, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
-                 const GemmArgs p) {
+                 const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
   extern __shared__ uint8_t pair_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pair_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PairSmemLayout::bars);
@@ -284,10 +332,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         }
       }
       if (!ok) break;
+      const int row0 = a_row0 + quad * 32;
+      uint8_t* out_buf = smem + PairSmemLayout::out_stage + warp * kPairOutStageBytes;
       if (kSfbMode == FP8Q_SFB_ROW) {
         // 16x256b fragments: acc[64h + 32g + 4k + 2i + j] is row 32*quad + 16g +
         // 8i + lane/4, column 64h + 8k + 2*(lane%4) + j of this half; 4 lanes
-        // write one 32-byte sector of a row per group k
+        // write one 32-byte sector of a row per group k.  (Tensor stores of
+        // these fragments measured slower on B200: their staging raised the
+        // register pressure of the chunk loop.)
         if (vcol) {
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
@@ -310,12 +362,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             }
           }
         }
-      } else if (vcol) {
-        const int row0 = a_row0 + quad * 32;
-        store_rows128_staged<kOut>(acc, lane, row0, min(32, p.M - row0), ncol0, p,
-                                   reinterpret_cast<uint4*>(smem + PairSmemLayout::out_stage + warp * kPairOutStageBytes));
+      } else if (vcol && row0 < p.M) {
+        if (kOut == kOutE4m3)
+          store_rows128_staged<kOut>(acc, lane, row0, min(32, p.M - row0), ncol0, p,
+                                     reinterpret_cast<uint4*>(out_buf));
+        else
+          store_rows128_tma<kOut>(acc, lane, row0, ncol0, &tmap_d, out_buf);
       }
     }
+    if (lane == 0) bulk_wait_group0();   // this warp's tensor stores are complete before the CTA exits
   }
 
   tc_fence_before();
