@@ -7,17 +7,22 @@ contiguous ranges over the ranks of the process group.  One call:
 
   1. layout (device): a stable counting sort of the (token, slot) entries by
      expert, giving the send order -- expert-major, hence rank-major;
-  2. the expert offsets come to the host (one synchronisation: the collective
-     needs the split sizes; without a process group nothing is exchanged: each
-     token is quantized once and scattered to its rows of the grouped GEMM's
-     input, and the host never waits);
-  3. quantize (device): each token's 1x128 FP8 codes and row-major scales,
-     computed once and written straight to its rows of the send buffer;
-  4. all_to_all_single of the per-(rank, local expert) row counts, then of the
-     codes and of the scales (NCCL over NVLink on GPUs);
+  2. quantize (device): each token's 1x128 FP8 codes and row-major scales,
+     computed once and written straight to its rows of the send buffer --
+     queued at once, since it needs only the layout's positions;
+  3. all_gather of every rank's expert offsets, read on the host once (the
+     one synchronisation of a call: the collective needs the split sizes);
+     that one table gives both what this rank sends to each rank and what it
+     receives per (source rank, local expert).  Without a process group
+     nothing is exchanged: each token is quantized once and scattered to its
+     rows of the grouped GEMM's input, and the host never waits;
+  4. all_to_all_single of the codes and of the scales (NCCL over NVLink on
+     GPUs);
   5. regroup (device): the received rows from (source, expert) order into
      (expert, source) order, the scales into the grouped GEMM's K-chunk-major
-     layout, so that the grouped GEMM runs on the result directly.
+     layout, so that the grouped GEMM runs on the result directly.  The order
+     is index arithmetic on the count table, uploaded from pinned memory
+     without another synchronisation.
 
 The device steps are this package's kernels (`CudaDispatchOps`).  The
 collectives are torch.distributed's.  The host part -- split sizes and the
@@ -106,6 +111,30 @@ class DispatchResult:
     recv_counts: np.ndarray  # int64 [world][E_local]: rows received per source rank and local expert (idem)
 
 
+_PINNED = {}
+
+
+def _upload(a: np.ndarray, device):
+    """int32 host array -> device, through a cached pinned buffer (no host
+    synchronisation; the buffer is reused once its previous copy is done)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a, np.int32))
+    if torch.device(device).type != "cuda":
+        return t.clone()
+    buf, ev = _PINNED.get(str(device), (None, None))
+    if buf is None or buf.numel() < t.numel():
+        buf = torch.empty(max(t.numel(), 1 << 16), dtype=torch.int32, pin_memory=True)
+        ev = None
+    if ev is not None:
+        ev.synchronize()                    # the last copy out of this buffer has finished
+    buf[:t.numel()].copy_(t)
+    out = buf[:t.numel()].to(device, non_blocking=True)
+    ev = torch.cuda.Event()
+    ev.record()
+    _PINNED[str(device)] = (buf, ev)
+    return out
+
+
 def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchResult:
     """x: bf16 [T][H] (H % 128 == 0) on this rank's device; expert_ids: int32
     [T][k] on the same device.  Collective over `group`: every rank calls it."""
@@ -126,14 +155,14 @@ def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchR
         # GEMM input, and nothing waits on the host
         q, sf = ops.quant_grouped(x, pos, expert_ids.numel())
         return DispatchResult(q=q, sf=sf, expert_offsets=offsets, pos=pos, send_counts=None, recv_counts=None)
-    off = offsets.cpu().numpy().astype(np.int64)                         # one host sync: the split sizes
-    per_expert = np.diff(off)
-    send_counts = per_expert.reshape(world, el).sum(axis=1)
-    q_send, sf_send = ops.quant_send(x, pos, expert_ids.numel())
-    counts_send = torch.from_numpy(per_expert.reshape(world, el).astype(np.int64)).to(x.device)
-    counts_recv = torch.empty_like(counts_send)
-    dist.all_to_all_single(counts_recv, counts_send, group=group)
-    recv_counts = counts_recv.cpu().numpy()
+    rank = dist.get_rank(group)
+    q_send, sf_send = ops.quant_send(x, pos, expert_ids.numel())       # queued before the host waits
+    gathered = [torch.empty_like(offsets) for _ in range(world)]
+    dist.all_gather(gathered, offsets, group=group)
+    off_all = torch.stack(gathered).cpu().numpy().astype(np.int64)     # the one host sync: every rank's offsets
+    per_expert = np.diff(off_all, axis=1)                               # [source rank][expert]
+    send_counts = per_expert[rank].reshape(world, el).sum(axis=1)
+    recv_counts = np.ascontiguousarray(per_expert[:, rank * el:(rank + 1) * el])
     recv_rows = recv_counts.sum(axis=1)
     M = int(recv_rows.sum())
     q_recv = torch.empty((M, H), dtype=torch.uint8, device=x.device)
@@ -141,6 +170,7 @@ def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchR
     dist.all_to_all_single(q_recv, q_send, recv_rows.tolist(), send_counts.tolist(), group=group)
     dist.all_to_all_single(sf_recv, sf_send, recv_rows.tolist(), send_counts.tolist(), group=group)
     order, exp_off = regroup_order(recv_counts)
-    q, sf = ops.regroup(q_recv, sf_recv, torch.from_numpy(order).to(x.device))
-    return DispatchResult(q=q, sf=sf, expert_offsets=torch.from_numpy(exp_off).to(x.device), pos=pos,
+    both = _upload(np.concatenate([order, exp_off]), x.device)
+    q, sf = ops.regroup(q_recv, sf_recv, both[:order.size])
+    return DispatchResult(q=q, sf=sf, expert_offsets=both[order.size:], pos=pos,
                           send_counts=send_counts, recv_counts=recv_counts)
