@@ -138,7 +138,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -151,23 +151,31 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        sm, smax, reasons = [], 0.0, set()
+        sm, pw, smax, reasons = [], [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = max(smax, float(parts[2]))
+                clk, mx, w = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
+            sm.append(clk)
+            pw.append(w)
+            smax = max(smax, mx)
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+        # the median over the samples taken under load (power draw at least half the
+        # run's peak): the samples before and after the timed kernels are idle
+        sm, pw = np.array(sm), np.array(pw)
+        load = pw >= 0.5 * pw.max()
+        return {"sm_mhz": float(np.median(sm[load])), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": int(sm.size), "samples_under_load": int(load.sum()),
+                "sm_mhz_min_under_load": float(sm[load].min()), "power_w_max": float(pw.max())}
 
 
 # ----------------------------------------------------------------------------- distributed helpers
@@ -921,6 +929,10 @@ def run_single(args):
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
+    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+    clocks.path = os.path.join(LOG_DIR, f"clocks_single_{name}.csv")
+    clocks.start()
+    time.sleep(0.2)
     times = []
     for _ in range(args.steps):
         scrub.zero_()                       # evict the inputs from L2 between launches
@@ -929,10 +941,11 @@ def run_single(args):
         s.record(); fn(); e.record()
         torch.cuda.synchronize()
         times.append(s.elapsed_time(e) * 1e-3)
+    clk = clocks.stop()
     code = fp8q.fp8q_device_status()
     t = float(np.median(times))
     out = {"kernel": name, "tokens": T, "median_us": round(t * 1e6, 2), "min_us": round(min(times) * 1e6, 2),
-           "status": code}
+           "status": code, "clocks": clk}
     if work[0] == "bytes":
         out["GBps"] = round(work[1] / t / 1e9, 1)
     else:
