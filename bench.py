@@ -461,24 +461,41 @@ def kernel_stats(events, K):
     return {n: (tot[n] / cnt[n], tot[n]) for n in tot}
 
 
-def fp8_peak_for_clock(pk, clk):
+def fp8_peak_for_clock(pk, clk, kernel_mhz=None):
     """The measured FP8 denominator that matches the run's clock record: the
-    burst figure (2 x the burst BF16 GEMM) when the median SM clock under load
-    stayed at its maximum, the sustained one (2 x the seconds-long BF16 loop at
-    the power cap) otherwise.  Returns (TFLOP/s, description)."""
-    at_max = clk is not None and clk.get("sm_max_mhz") and clk["sm_mhz"] >= 0.97 * clk["sm_max_mhz"]
-    if at_max:
+    burst figure (2 x the burst BF16 GEMM) when the SM clock stayed at its
+    maximum, the sustained one (2 x the seconds-long BF16 loop at the power
+    cap) otherwise.  The clock taken is the one measured inside the GEMM
+    kernels (kernel_mhz, cycles over global-timer nanoseconds) when there is
+    one -- under FP8 load the clock drops to the power limit between
+    nvidia-smi's samples -- else the sampled median.  Returns (TFLOP/s,
+    description)."""
+    smax = (clk or {}).get("sm_max_mhz") or 0.0
+    if kernel_mhz is not None:
+        mhz, what = kernel_mhz, "SM clock inside the GEMM kernels"
+    elif clk is not None:
+        mhz, what = clk["sm_mhz"], "median sampled SM clock"
+    else:
+        mhz, what = None, None
+    if mhz is not None and smax and mhz >= 0.97 * smax:
         return pk["bf16"] * FP8_OVER_BF16, (f"{pk['src']} MEASURED_PEAKS.json burst BF16 TFLOP/s x 2 (nominal "
-                                            f"FP8:BF16 ratio); median SM clock {clk['sm_mhz']:.0f} MHz = max")
-    why = "no clock record" if clk is None else f"median SM clock {clk['sm_mhz']:.0f} MHz below max"
+                                            f"FP8:BF16 ratio); {what} {mhz:.0f} MHz = max")
+    why = "no clock record" if mhz is None else f"{what} {mhz:.0f} MHz below the {smax:.0f} MHz max"
     return pk["bf16_sus"] * FP8_OVER_BF16, (f"{pk['src']} MEASURED_PEAKS.json sustained BF16 TFLOP/s x 2 "
                                             f"(nominal FP8:BF16 ratio); {why}")
 
 
-def build_breakdown(stats, pk, moe_w_bytes, moe_other_bytes, clk=None):
+def gemm_kernel_mhz(name, kclk):
+    """The in-kernel SM clock of the kernel kind that runs a step GEMM."""
+    if not kclk:
+        return None
+    kind = "one_cta" if name.startswith("moe") else "pair"
+    return kclk.get(kind, {}).get("mhz")
+
+
+def build_breakdown(stats, pk, moe_w_bytes, moe_other_bytes, clk=None, kclk=None):
     fl = gemm_flops()
     qb = quant_bytes()
-    fp8_peak, _ = fp8_peak_for_clock(pk, clk)
     out = {}
     for name, (avg, total) in stats.items():
         ent = {"avg_us": round(avg * 1e6, 2), "share": None}
@@ -489,8 +506,12 @@ def build_breakdown(stats, pk, moe_w_bytes, moe_other_bytes, clk=None):
                        bar_70pct_hbm_spec=bool(gbs / SPEC_HBM_GBS >= BAR_QUANT_HBM))
         if name in fl:
             tf = fl[name] / avg / 1e12
+            fp8_peak, _ = fp8_peak_for_clock(pk, clk, gemm_kernel_mhz(name, kclk))
             ent.update(flops=fl[name], tflops=round(tf, 1), frac_fp8=round(tf / fp8_peak, 3),
+                       frac_fp8_burst=round(tf / (pk["bf16"] * FP8_OVER_BF16), 3),
                        frac_fp8_spec=round(tf / SPEC_FP8_TFLOPS, 3))
+            if gemm_kernel_mhz(name, kclk) is not None:
+                ent.update(kernel_sm_mhz=gemm_kernel_mhz(name, kclk))
             if name.startswith("moe"):
                 b = moe_w_bytes + moe_other_bytes[name]
                 ent.update(bytes=b, gbps=round(b / avg / 1e9, 1), frac_hbm=round(b / avg / 1e9 / pk["hbm"], 3),
@@ -504,7 +525,7 @@ def build_breakdown(stats, pk, moe_w_bytes, moe_other_bytes, clk=None):
     return out
 
 
-def roofline_for(name, stats, pk, breakdown, clk=None):
+def roofline_for(name, stats, pk, breakdown, clk=None, kclk=None):
     avg, _ = stats[name]
     ent = breakdown[name]
     if name.startswith("moe") or name.startswith("quant"):
@@ -514,12 +535,15 @@ def roofline_for(name, stats, pk, breakdown, clk=None):
         src = f"{pk['src']} MEASURED_PEAKS.json: HBM copy GB/s"
     else:
         achieved = ent["flops"] / avg / 1e12
-        peak, src = fp8_peak_for_clock(pk, clk)
+        peak, src = fp8_peak_for_clock(pk, clk, gemm_kernel_mhz(name, kclk))
         spec = SPEC_FP8_TFLOPS
         bound, unit = "tensor", "TFLOP/s"
-    return {"kernel": name, "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": recorded_traffic(name), "peak_source": src,
-            "spec_peak": spec, "frac_spec": round(achieved / spec, 4)}
+    out = {"kernel": name, "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+           "frac": round(achieved / peak, 4), "traffic": recorded_traffic(name), "peak_source": src,
+           "spec_peak": spec, "frac_spec": round(achieved / spec, 4)}
+    if bound == "tensor":
+        out["frac_burst"] = round(achieved / (pk["bf16"] * FP8_OVER_BF16), 4)
+    return out
 
 
 def linear_y_wx_latency(fp8q, device, reps=50):
@@ -587,6 +611,7 @@ def run_fp8q(args):
         raise RuntimeError(f"device status 0x{code:x} after warm-up")
 
     # ---- device-resident timed region
+    fp8q.fp8q_kernel_clock_counters(reset=True)
     uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     clocks = ClockSampler(uuid)
     clocks.path = os.path.join(LOG_DIR, f"clocks_rank{rank}.csv")
@@ -604,6 +629,9 @@ def run_fp8q(args):
     t1.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
+    kclk = fp8q.fp8q_kernel_clock_counters(reset=True)   # the SM clock inside the GEMM kernels
+    if clk is not None:
+        clk["gemm_kernel_sm_mhz"] = {k: v["mhz"] for k, v in kclk.items()}
     barrier(world, device)
     elapsed = t0.elapsed_time(t1) * 1e-3
     t_max = max_over_ranks(elapsed, world, device)
@@ -665,9 +693,9 @@ def run_fp8q(args):
     mt = st.mt
     moe_other = {"moe_up": mt * HID + (HID // 128) * mt * 4 + mt * MOE_FF + (MOE_FF // 128) * mt * 4,
                  "moe_down": mt * MOE_FF + (MOE_FF // 128) * mt * 4 + mt * HID * 2}
-    breakdown = build_breakdown(stats, pk, moe_w, moe_other, clk)
+    breakdown = build_breakdown(stats, pk, moe_w, moe_other, clk, kclk)
     dominant = max(stats, key=lambda n: stats[n][1])
-    roof = roofline_for(dominant, stats, pk, breakdown, clk)
+    roof = roofline_for(dominant, stats, pk, breakdown, clk, kclk)
     latency = {"linear_y_wx_us": linear_y_wx_latency(fp8q, device)}
 
     cpu = None
@@ -933,6 +961,7 @@ def run_single(args):
     clocks.path = os.path.join(LOG_DIR, f"clocks_single_{name}.csv")
     clocks.start()
     time.sleep(0.2)
+    fp8q.fp8q_kernel_clock_counters(reset=True)
     times = []
     for _ in range(args.steps):
         scrub.zero_()                       # evict the inputs from L2 between launches
@@ -942,6 +971,9 @@ def run_single(args):
         torch.cuda.synchronize()
         times.append(s.elapsed_time(e) * 1e-3)
     clk = clocks.stop()
+    kclk = fp8q.fp8q_kernel_clock_counters(reset=True)
+    if clk is not None:
+        clk["gemm_kernel_sm_mhz"] = {k: v["mhz"] for k, v in kclk.items()}
     code = fp8q.fp8q_device_status()
     t = float(np.median(times))
     out = {"kernel": name, "tokens": T, "median_us": round(t * 1e6, 2), "min_us": round(min(times) * 1e6, 2),

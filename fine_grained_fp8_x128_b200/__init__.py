@@ -59,6 +59,7 @@ EXPORTS = (
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
     "fp8q_moe_dispatch_layout_noalloc",
     "fp8q_quant_act_1x128_ue8m0", "fp8q_quant_w_128x128_ue8m0", "fp8q_gemm_mxf8_ue8m0",
+    "fp8q_kernel_clock_counters",
 )
 
 _P = ctypes.c_void_p
@@ -98,6 +99,7 @@ _lib.fp8q_grouped_gemm_blockscaled_q1x128.argtypes = [_P, _I, _P, _I, _P, _P, _P
 _lib.fp8q_debug_cast_e4m3_bits.argtypes = [ctypes.c_uint32, _I, _P, _P]
 _lib.fp8q_debug_wait_timeout.argtypes = [_I, _P]
 _lib.fp8q_debug_force_dense_kernel.argtypes = [ctypes.c_int]
+_lib.fp8q_kernel_clock_counters.argtypes = [_P, ctypes.c_int]
 _lib.fp8q_quant_act_1x128_ue8m0.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_quant_w_128x128_ue8m0.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_mxf8_ue8m0.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P]
@@ -390,6 +392,23 @@ def fp8q_gemm_mxf8_ue8m0(a, sfa_mx, b, sfb_mx, d, stream=None):
     N = b.shape[0]
     _check(_lib.fp8q_gemm_mxf8_ue8m0(_ptr(a), _ld(a), _ptr(sfa_mx), _ptr(b), _ld(b), _ptr(sfb_mx), _ptr(d), _ld(d),
                                      M, N, K, _stream(stream)), "fp8q_gemm_mxf8_ue8m0")
+
+
+GEMM_CLOCK_KINDS = ("pair", "one_cta", "pertensor", "mx")
+
+
+def fp8q_kernel_clock_counters(reset: bool = True) -> dict:
+    """Effective SM clock inside the GEMM kernels since the last reset:
+    {kind: {"cycles", "ns", "ctas", "mhz"}} for the kinds that ran."""
+    buf = (ctypes.c_ulonglong * 12)()
+    _check(_lib.fp8q_kernel_clock_counters(ctypes.cast(buf, ctypes.c_void_p), 1 if reset else 0),
+           "fp8q_kernel_clock_counters")
+    out = {}
+    for i, kind in enumerate(GEMM_CLOCK_KINDS):
+        cyc, ns, ctas = buf[3 * i], buf[3 * i + 1], buf[3 * i + 2]
+        if ctas:
+            out[kind] = {"cycles": cyc, "ns": ns, "ctas": ctas, "mhz": round(cyc / ns * 1e3, 1)}
+    return out
 
 
 def fp8q_debug_force_dense_kernel(choice: int):

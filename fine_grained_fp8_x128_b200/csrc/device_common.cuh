@@ -37,6 +37,36 @@ __device__ __forceinline__ void report_status(uint32_t code, uint32_t where) {
   atomicCAS(&g_status, 0u, (code & 0xFFu) | (where << 8));
 }
 
+// ---------------------------------------------------------------------------
+// Clock record of the GEMM kernels: each CTA adds its SM-clock cycles
+// (clock64) and nanoseconds (%globaltimer) from entry to exit, so that
+// cycles / ns is the effective SM clock inside the kernels of a kind -- the
+// clock a power-capped GEMM actually runs at, which a sampled nvidia-smi
+// reading does not resolve.  [kind][cycles, ns, CTAs]; read and cleared by
+// fp8q_kernel_clock_counters.
+// ---------------------------------------------------------------------------
+enum : int { CLOCK_PAIR = 0, CLOCK_ONE_CTA = 1, CLOCK_PERTENSOR = 2, CLOCK_MX = 3 };
+__device__ unsigned long long g_kernel_clock[4][3];
+
+struct KernelClock {
+  long long c0;
+  unsigned long long g0;
+};
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ KernelClock kernel_clock_begin() { return KernelClock{clock64(), global_timer_ns()}; }
+// Thread 0 of the CTA adds its span.
+__device__ __forceinline__ void kernel_clock_end(int kind, const KernelClock& k) {
+  if (threadIdx.x == 0) {
+    atomicAdd(&g_kernel_clock[kind][0], static_cast<unsigned long long>(clock64() - k.c0));
+    atomicAdd(&g_kernel_clock[kind][1], global_timer_ns() - k.g0);
+    atomicAdd(&g_kernel_clock[kind][2], 1ull);
+  }
+}
+
 // Default budget of one bounded wait in SM clocks: ~1 s at the B200's clocks.
 constexpr long long kWaitBudget = 1ll << 31;
 

@@ -958,6 +958,18 @@ fp8q_status fp8q_debug_cast_e4m3_bits(uint32_t start, int64_t count, void* out, 
   return launch_status();
 }
 
+fp8q_status fp8q_kernel_clock_counters(unsigned long long* out, int reset) {
+  if (out == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(out, fp8q::g_kernel_clock, sizeof(unsigned long long) * 12) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (reset) {
+    const unsigned long long zero[12] = {};
+    if (cudaMemcpyToSymbol(fp8q::g_kernel_clock, zero, sizeof(zero)) != cudaSuccess) return FP8Q_ERR_CUDA;
+  }
+  return FP8Q_OK;
+}
+
 fp8q_status fp8q_debug_force_dense_kernel(int choice) {
   if (choice != FP8Q_DENSE_AUTO && choice != FP8Q_DENSE_SINGLE && choice != FP8Q_DENSE_PAIR)
     return FP8Q_ERR_INVALID_ARG;

@@ -469,6 +469,7 @@ template <bool kGrouped, int kSfbMode, int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
+  const KernelClock kclock = kernel_clock_begin();
   extern __shared__ uint8_t gemm_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GemmSmemLayout::bars);
@@ -660,6 +661,7 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+  kernel_clock_end(CLOCK_ONE_CTA, kclock);
 }
 
 }  // namespace fp8q

@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
                  const __grid_constant__ CUtensorMap tmap_d, const GemmArgs p) {
+  const KernelClock kclock = kernel_clock_begin();
   extern __shared__ uint8_t pair_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pair_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PairSmemLayout::bars);
@@ -380,6 +381,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);
   }
+  kernel_clock_end(CLOCK_PAIR, kclock);
 }
 
 }  // namespace fp8q

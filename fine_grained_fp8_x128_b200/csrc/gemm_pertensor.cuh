@@ -106,6 +106,7 @@ template <int kOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_pertensor_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const GemmArgs p, const float* __restrict__ scale_a, const float* __restrict__ scale_b) {
+  const KernelClock kclock = kernel_clock_begin();
   extern __shared__ uint8_t pt_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pt_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PtSmemLayout::bars);
@@ -256,6 +257,7 @@ gemm_pertensor_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __g
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);
   }
+  kernel_clock_end(CLOCK_PERTENSOR, kclock);
 }
 
 }  // namespace fp8q

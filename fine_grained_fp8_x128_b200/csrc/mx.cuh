@@ -227,6 +227,7 @@ __device__ __forceinline__ void umma_mxf8f6f4(uint32_t tmem_d, uint64_t adesc, u
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_mx_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                const MxArgs p) {
+  const KernelClock kclock = kernel_clock_begin();
   extern __shared__ uint8_t mx_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(mx_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MxSmemLayout::bars);
@@ -375,6 +376,7 @@ gemm_mx_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+  kernel_clock_end(CLOCK_MX, kclock);
 }
 
 }  // namespace fp8q

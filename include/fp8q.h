@@ -547,6 +547,18 @@ fp8q_status fp8q_gemm_mxf8_ue8m0(const void* a, int64_t lda, const uint32_t* sfa
                                  const uint32_t* sfb_mx, void* d, int64_t ldd, int64_t M, int64_t N, int64_t K,
                                  void* stream);
 
+/*
+ * Clock record of the GEMM kernels.  Every CTA of a GEMM kernel adds, on exit,
+ * the SM-clock cycles and the nanoseconds (global timer) it ran; their ratio is
+ * the effective SM clock inside those kernels -- under sustained FP8 load the
+ * B200 lowers its clock to its power limit, which a sampled nvidia-smi reading
+ * does not resolve.  out receives 4 kinds x {cycles, ns, CTAs} as 12
+ * unsigned 64-bit counts: kind 0 the CTA-pair block-scaled GEMM, 1 the one-CTA
+ * and grouped GEMM, 2 the per-tensor GEMM, 3 the UE8M0 study's GEMM.
+ * Synchronises the device; reset != 0 clears the counters after the read.
+ */
+fp8q_status fp8q_kernel_clock_counters(unsigned long long* out, int reset);
+
 /* ---- diagnostics (used by the test suite; not on the hot path) ---------- */
 
 /*

@@ -16,6 +16,14 @@ def test_peak_follows_the_clock_record():
     assert sus == 2 * 1404.4 and "sustained" in why_s
     none, why_n = bench.fp8_peak_for_clock(PK, None)
     assert none == 2 * 1404.4 and "no clock record" in why_n
+    # the clock measured inside the GEMM kernels overrides the sampled median
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped, why_k = bench.fp8_peak_for_clock(PK, at_max, kernel_mhz=1370.0)
+    assert capped == 2 * 1404.4 and "inside the GEMM kernels 1370 MHz" in why_k
+    full, _ = bench.fp8_peak_for_clock(PK, at_max, kernel_mhz=1960.0)
+    assert full == 2 * 1662.0
+    kclk = {"pair": {"mhz": 1370.0}, "one_cta": {"mhz": 1450.0}}
+    assert bench.gemm_kernel_mhz("wgrad", kclk) == 1370.0 and bench.gemm_kernel_mhz("moe_up", kclk) == 1450.0
 
 
 def test_roofline_reproduces_from_the_breakdown():
@@ -29,6 +37,11 @@ def test_roofline_reproduces_from_the_breakdown():
     assert abs(roof["achieved"] - achieved) < 0.1
     assert abs(roof["frac"] - achieved / 3324.0) < 1e-4
     assert abs(roof["frac_spec"] - achieved / 4500.0) < 1e-4
+    assert abs(roof["frac_burst"] - achieved / 3324.0) < 1e-4
+    # with the in-kernel clock below max the sustained denominator applies
+    kclk = {"pair": {"mhz": 1370.0}}
+    roof2 = bench.roofline_for("wgrad", stats, PK, bench.build_breakdown(stats, PK, 0, {}, clk, kclk), clk, kclk)
+    assert abs(roof2["frac"] - achieved / 2808.8) < 1e-4
     assert abs(bd["wgrad"]["frac_fp8"] - achieved / 3324.0) < 1e-3
     assert bd["wgrad"]["bar_60pct_fp8_spec"] is False
     q = bd["quant_x"]

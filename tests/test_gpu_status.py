@@ -32,3 +32,22 @@ def test_bounded_wait_expires_and_reports(fp8q):
     oq, osf = oracle.quant_act_1x128(x)
     assert np.array_equal(q.cpu().numpy(), oq)
     assert fp8q.fp8q_device_status() == 0
+
+
+def test_gemm_clock_record(fp8q):
+    """Every GEMM CTA adds its SM cycles and global-timer nanoseconds on exit;
+    the ratio is the effective SM clock inside the kernels, and the CTA count
+    is the launch's grid."""
+    import torch
+    x = W.activations_with_outliers(512, 512, seed=2, channel_frac=0, elem_frac=0)
+    qa, sa = fp8q.quant_act_1x128(to_dev_bf16(x))
+    qb, sb = fp8q.quant_w_128x128(to_dev_bf16(W.weights(512, 512, seed=3)))
+    d = torch.empty((512, 512), dtype=torch.bfloat16, device="cuda")
+    fp8q.fp8q_kernel_clock_counters(reset=True)
+    fp8q.fp8q_gemm_blockscaled(qa, sa, qb, sb, fp8q.FP8Q_SFB_BLOCK128, d)      # M > 128: the CTA-pair kernel
+    rec = fp8q.fp8q_kernel_clock_counters(reset=True)
+    assert set(rec) == {"pair"}
+    assert rec["pair"]["ctas"] == 8                  # 2 m-pairs x 2 n-tiles, two CTAs each
+    assert 300.0 < rec["pair"]["mhz"] < 3000.0
+    assert fp8q.fp8q_kernel_clock_counters(reset=True) == {}
+    assert fp8q.fp8q_device_status() == 0
