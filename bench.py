@@ -4,9 +4,9 @@ A step is one pass of every hot-path operation over one batch of synthetic,
 seeded, outlier-injected input:
   dense linear layer, 8192 tokens x 7168 -> 18432 (forward and backward):
     quant_w_128x128(W, with W^T)           weights re-quantized once per step
-    quant_act_1x128(X)  -> Fprop  Y  = X W^T          (BF16 out)
-    quant_act_1x128(dY) -> Dgrad  dX = dY W           (BF16 out)
-    quant_act_128x1(dY), quant_act_128x1(X) -> Wgrad dW = dY^T X   (FP32 out)
+    quant_act_dual(X): 1x128 and 128x1 from one read  -> Fprop  Y  = X W^T   (BF16 out)
+    quant_act_dual(dY): 1x128 and 128x1 from one read -> Dgrad  dX = dY W    (BF16 out)
+    Wgrad dW = dY^T X on both 128x1 quantizations     (FP32 out)
   MoE layer, 4096 tokens, top-8 of 256 experts (Zipf 1.1), hidden 7168, expert 2048:
     quant_act_1x128 of each token once, scattered to its 8 expert rows (the dispatch)
     grouped up-projection, epilogue emitting H as 1x128 FP8 tiles
@@ -75,12 +75,16 @@ def quant_bytes():
     """Algorithmic bytes of each quantizer launch: read BF16 + write E4M3 + write FP32 scales."""
     def act(m, k):
         return m * k * 2 + m * k + (m * k // 128) * 4
+    def dual(m, k):   # one read, both orientations written (codes and scales twice)
+        return m * k * 2 + 2 * m * k + 2 * (m * k // 128) * 4
     return {
         "quant_w": OUT * HID * 2 + 2 * OUT * HID + 2 * (OUT // 128) * (HID // 128) * 4,
         "quant_x": act(TOK, HID),
         "quant_dy": act(TOK, OUT),
         "quant_dy_t": act(TOK, OUT),
         "quant_x_t": act(TOK, HID),
+        "quant_x_dual": dual(TOK, HID),
+        "quant_dy_dual": dual(TOK, OUT),
         # the gather reads each token once from HBM (the 59 MB of tokens stay
         # in the L2 across their top-k copies) and writes every expert row
         "quant_moe_x": MOE_TOK * HID * 2 + MOE_TOK * MOE_K * HID + (MOE_TOK * MOE_K * HID // 128) * 4,
@@ -297,11 +301,11 @@ def time_cpu_sample(sample: CpuSample):
 
 # ----------------------------------------------------------------------------- the device step
 class DeviceStep:
-    """All buffers of one step, resident on the device; step() launches the 11
+    """All buffers of one step, resident on the device; step() launches the 9
     kernels of the hot path on the current stream."""
 
-    KERNELS = ("quant_w", "quant_x", "fprop", "quant_dy", "dgrad", "quant_dy_t", "quant_x_t", "wgrad",
-               "quant_moe_x", "moe_up", "moe_down")
+    KERNELS = ("quant_w", "quant_x_dual", "fprop", "quant_dy_dual", "dgrad", "wgrad", "quant_moe_x", "moe_up",
+               "moe_down")
 
     def __init__(self, fp8q, seed: int, device):
         import torch
@@ -403,18 +407,18 @@ class DeviceStep:
         self.h_out.copy_(self.out, non_blocking=True)
 
     def step(self, events=None):
-        """Launch the 11 kernels; if `events` is a list, append (name, start, end) CUDA events."""
+        """Launch the 9 kernels; if `events` is a list, append (name, start, end) CUDA events."""
         import torch
         f = self.fp8q
         ops = (
             ("quant_w", lambda: f.fp8q_quant_w_128x128(self.w, self.wq, self.sw, self.wqt, self.swt)),
-            ("quant_x", lambda: f.fp8q_quant_act_1x128(self.x, self.xq, self.sx)),
+            # X in 1x128 tiles (Fprop) and 128x1 tiles (Wgrad) from one read
+            ("quant_x_dual", lambda: f.fp8q_quant_act_dual(self.x, self.xq, self.sx, self.xqt, self.sxt)),
             ("fprop", lambda: f.fp8q_gemm_blockscaled(self.xq, self.sx, self.wq, self.sw, f.FP8Q_SFB_BLOCK128, self.y)),
-            ("quant_dy", lambda: f.fp8q_quant_act_1x128(self.dy, self.dyq, self.sdy)),
+            # dY in 1x128 tiles (Dgrad) and 128x1 tiles (Wgrad) from one read
+            ("quant_dy_dual", lambda: f.fp8q_quant_act_dual(self.dy, self.dyq, self.sdy, self.dyqt, self.sdyt)),
             ("dgrad", lambda: f.fp8q_gemm_blockscaled(self.dyq, self.sdy, self.wqt, self.swt, f.FP8Q_SFB_BLOCK128,
                                                       self.dx)),
-            ("quant_dy_t", lambda: f.fp8q_quant_act_128x1(self.dy, self.dyqt, self.sdyt)),
-            ("quant_x_t", lambda: f.fp8q_quant_act_128x1(self.x, self.xqt, self.sxt)),
             ("wgrad", lambda: f.fp8q_gemm_blockscaled(self.dyqt, self.sdyt, self.xqt, self.sxt, f.FP8Q_SFB_ROW,
                                                       self.dw)),
             ("quant_moe_x", lambda: f.fp8q_quant_act_1x128_scatter(self.xm, self.pos, self.xpq, self.sxp)),
@@ -440,7 +444,8 @@ class DeviceStep:
 def config_block(world):
     return {
         "workload": ("one training step of a 8192-token linear layer 7168->18432 (weight quant with W^T, "
-                     "Fprop, Dgrad, Wgrad with 1x128 / 128x1 / 128x128 quantization) plus a 4096-token MoE "
+                     "X and dY each quantized 1x128 and 128x1 from one read, Fprop, Dgrad, Wgrad with "
+                     "1x128 / 128x1 / 128x128 quantization) plus a 4096-token MoE "
                      "layer (top-8 of 256 experts, Zipf 1.1, 8 empty; dispatch gather fused into the 1x128 "
                      "quantizer, grouped up 7168->2048 with FP8 epilogue, grouped down 2048->7168)"),
         "tokens": TOK, "hidden": HID, "out_features": OUT,
@@ -752,7 +757,8 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- single-kernel timing
-SINGLE_KERNELS = ("linear_y_wx", "mx_fprop", "fprop_single", "quant_x_ue8m0", "quant_w_ue8m0", "quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "quant_moe_x_gather", "moe_up", "moe_up_q",
+SINGLE_KERNELS = ("linear_y_wx", "mx_fprop", "fprop_single", "quant_x_dual", "quant_dy_dual", "quant_dy",
+                  "quant_dy_t", "quant_x_ue8m0", "quant_w_ue8m0", "quant_x", "quant_x_scaled", "quant_x_pct", "quant_x_pt", "pt_fprop", "quant_x_t", "requant_x_t", "quant_dy_e5m2", "dgrad_e5m2", "moe_dispatch", "moe_dispatch_nccl", "moe_layout", "quant_w", "fprop", "dgrad", "wgrad", "quant_moe_x", "quant_moe_x_gather", "moe_up", "moe_up_q",
                   "moe_down")
 
 
@@ -810,6 +816,21 @@ def run_single(args):
             sf = torch.empty((HID // 128, OUT // 128, 128), dtype=torch.int32, device=dev)
             fn = lambda: fp8q.fp8q_quant_w_128x128_ue8m0(w, q, sf)
             work = ("bytes", OUT * HID * 3 + OUT * HID // 128 * 4)
+    elif name in ("quant_x_dual", "quant_dy_dual", "quant_dy", "quant_dy_t"):
+        # both orientations from one read (dual), or the gradient's single-orientation passes
+        C = HID if name == "quant_x_dual" else OUT
+        x = randn(T, C) if name == "quant_x_dual" else randn(T, C, sigma=1e-3)
+        q = torch.empty((T, C), dtype=u8, device=dev); sf = torch.empty((C // 128, ld(T)), dtype=f32, device=dev)
+        qt = torch.empty((C, T), dtype=u8, device=dev); sft = torch.empty((T // 128, ld(C)), dtype=f32, device=dev)
+        if name == "quant_dy":
+            fn = lambda: fp8q.fp8q_quant_act_1x128(x, q, sf)
+            work = ("bytes", T * C * 3 + T * C // 128 * 4)
+        elif name == "quant_dy_t":
+            fn = lambda: fp8q.fp8q_quant_act_128x1(x, qt, sft)
+            work = ("bytes", T * C * 3 + T * C // 128 * 4)
+        else:
+            fn = lambda: fp8q.fp8q_quant_act_dual(x, q, sf, qt, sft)
+            work = ("bytes", T * C * 4 + 2 * (T * C // 128) * 4)
     elif name == "quant_x_pt":
         # per-tensor baseline quantizer: amax pass + cast pass (reads x twice)
         x = randn(T, HID)

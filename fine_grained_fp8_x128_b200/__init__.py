@@ -59,7 +59,7 @@ EXPORTS = (
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
     "fp8q_moe_dispatch_layout_noalloc",
     "fp8q_quant_act_1x128_ue8m0", "fp8q_quant_w_128x128_ue8m0", "fp8q_gemm_mxf8_ue8m0",
-    "fp8q_kernel_clock_counters",
+    "fp8q_kernel_clock_counters", "fp8q_quant_act_dual",
 )
 
 _P = ctypes.c_void_p
@@ -100,6 +100,7 @@ _lib.fp8q_debug_cast_e4m3_bits.argtypes = [ctypes.c_uint32, _I, _P, _P]
 _lib.fp8q_debug_wait_timeout.argtypes = [_I, _P]
 _lib.fp8q_debug_force_dense_kernel.argtypes = [ctypes.c_int]
 _lib.fp8q_kernel_clock_counters.argtypes = [_P, ctypes.c_int]
+_lib.fp8q_quant_act_dual.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_ue8m0.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_quant_w_128x128_ue8m0.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_mxf8_ue8m0.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P]
@@ -203,6 +204,14 @@ def fp8q_quant_act_128x1(x, qt, sf, stream=None):
     T, C = x.shape
     _check(_lib.fp8q_quant_act_128x1(_ptr(x), T, C, _ld(x), _ptr(qt), _ld(qt), _ptr(sf), _ld(sf), _stream(stream)),
            "fp8q_quant_act_128x1")
+
+
+def fp8q_quant_act_dual(x, q, sf, qt, sft, stream=None):
+    """Both orientations from one read: x bf16 [T][C] -> q uint8 [T][C] with sf [C/128][ld >= T]
+    (1x128 tiles) and qt uint8 [C][T] with sft [T/128][ld >= C] (128x1 tiles)."""
+    T, C = x.shape
+    _check(_lib.fp8q_quant_act_dual(_ptr(x), T, C, _ld(x), _ptr(q), _ld(q), _ptr(sf), _ld(sf), _ptr(qt), _ld(qt),
+                                    _ptr(sft), _ld(sft), _stream(stream)), "fp8q_quant_act_dual")
 
 
 def fp8q_quant_w_128x128(w, q, sf, qt=None, sft=None, stream=None):
@@ -457,6 +466,17 @@ def quant_pertensor(x, stream=None):
     amax_scale = torch.empty(2, dtype=torch.float32, device=x.device)
     fp8q_quant_pertensor(x, q, amax_scale, stream)
     return q, amax_scale
+
+
+def quant_act_dual(x, stream=None):
+    """Returns (q, sf, qt, sft): the 1x128 and the 128x1 quantizations of x from one read."""
+    T, C = x.shape
+    q = torch.empty((T, C), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((C // 128, sf_ld(T)), dtype=torch.float32, device=x.device)
+    qt = torch.empty((C, T), dtype=torch.uint8, device=x.device)
+    sft = torch.empty((T // 128, sf_ld(C)), dtype=torch.float32, device=x.device)
+    fp8q_quant_act_dual(x, q, sf, qt, sft, stream)
+    return q, sf, qt, sft
 
 
 def quant_act_128x1(x, stream=None):

@@ -51,6 +51,8 @@ struct DeviceInfo {
   int pt_cast_per_sm = 0;
   int q2_per_sm = 0;
   int qw_per_sm = 0;
+  bool qd_attr = false;            // both-orientation quantizer
+  int qd_per_sm = 0;
   bool mx_attr = false;            // UE8M0 block-scaled GEMM (study)
   int qmx_per_sm = 0;
   int qwmx_per_sm = 0;
@@ -865,6 +867,38 @@ fp8q_status fp8q_requant_1x128_to_128x1(const void* q, int64_t T, int64_t C, int
   fp8q::requant_1x128_to_128x1_kernel<<<static_cast<unsigned>(grid), fp8q::kQTThreads, fp8q::kRQSmem,
                                         static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t*>(q), T, C, ldq, sf_in, ld_sf_in, static_cast<uint8_t*>(qt), ldqt, sf, ld_sf);
+  return launch_status();
+}
+
+fp8q_status fp8q_quant_act_dual(const void* x, int64_t T, int64_t C, int64_t ldx, void* q, int64_t ldq, float* sf,
+                                int64_t ld_sf, void* qt, int64_t ldqt, float* sft, int64_t ld_sft, void* stream) {
+  if (T < 0 || C < 0 || T % 128 != 0 || C % 128 != 0 || ldx < C || ldq < C || ld_sf < T || ldqt < T ||
+      ld_sft < C)
+    return FP8Q_ERR_INVALID_ARG;
+  if (T == 0 || C == 0) return FP8Q_OK;
+  if (x == nullptr || q == nullptr || sf == nullptr || qt == nullptr || sft == nullptr) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(qt, 16) || !aligned(sf, 4) || !aligned(sft, 4) ||
+      ldx % 8 != 0 || ldq % 16 != 0 || ldqt % 16 != 0)
+    return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  auto kern = fp8q::quant_act_dual_kernel<fp8q::kFmtE4M3>;
+  const int smem = fp8q::kQTSmem;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!dev->qd_attr) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return FP8Q_ERR_CUDA;
+      dev->qd_attr = true;
+    }
+  }
+  const int64_t items = (T / 128) * (C / 128);
+  const int per_sm = blocks_per_sm(&dev->qd_per_sm, kern, fp8q::kQTThreads, smem);
+  const int64_t grid = grid_for(items, dev->sm_count, per_sm);
+  kern<<<static_cast<unsigned>(grid), fp8q::kQTThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), T, C, ldx, static_cast<uint8_t*>(q), ldq, sf, ld_sf,
+      static_cast<uint8_t*>(qt), ldqt, sft, ld_sft);
   return launch_status();
 }
 

@@ -339,8 +339,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         // 16x256b fragments: acc[64h + 32g + 4k + 2i + j] is row 32*quad + 16g +
         // 8i + lane/4, column 64h + 8k + 2*(lane%4) + j of this half; 4 lanes
         // write one 32-byte sector of a row per group k.  (Tensor stores of
-        // these fragments measured slower on B200: their staging raised the
-        // register pressure of the chunk loop.)
+        // these fragments measured slower on B200, twice: their staging raised
+        // the register pressure of the chunk loop.)
         if (vcol) {
 #pragma unroll
           for (int g = 0; g < 2; ++g) {

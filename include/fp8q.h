@@ -346,6 +346,26 @@ fp8q_status fp8q_requant_1x128_to_128x1(const void* q, int64_t T, int64_t C, int
                                         void* qt, int64_t ldqt, float* sf, int64_t ld_sf, void* stream);
 
 /*
+ * Both tile orientations of one BF16 tensor from a single read: the 1x128
+ * quantization of fp8q_quant_act_1x128 (operand A of the forward GEMM and of
+ * Dgrad) and the 128x1 transposed quantization of fp8q_quant_act_128x1
+ * (operand A or B of Wgrad), bit for bit the same codes and scales as those two
+ * calls.  The backward pass needs the gradient in both layouts ("Introduction
+ * to LLM Quantization", "3) Backward propagation"; "Fine-Grained FP8
+ * Quantization in DeepSeek", section 2 and section 4 "transpose layout"), and
+ * so does the activation: each 128-token x 128-channel tile is read from HBM
+ * once instead of twice.
+ *   x   : BF16 [T][ldx] (token t, channel c).
+ *   q   : E4M3 [T][ldq];  sf  : FP32 sf[(c/128) * ld_sf + t]   (as fp8q_quant_act_1x128).
+ *   qt  : E4M3 [C][ldqt]; sft : FP32 sft[(t/128) * ld_sft + c] (as fp8q_quant_act_128x1).
+ * Requirements: T % 128 == 0, C % 128 == 0, ldx >= C, ldq >= C, ldqt >= T,
+ * ld_sf >= T, ld_sft >= C; x, q, qt 16-byte aligned, ldx % 8 == 0,
+ * ldq % 16 == 0, ldqt % 16 == 0; sf, sft 4-byte aligned.
+ */
+fp8q_status fp8q_quant_act_dual(const void* x, int64_t T, int64_t C, int64_t ldx, void* q, int64_t ldq, float* sf,
+                                int64_t ld_sf, void* qt, int64_t ldqt, float* sft, int64_t ld_sft, void* stream);
+
+/*
  * 128x128 weight block quantization ("Fine-Grained FP8 Quantization in
  * DeepSeek", section 3 "Weights use 128x128 blocks"; "FP8 Mixed Precision",
  * eq. s_W = max|W_block| / 448).  Run once per optimizer step; the result is

@@ -42,8 +42,8 @@ def test_library_exports_every_declared_symbol(fp8q):
 
 def test_version_and_status_strings(fp8q):
     assert fp8q.fp8q_version() >= 100
-    for code in range(6):
-        assert fp8q.fp8q_status_string(code)
+    for code in range(7):
+        assert fp8q.fp8q_status_string(code) != "unknown status"
     assert fp8q.fp8q_status_string(99) == "unknown status"
 
 
@@ -64,6 +64,23 @@ def test_quant_act_validation(fp8q):
     assert L.fp8q_quant_act_128x1(FAKE, 128, 8, 8, FAKE, 120, FAKE, 8, None) == INV      # ldqt < T
     assert L.fp8q_quant_act_128x1(FAKE, 128, 8, 8, FAKE + 4, 128, FAKE, 8, None) == ALN
     assert L.fp8q_quant_act_128x1(None, 0, 8, 8, None, 0, None, 8, None) == 0
+
+
+def test_quant_dual_validation(fp8q):
+    L = fp8q.lib()
+    INV, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_ALIGNMENT
+
+    def qd(x=FAKE, T=256, C=256, ldx=256, q=FAKE, ldq=256, sf=FAKE, ld_sf=256, qt=FAKE, ldqt=256, sft=FAKE,
+           ld_sft=256):
+        return L.fp8q_quant_act_dual(x, T, C, ldx, q, ldq, sf, ld_sf, qt, ldqt, sft, ld_sft, None)
+
+    assert qd(T=200) == INV and qd(C=200) == INV and qd(T=-128) == INV          # whole 128 x 128 tiles
+    assert qd(ldx=128) == INV and qd(ldq=128) == INV and qd(ldqt=128) == INV
+    assert qd(ld_sf=128) == INV and qd(ld_sft=128) == INV
+    assert qd(x=None) == INV and qd(qt=None) == INV and qd(sft=None) == INV
+    assert qd(x=FAKE + 8) == ALN and qd(qt=FAKE + 8) == ALN and qd(ldx=260) == ALN and qd(ldq=264) == ALN
+    assert qd(ldqt=264) == ALN and qd(sf=FAKE + 2) == ALN
+    assert qd(T=0, x=None, q=None, sf=None, qt=None, sft=None) == 0          # empty: nothing launched
 
 
 def test_quant_gather_validation(fp8q):
