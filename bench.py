@@ -145,6 +145,14 @@ class ClockSampler:
                  "-lms", "20"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # nvidia-smi takes a few hundred ms to print its first sample: wait for it
+        # (up to 2 s), so that the samples cover the whole timed region
+        t_end = time.time() + 2.0
+        while time.time() < t_end and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
