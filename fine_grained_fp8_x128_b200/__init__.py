@@ -59,7 +59,7 @@ EXPORTS = (
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
     "fp8q_moe_dispatch_layout_noalloc",
     "fp8q_quant_act_1x128_ue8m0", "fp8q_quant_w_128x128_ue8m0", "fp8q_gemm_mxf8_ue8m0",
-    "fp8q_kernel_clock_counters", "fp8q_quant_act_dual",
+    "fp8q_kernel_clock_counters", "fp8q_quant_act_dual", "fp8q_moe_regroup_order",
 )
 
 _P = ctypes.c_void_p
@@ -85,6 +85,7 @@ _lib.fp8q_quant_act_1x128_gather_rowscales.argtypes = [_P, _I, _I, _I, _P, _I, _
 _lib.fp8q_quant_act_1x128_scatter.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_quant_act_1x128_scatter_rowscales.argtypes = [_P, _I, _I, _I, _P, ctypes.c_int, _I, _P, _I, _P, _I, _P]
 _lib.fp8q_gather_rows_fp8.argtypes = [_P, _I, _P, _I, _I, _P, _I, _I, _P, _I, _P, _I, _P]
+_lib.fp8q_moe_regroup_order.argtypes = [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I, _P, _P, _P]
 _lib.fp8q_quant_pertensor.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
 _lib.fp8q_gemm_pertensor.argtypes = [_P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_int, _I, _I, _I, _P]
 _lib.fp8q_scale_history_update.argtypes = [ctypes.c_int, ctypes.c_float, _P, _P, _P, _I, _P]
@@ -330,6 +331,15 @@ def fp8q_gather_rows_fp8(q_in, sf_in, rows, q_out, sf_out, stream=None):
     _check(_lib.fp8q_gather_rows_fp8(_ptr(q_in), _ld(q_in), _ptr(sf_in), _ld(sf_in), M_in, _ptr(rows), rows.numel(), K,
                                      _ptr(q_out), _ld(q_out), _ptr(sf_out), _ld(sf_out), _stream(stream)),
            "fp8q_gather_rows_fp8")
+
+
+def fp8q_moe_regroup_order(all_offsets, world, rank, num_experts, rows, expert_offsets, stream=None):
+    """rows int32 [M_recv] <- received row of each output row (local expert, then
+    source rank); expert_offsets int32 [num_experts/world + 1].  all_offsets:
+    int32 [world * (num_experts + 1)], every rank's layout offsets."""
+    _check(_lib.fp8q_moe_regroup_order(_ptr(all_offsets), int(world), int(rank), int(num_experts), rows.numel(),
+                                       _ptr(rows), _ptr(expert_offsets), _stream(stream)),
+           "fp8q_moe_regroup_order")
 
 
 def fp8q_quant_pertensor(x, q, amax_scale, stream=None):

@@ -31,6 +31,7 @@ enum : uint32_t {
   BAD_GROUP_OFFSETS = 7,
   BAD_ROW_INDEX = 8,
   BAD_EXPERT_ID = 9,
+  BAD_COUNT_TABLE = 10,
 };
 
 __device__ __forceinline__ void report_status(uint32_t code, uint32_t where) {

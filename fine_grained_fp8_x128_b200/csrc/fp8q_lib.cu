@@ -706,6 +706,26 @@ fp8q_status fp8q_gather_rows_fp8(const void* q_in, int64_t ldq_in, const float* 
   return launch_status();
 }
 
+fp8q_status fp8q_moe_regroup_order(const int32_t* all_offsets, int world, int rank, int num_experts, int64_t M_recv,
+                                   int32_t* rows, int32_t* expert_offsets, void* stream) {
+  if (world < 1 || rank < 0 || rank >= world || num_experts < 1 || num_experts > fp8q::kLayoutMaxExperts ||
+      num_experts % world != 0 || M_recv < 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M_recv > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED;
+  if (all_offsets == nullptr || expert_offsets == nullptr || (M_recv > 0 && rows == nullptr))
+    return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(all_offsets, 4) || !aligned(expert_offsets, 4) || !aligned(rows, 4)) return FP8Q_ERR_ALIGNMENT;
+  DeviceInfo* dev = nullptr;
+  fp8q_status st = device_info(&dev);
+  if (st != FP8Q_OK) return st;
+  const int64_t grid = grid_for((M_recv + fp8q::kRegroupOrderThreads - 1) / fp8q::kRegroupOrderThreads,
+                                dev->sm_count, 1);
+  fp8q::moe_regroup_order_kernel<<<static_cast<unsigned>(grid), fp8q::kRegroupOrderThreads, 0,
+                                   static_cast<cudaStream_t>(stream)>>>(all_offsets, world, rank, num_experts, M_recv,
+                                                                        rows, expert_offsets);
+  return launch_status();
+}
+
 fp8q_status fp8q_quant_act_1x128_scaled(const void* x, int64_t M, int64_t K, int64_t ldx, const float* sf,
                                         int64_t ld_sf, void* q, int64_t ldq, float* amax, int64_t ld_amax,
                                         unsigned long long* clipped, void* stream) {

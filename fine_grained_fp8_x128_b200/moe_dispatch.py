@@ -7,22 +7,24 @@ contiguous ranges over the ranks of the process group.  One call:
 
   1. layout (device): a stable counting sort of the (token, slot) entries by
      expert, giving the send order -- expert-major, hence rank-major;
-  2. quantize (device): each token's 1x128 FP8 codes and row-major scales,
-     computed once and written straight to its rows of the send buffer --
-     queued at once, since it needs only the layout's positions;
-  3. all_gather of every rank's expert offsets, read on the host once (the
-     one synchronisation of a call: the collective needs the split sizes);
-     that one table gives both what this rank sends to each rank and what it
-     receives per (source rank, local expert).  Without a process group
-     nothing is exchanged: each token is quantized once and scattered to its
-     rows of the grouped GEMM's input, and the host never waits;
-  4. all_to_all_single of the codes and of the scales (NCCL over NVLink on
-     GPUs);
+  2. all_gather of every rank's expert offsets, copied to the host
+     asynchronously;
+  3. quantize (device): each token's 1x128 FP8 codes and scales, computed once
+     and written straight to its rows of the send buffer; a send row holds the
+     codes and then the row's scales, so one exchange moves both.  It is queued
+     behind the copy of step 2, and the host waits only for that copy (the one
+     synchronisation of a call: the collective needs the split sizes), so the
+     quantizer runs while the host works out the splits.  The offsets table
+     gives both what this rank sends to each rank and what it receives per
+     (source rank, local expert).  Without a process group nothing is
+     exchanged: each token is quantized once and scattered to its rows of the
+     grouped GEMM's input, and the host never waits;
+  4. all_to_all_single of the packed rows (NCCL over NVLink on GPUs);
   5. regroup (device): the received rows from (source, expert) order into
      (expert, source) order, the scales into the grouped GEMM's K-chunk-major
      layout, so that the grouped GEMM runs on the result directly.  The order
-     is index arithmetic on the count table, uploaded from pinned memory
-     without another synchronisation.
+     is index arithmetic on the offsets table, done on the device from the
+     all-gathered table itself (`regroup_order` is its host statement).
 
 The device steps are this package's kernels (`CudaDispatchOps`).  The
 collectives are torch.distributed's.  The host part -- split sizes and the
@@ -43,16 +45,17 @@ class CudaDispatchOps:
         return moe_dispatch_layout(expert_ids, num_experts)
 
     def quant_send(self, x, pos, M):
-        """The send buffer: each token quantized once and written to its M-row
-        layout positions, scales row-major so that they travel with their rows."""
+        """The send buffer, uint8 [M][send_row_bytes(K)]: each token quantized
+        once and written to its M-row layout positions; a row holds the K codes
+        and then the row's K/128 FP32 scales, so they travel together."""
         import torch
         from . import fp8q_quant_act_1x128_scatter_rowscales
         K = x.shape[1]
-        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
-        sf = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+        buf = torch.empty((M, send_row_bytes(K)), dtype=torch.uint8, device=x.device)
+        q, sf = split_send_rows(buf, K)
         if M > 0 and x.shape[0] > 0:
             fp8q_quant_act_1x128_scatter_rowscales(x, pos, q, sf)
-        return q, sf
+        return buf
 
     def quant_grouped(self, x, pos, M):
         """Without an exchange: the grouped GEMM's input directly (scales K-chunk-major),
@@ -66,15 +69,39 @@ class CudaDispatchOps:
             fp8q_quant_act_1x128_scatter(x, pos, q, sf)
         return q, sf
 
-    def regroup(self, q, sf, rows):
+    def regroup_order(self, all_off, world, rank, num_experts, M):
+        """Device form of regroup_order from the all-gathered offsets table:
+        (rows int32 [M], local expert offsets int32 [el + 1])."""
+        import torch
+        from . import fp8q_moe_regroup_order
+        rows = torch.empty(M, dtype=torch.int32, device=all_off.device)
+        off = torch.empty(num_experts // world + 1, dtype=torch.int32, device=all_off.device)
+        fp8q_moe_regroup_order(all_off, world, rank, num_experts, rows, off)
+        return rows, off
+
+    def regroup(self, recv, K, rows):
         import torch
         from . import fp8q_gather_rows_fp8, sf_ld
-        M, K = rows.numel(), q.shape[1]
-        q_out = torch.empty((M, K), dtype=torch.uint8, device=q.device)
-        sf_out = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=q.device)
+        q, sf = split_send_rows(recv, K)
+        M = rows.numel()
+        q_out = torch.empty((M, K), dtype=torch.uint8, device=recv.device)
+        sf_out = torch.empty((K // 128, sf_ld(M)), dtype=torch.float32, device=recv.device)
         if M > 0:
             fp8q_gather_rows_fp8(q, sf, rows, q_out, sf_out)
         return q_out, sf_out
+
+
+def send_row_bytes(K: int) -> int:
+    """Bytes of one exchanged row: K FP8 codes, then K/128 FP32 scales, padded
+    to a multiple of 16 bytes."""
+    return (K + 4 * (K // 128) + 15) // 16 * 16
+
+
+def split_send_rows(buf, K: int):
+    """Views of a packed row buffer: the codes uint8 [M][K] and the scales
+    float32 [M][K/128] (both with the packed row stride)."""
+    import torch
+    return buf[:, :K], buf[:, K:K + 4 * (K // 128)].view(torch.float32)
 
 
 def regroup_order(recv_counts: np.ndarray):
@@ -111,28 +138,27 @@ class DispatchResult:
     recv_counts: np.ndarray  # int64 [world][E_local]: rows received per source rank and local expert (idem)
 
 
-_PINNED = {}
+_HOST = {}
 
 
-def _upload(a: np.ndarray, device):
-    """int32 host array -> device, through a cached pinned buffer (no host
-    synchronisation; the buffer is reused once its previous copy is done)."""
+def _to_host(t):
+    """Copies a small int32 device tensor to the host without waiting: returns
+    (host tensor, wait), where wait() blocks until the copy is done.  The host
+    buffer is pinned and kept per device; each call reads it before the next
+    call writes it."""
     import torch
-    t = torch.from_numpy(np.ascontiguousarray(a, np.int32))
-    if torch.device(device).type != "cuda":
-        return t.clone()
-    buf, ev = _PINNED.get(str(device), (None, None))
+    if t.device.type != "cuda":
+        return t, lambda: None
+    key = str(t.device)
+    buf = _HOST.get(key)
     if buf is None or buf.numel() < t.numel():
-        buf = torch.empty(max(t.numel(), 1 << 16), dtype=torch.int32, pin_memory=True)
-        ev = None
-    if ev is not None:
-        ev.synchronize()                    # the last copy out of this buffer has finished
-    buf[:t.numel()].copy_(t)
-    out = buf[:t.numel()].to(device, non_blocking=True)
+        buf = torch.empty(max(t.numel(), 4096), dtype=t.dtype, pin_memory=True)
+        _HOST[key] = buf
+    out = buf[:t.numel()]
+    out.copy_(t, non_blocking=True)
     ev = torch.cuda.Event()
     ev.record()
-    _PINNED[str(device)] = (buf, ev)
-    return out
+    return out, ev.synchronize
 
 
 def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchResult:
@@ -147,7 +173,6 @@ def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchR
         raise ValueError("num_experts must be a multiple of the group size")
     el = num_experts // world
     H = x.shape[1]
-    KB = H // 128
     rows, pos, offsets = ops.layout(expert_ids, num_experts)
     if not collective:
         # one process, all experts local: the layout order is the grouped GEMM's
@@ -156,21 +181,20 @@ def dispatch(x, expert_ids, num_experts: int, group=None, ops=None) -> DispatchR
         q, sf = ops.quant_grouped(x, pos, expert_ids.numel())
         return DispatchResult(q=q, sf=sf, expert_offsets=offsets, pos=pos, send_counts=None, recv_counts=None)
     rank = dist.get_rank(group)
-    q_send, sf_send = ops.quant_send(x, pos, expert_ids.numel())       # queued before the host waits
-    gathered = [torch.empty_like(offsets) for _ in range(world)]
-    dist.all_gather(gathered, offsets, group=group)
-    off_all = torch.stack(gathered).cpu().numpy().astype(np.int64)     # the one host sync: every rank's offsets
+    all_off = torch.empty(world * (num_experts + 1), dtype=offsets.dtype, device=offsets.device)
+    dist.all_gather_into_tensor(all_off, offsets, group=group)
+    off_host, wait = _to_host(all_off)
+    send = ops.quant_send(x, pos, expert_ids.numel())                  # runs while the host waits
+    wait()                                                              # the one host sync: every rank's offsets
+    off_all = off_host.numpy().astype(np.int64).reshape(world, num_experts + 1)
     per_expert = np.diff(off_all, axis=1)                               # [source rank][expert]
     send_counts = per_expert[rank].reshape(world, el).sum(axis=1)
     recv_counts = np.ascontiguousarray(per_expert[:, rank * el:(rank + 1) * el])
     recv_rows = recv_counts.sum(axis=1)
     M = int(recv_rows.sum())
-    q_recv = torch.empty((M, H), dtype=torch.uint8, device=x.device)
-    sf_recv = torch.empty((M, KB), dtype=torch.float32, device=x.device)
-    dist.all_to_all_single(q_recv, q_send, recv_rows.tolist(), send_counts.tolist(), group=group)
-    dist.all_to_all_single(sf_recv, sf_send, recv_rows.tolist(), send_counts.tolist(), group=group)
-    order, exp_off = regroup_order(recv_counts)
-    both = _upload(np.concatenate([order, exp_off]), x.device)
-    q, sf = ops.regroup(q_recv, sf_recv, both[:order.size])
-    return DispatchResult(q=q, sf=sf, expert_offsets=both[order.size:], pos=pos,
+    order, exp_off = ops.regroup_order(all_off, world, rank, num_experts, M)   # on the device, from the table
+    recv = torch.empty((M, send.shape[1]), dtype=torch.uint8, device=x.device)
+    dist.all_to_all_single(recv, send, recv_rows.tolist(), send_counts.tolist(), group=group)
+    q, sf = ops.regroup(recv, H, order)
+    return DispatchResult(q=q, sf=sf, expert_offsets=exp_off, pos=pos,
                           send_counts=send_counts, recv_counts=recv_counts)

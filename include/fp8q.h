@@ -90,8 +90,8 @@ const char* fp8q_status_string(fp8q_status s);
  * bits 8-31 say where it happened (which wait gave up, or which input check
  * failed).  Returns FP8Q_OK for a clean word, else the code in bits 0-7:
  * FP8Q_ERR_TIMEOUT (a bounded wait gave up) or FP8Q_ERR_INVALID_ARG (a
- * device-side input check failed: group offsets, a row index or an expert id
- * out of range).  FP8Q_ERR_CUDA if reading the word failed.
+ * device-side input check failed: group offsets, a row index, an expert id
+ * or a dispatch count table out of range).  FP8Q_ERR_CUDA if reading the word failed.
  */
 fp8q_status fp8q_device_status(void* stream, int* out_code);
 
@@ -234,6 +234,32 @@ fp8q_status fp8q_quant_act_1x128_gather_rowscales(const void* x, int64_t M_src, 
 fp8q_status fp8q_gather_rows_fp8(const void* q_in, int64_t ldq_in, const float* sf_in, int64_t ld_sf_in, int64_t M_in,
                                  const int32_t* rows, int64_t M_out, int64_t K, void* q_out, int64_t ldq_out,
                                  float* sf_out, int64_t ld_sf_out, void* stream);
+
+/*
+ * The regroup order of the dispatch exchange, built on the device from the
+ * exchanged layout offsets, so that the host needs nothing from the exchange
+ * but the split sizes.  Received rows arrive source-rank-major, each source's
+ * rows expert-major (the send order of fp8q_moe_dispatch_layout); the grouped
+ * GEMM wants them expert-major, each expert's rows source-major.  This call
+ * writes rows[m] = the received row that becomes output row m, for use with
+ * fp8q_gather_rows_fp8, and the local experts' output offsets.
+ *   all_offsets    : device int32 [world][num_experts + 1]: every rank's
+ *                    fp8q_moe_dispatch_layout offsets, rank-major (an all_gather).
+ *   world, rank    : the group size and this rank; this rank's experts are
+ *                    rank * el .. rank * el + el - 1, el = num_experts / world.
+ *   M_recv         : the rows this rank receives (the sum of its split sizes).
+ *   rows           : device int32 [M_recv] (caller-owned).
+ *   expert_offsets : device int32 [el + 1] (caller-owned): local expert e owns
+ *                    output rows expert_offsets[e] .. expert_offsets[e+1] - 1.
+ * Requirements: 1 <= num_experts <= 1024, num_experts % world == 0,
+ * 0 <= rank < world, M_recv < 2^31.  A table whose offsets decrease, or whose
+ * received total differs from M_recv, records FP8Q_ERR_INVALID_ARG in the
+ * device status word; output rows past the table's total get -1.  One launch,
+ * no workspace.  The pages describe the exchange, not this bookkeeping
+ * ("FP8 Mixed Precision: DeepSeek-V3 Training Architecture", section 4).
+ */
+fp8q_status fp8q_moe_regroup_order(const int32_t* all_offsets, int world, int rank, int num_experts, int64_t M_recv,
+                                   int32_t* rows, int32_t* expert_offsets, void* stream);
 
 /*
  * 1x128 quantization with GIVEN tile scales -- a scale policy's (fixed

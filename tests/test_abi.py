@@ -229,3 +229,17 @@ def test_debug_entry_validation(fp8q):
     assert L.fp8q_debug_cast_e4m3_bits(0, 0, None, None) == 0
     assert L.fp8q_debug_wait_timeout(0, None) == INV
     assert L.fp8q_debug_wait_timeout((1 << 34) + 1, None) == INV
+
+
+def test_regroup_order_validation(fp8q):
+    L = fp8q.lib()
+    INV, UNS, ALN = fp8q.FP8Q_ERR_INVALID_ARG, fp8q.FP8Q_ERR_UNSUPPORTED, fp8q.FP8Q_ERR_ALIGNMENT
+
+    def ro(off=FAKE, world=2, rank=0, E=16, M=100, rows=FAKE, eo=FAKE):
+        return L.fp8q_moe_regroup_order(off, world, rank, E, M, rows, eo, None)
+
+    assert ro(world=0) == INV and ro(rank=2) == INV and ro(rank=-1) == INV
+    assert ro(E=0) == INV and ro(E=2048, world=1) == INV and ro(E=15) == INV     # 15 % 2 != 0
+    assert ro(M=-1) == INV and ro(M=1 << 31) == UNS
+    assert ro(off=None) == INV and ro(eo=None) == INV and ro(rows=None) == INV
+    assert ro(off=FAKE + 2) == ALN and ro(rows=FAKE + 1) == ALN and ro(eo=FAKE + 3) == ALN

@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 import workloads as W
-from fine_grained_fp8_x128_b200.moe_dispatch import dispatch, regroup_order
+from fine_grained_fp8_x128_b200.moe_dispatch import dispatch, regroup_order, send_row_bytes
 
 
 def test_regroup_order_small():
@@ -61,25 +61,36 @@ class OracleOps:
         return torch.from_numpy(rows), torch.from_numpy(pos), torch.from_numpy(off)
 
     def quant_send(self, x, pos, M):
+        """Packed send rows: the codes, then the row's scales as bytes."""
         import torch
         qx, sx = oracle.quant_act_1x128(x.numpy())
+        K = qx.shape[1]
         p = pos.numpy()
         tok = np.nonzero(p >= 0)[0]
-        q = np.zeros((M, qx.shape[1]), np.uint8)
-        sf = np.zeros((M, sx.shape[1]), np.float32)
-        q[p[p >= 0]] = qx[tok]
-        sf[p[p >= 0]] = sx[tok]
-        return torch.from_numpy(q), torch.from_numpy(sf)
+        buf = np.zeros((M, send_row_bytes(K)), np.uint8)
+        buf[p[p >= 0], :K] = qx[tok]
+        buf[p[p >= 0], K:K + 4 * (K // 128)] = np.ascontiguousarray(sx[tok]).view(np.uint8)
+        return torch.from_numpy(buf)
 
-    def regroup(self, q, sf, rows):
+    def regroup_order(self, all_off, world, rank, num_experts, M):
+        """The host statement of the order, from the same offsets table."""
         import torch
-        r = rows.numpy()
-        return torch.from_numpy(q.numpy()[r]), torch.from_numpy(np.ascontiguousarray(sf.numpy()[r].T))
+        el = num_experts // world
+        per_expert = np.diff(all_off.numpy().astype(np.int64).reshape(world, num_experts + 1), axis=1)
+        rows, off = regroup_order(per_expert[:, rank * el:(rank + 1) * el])
+        assert rows.size == M
+        return torch.from_numpy(rows), torch.from_numpy(off)
+
+    def regroup(self, recv, K, rows):
+        import torch
+        r = np.asarray(rows)
+        b = recv.numpy()[r]
+        sf = np.ascontiguousarray(b[:, K:K + 4 * (K // 128)]).view(np.float32)
+        return torch.from_numpy(np.ascontiguousarray(b[:, :K])), torch.from_numpy(np.ascontiguousarray(sf.T))
 
     def quant_grouped(self, x, pos, M):
-        import torch
-        q, sf = self.quant_send(x, pos, M)
-        return q, torch.from_numpy(np.ascontiguousarray(sf.numpy().T))
+        K = x.shape[1]
+        return self.regroup(self.quant_send(x, pos, M), K, np.arange(M, dtype=np.int32))
 
 
 def test_dispatch_without_a_process_group():

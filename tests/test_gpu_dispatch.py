@@ -75,21 +75,88 @@ def test_gather_rowscales_matches_oracle(fp8q):
     assert np.array_equal(sh[:, :6], osf[rows]) and np.all(sh[:, 6:] == -1.0)
 
 
-def test_regroup_matches_numpy(fp8q):
+@pytest.mark.parametrize("K,packed", [(512, False), (4224, True), (7168, True)])
+def test_regroup_matches_numpy(fp8q, K, packed):
+    """Separate code and scale arrays, and the dispatch's packed receive rows
+    (codes then scales in one row); K = 4224 ends in a partial batch of
+    16-byte copies."""
     import torch
-    rng = np.random.default_rng(4)
-    M_in, M_out, K = 777, 1500, 512
+    from fine_grained_fp8_x128_b200.moe_dispatch import send_row_bytes, split_send_rows
+    rng = np.random.default_rng(4 + K)
+    M_in, M_out = 777, 1500
     q_in = rng.integers(0, 256, (M_in, K)).astype(np.uint8)
     sf_in = rng.random((M_in, K // 128)).astype(np.float32)
     rows = rng.integers(0, M_in, M_out).astype(np.int32)
     ld = M_out + 4
     q_out = torch.full((M_out, K), 0x5A, dtype=torch.uint8, device="cuda")
     sf_out = torch.full((K // 128, ld), -1.0, dtype=torch.float32, device="cuda")
-    fp8q.fp8q_gather_rows_fp8(to_dev_u8(q_in), to_dev_f32(sf_in), torch.from_numpy(rows).cuda(), q_out, sf_out)
+    if packed:
+        buf = np.zeros((M_in, send_row_bytes(K)), np.uint8)
+        buf[:, :K] = q_in
+        buf[:, K:K + 4 * (K // 128)] = sf_in.view(np.uint8)
+        qd, sd = split_send_rows(to_dev_u8(buf), K)
+    else:
+        qd, sd = to_dev_u8(q_in), to_dev_f32(sf_in)
+    fp8q.fp8q_gather_rows_fp8(qd, sd, torch.from_numpy(rows).cuda(), q_out, sf_out)
     assert fp8q.fp8q_device_status() == 0
     assert np.array_equal(q_out.cpu().numpy(), q_in[rows])
     s = sf_out.cpu().numpy()
     assert np.array_equal(s[:, :M_out], sf_in[rows].T) and np.all(s[:, M_out:] == -1.0)
+
+
+def _offsets_table(counts_all):
+    """Every source rank's layout offsets over all experts, rank-major."""
+    world, E = counts_all.shape
+    off = np.zeros((world, E + 1), np.int32)
+    off[:, 1:] = np.cumsum(counts_all, axis=1)
+    return off
+
+
+def test_regroup_order_kernel_matches_host(fp8q):
+    """The device order from the all-gathered offsets table against the host
+    statement (regroup_order) on random tables: 1 to 8 ranks, empty sources
+    and experts, every rank of the group, up to 1024 experts."""
+    import torch
+    from fine_grained_fp8_x128_b200.moe_dispatch import regroup_order
+    rng = np.random.default_rng(11)
+    cases = [(1, 256), (2, 8), (4, 64), (8, 1024), (3, 9), (8, 8)]
+    for world, E in cases:
+        el = E // world
+        counts_all = rng.integers(0, 40, (world, E))
+        counts_all[rng.random((world, E)) < 0.25] = 0
+        if world > 2:
+            counts_all[1, :] = 0                        # a source that sends nothing
+        off = torch.from_numpy(_offsets_table(counts_all).reshape(-1)).cuda()
+        for rank in range(world):
+            recv = counts_all[:, rank * el:(rank + 1) * el]
+            want_rows, want_off = regroup_order(recv)
+            M = int(recv.sum())
+            rows = torch.full((M,), -7, dtype=torch.int32, device="cuda")
+            eo = torch.full((el + 1,), -7, dtype=torch.int32, device="cuda")
+            fp8q.fp8q_moe_regroup_order(off, world, rank, E, rows, eo)
+            assert fp8q.fp8q_device_status() == 0
+            assert np.array_equal(rows.cpu().numpy(), want_rows), (world, E, rank)
+            assert np.array_equal(eo.cpu().numpy(), want_off), (world, E, rank)
+
+
+def test_regroup_order_kernel_reports_a_bad_table(fp8q):
+    """M_recv larger than the table's total: the extra rows get -1 and the
+    status word records FP8Q_ERR_INVALID_ARG; a decreasing table too."""
+    import torch
+    counts_all = np.array([[3, 0, 2, 1], [1, 4, 0, 2]])
+    off = torch.from_numpy(_offsets_table(counts_all).reshape(-1)).cuda()
+    rows = torch.full((8 + 3,), -7, dtype=torch.int32, device="cuda")
+    eo = torch.empty(3, dtype=torch.int32, device="cuda")
+    fp8q.fp8q_moe_regroup_order(off, 2, 0, 4, rows, eo)        # rank 0 receives 3+0+1+4 = 8 rows
+    assert fp8q.fp8q_device_status() & 0xFF == fp8q.FP8Q_ERR_INVALID_ARG
+    r = rows.cpu().numpy()
+    assert np.all(r[8:] == -1) and np.array_equal(np.sort(r[:8]), np.arange(8))
+    bad = _offsets_table(counts_all)
+    bad[1, 2] = bad[1, 1] - 1                                   # a decreasing offset
+    rows = torch.empty(8, dtype=torch.int32, device="cuda")
+    fp8q.fp8q_moe_regroup_order(torch.from_numpy(bad.reshape(-1)).cuda(), 2, 0, 4, rows, eo)
+    assert fp8q.fp8q_device_status() & 0xFF == fp8q.FP8Q_ERR_INVALID_ARG
+    assert fp8q.fp8q_device_status() == 0
 
 
 def _check_dispatch(res, x, ids, E):
