@@ -32,6 +32,7 @@ FP8Q_ERR_UNSUPPORTED = 3
 FP8Q_ERR_CUDA = 4
 FP8Q_ERR_TIMEOUT = 5
 FP8Q_ERR_SCRATCH_LIMIT = 6
+FP8Q_ERR_BOUNDS = 7
 FP8Q_LAYOUT_NOALLOC_SCRATCH_INTS = 262144
 FP8Q_SFB_BLOCK128 = 0
 FP8Q_SFB_ROW = 1
@@ -59,12 +60,13 @@ EXPORTS = (
     "fp8q_debug_cast_e4m3_bits", "fp8q_debug_wait_timeout", "fp8q_debug_force_dense_kernel",
     "fp8q_moe_dispatch_layout_noalloc",
     "fp8q_quant_act_1x128_ue8m0", "fp8q_quant_w_128x128_ue8m0", "fp8q_gemm_mxf8_ue8m0",
-    "fp8q_kernel_clock_counters", "fp8q_quant_act_dual", "fp8q_moe_regroup_order",
+    "fp8q_kernel_clock_counters", "fp8q_quant_act_dual", "fp8q_moe_regroup_order", "fp8q_build_checks",
 )
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int64
 _lib.fp8q_version.restype = ctypes.c_int
+_lib.fp8q_build_checks.restype = ctypes.c_int
 _lib.fp8q_status_string.argtypes = [ctypes.c_int]
 _lib.fp8q_status_string.restype = ctypes.c_char_p
 _lib.fp8q_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int)]
@@ -151,11 +153,16 @@ def _check(rc: int, call: str):
         raise FP8QError(rc, call)
 
 
+def fp8q_build_checks() -> bool:
+    """True for the checked build (device-side bounds checks, libfp8q_checks.so)."""
+    return bool(_lib.fp8q_build_checks())
+
+
 def fp8q_device_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word (0 = clean)."""
     code = ctypes.c_int(0)
     rc = _lib.fp8q_device_status(_stream(stream), ctypes.byref(code))
-    if rc not in (FP8Q_OK, FP8Q_ERR_TIMEOUT, FP8Q_ERR_INVALID_ARG):
+    if rc not in (FP8Q_OK, FP8Q_ERR_TIMEOUT, FP8Q_ERR_INVALID_ARG, FP8Q_ERR_BOUNDS):
         raise FP8QError(rc, "fp8q_device_status")
     return code.value
 

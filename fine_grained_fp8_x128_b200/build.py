@@ -10,6 +10,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfp8q.so")
+# The checked build: the same sources with -DFP8Q_CHECKS (device-side bounds
+# checks that record FP8Q_ERR_BOUNDS instead of writing out of bounds).
+LIB_CHECKS = os.path.join(HERE, "libfp8q_checks.so")
 MAIN = os.path.join(CSRC, "fp8q_lib.cu")
 
 NVCC_FLAGS = [
@@ -34,25 +37,27 @@ def _nvcc():
     return "nvcc"
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(checks: bool = False) -> bool:
+    lib = LIB_CHECKS if checks else LIB
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-o", tmp, MAIN]
+def build(force: bool = False, verbose: bool = False, checks: bool = False) -> str:
+    lib = LIB_CHECKS if checks else LIB
+    if not force and not needs_build(checks):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *NVCC_FLAGS, *(["-DFP8Q_CHECKS"] if checks else []), "-o", tmp, MAIN]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, checks="--checks" in sys.argv))

@@ -39,6 +39,34 @@ __device__ __forceinline__ void report_status(uint32_t code, uint32_t where) {
 }
 
 // ---------------------------------------------------------------------------
+// Debug bounds checks, compiled in with -DFP8Q_CHECKS (build.py --checks):
+// chk(i, n, site) holds when 0 <= i < n; otherwise it records FP8Q_ERR_BOUNDS
+// and the site in the status word, and the caller skips the access.  Without
+// the flag it is the constant true and the compiler drops it.  Sites:
+// ---------------------------------------------------------------------------
+enum : uint32_t {
+  CHK_Q1 = 16,        // 1x128 quantizers: codes
+  CHK_Q1_SF = 17,     //   and scales
+  CHK_SCATTER = 18,   // dispatch scatter quantizer: codes and scales
+  CHK_QT = 19,        // 128x1 and dual quantizers: transposed codes
+  CHK_QT_SF = 20,     //   and their scales
+  CHK_QW = 21,        // weight quantizer: codes, transposed codes, scales
+  CHK_GEMM_D = 22,    // GEMM tile-end stores
+  CHK_GEMM_SFD = 23,  // GEMM FP8 epilogue scales
+  CHK_GROUP = 24,     // grouped GEMM: a tile's rows inside its group and M_total
+  CHK_LAYOUT = 25,    // dispatch layout and regroup: row maps
+};
+#ifdef FP8Q_CHECKS
+__device__ __forceinline__ bool chk(int64_t i, int64_t n, uint32_t site) {
+  if (i >= 0 && i < n) return true;
+  report_status(FP8Q_ERR_BOUNDS, site);
+  return false;
+}
+#else
+__device__ __forceinline__ constexpr bool chk(int64_t, int64_t, uint32_t) { return true; }
+#endif
+
+// ---------------------------------------------------------------------------
 // Clock record of the GEMM kernels: each CTA adds its SM-clock cycles
 // (clock64) and nanoseconds (%globaltimer) from entry to exit, so that
 // cycles / ns is the effective SM clock inside the kernels of a kind -- the

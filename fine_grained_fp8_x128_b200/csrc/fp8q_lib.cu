@@ -557,8 +557,17 @@ const char* fp8q_status_string(fp8q_status s) {
     case FP8Q_ERR_CUDA: return "CUDA error";
     case FP8Q_ERR_TIMEOUT: return "device-side bounded wait gave up";
     case FP8Q_ERR_SCRATCH_LIMIT: return "request needs more scratch than the fixed no-allocation array holds";
+    case FP8Q_ERR_BOUNDS: return "device-side bounds check failed (checked build)";
     default: return "unknown status";
   }
+}
+
+int fp8q_build_checks(void) {
+#ifdef FP8Q_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 fp8q_status fp8q_device_status(void* stream, int* out_code) {
@@ -575,8 +584,9 @@ fp8q_status fp8q_device_status(void* stream, int* out_code) {
   if (word == 0) return FP8Q_OK;
   // bits 0-7 hold the FP8Q_ERR_* code of the first report
   const unsigned int code = word & 0xFFu;
-  return code == FP8Q_ERR_INVALID_ARG || code == FP8Q_ERR_TIMEOUT ? static_cast<fp8q_status>(code)
-                                                                  : FP8Q_ERR_CUDA;
+  return code == FP8Q_ERR_INVALID_ARG || code == FP8Q_ERR_TIMEOUT || code == FP8Q_ERR_BOUNDS
+             ? static_cast<fp8q_status>(code)
+             : FP8Q_ERR_CUDA;
 }
 
 fp8q_status fp8q_quant_act_1x128(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, int64_t ldq,

@@ -266,7 +266,7 @@ __device__ __forceinline__ void store_rows128_tma64(const float2* acc, int lane,
         put(chunk);
         tma_store_pass(buf, tmap_d, ncol0 + 64 * h, row0, lane);
       }
-      p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
+      if (chk(row0 + lane, p.ld_sfd, CHK_GEMM_SFD)) p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
     }
   }
 }
@@ -324,7 +324,8 @@ __device__ __forceinline__ void store_rows128_staged4(const float2* acc, int lan
         }
         stage_store_pass4(stage, chunk, lane, base + 64 * h, p.ldd, rows_valid);
       }
-      if (lane < rows_valid) p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
+      if (lane < rows_valid && chk(row0 + lane, p.ld_sfd, CHK_GEMM_SFD))
+        p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
     }
   }
 }
@@ -385,7 +386,8 @@ __device__ __forceinline__ void store_rows128_staged(const float2* acc, int lane
       }
       stage_store_pass(stage, chunk, lane, static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0,
                        p.ldd, rows_valid);
-      if (lane < rows_valid) p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
+      if (lane < rows_valid && chk(row0 + lane, p.ld_sfd, CHK_GEMM_SFD))
+        p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
     }
   }
 }
@@ -646,7 +648,10 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
         // a box of 32 full rows leaves as tensor stores; a part-filled box (the
         // last rows of an expert or of M) keeps the per-row staged stores, so
         // nothing is written past the expert's rows
-        if (rows_valid == 32)
+        const bool inside = rows_valid <= 0 || (chk(row0, p.M, CHK_GROUP) && chk(row0 + rows_valid - 1, p.M, CHK_GROUP) &&
+                                                chk(ncol0 + 127, p.N, CHK_GEMM_D));
+        if (!inside) {
+        } else if (rows_valid == 32)
           store_rows128_tma64<kOut>(acc, lane, row0, ncol0, p, &tmap_d, out_buf);
         else if (rows_valid > 0)
           store_rows128_staged4<kOut>(acc, lane, row0, rows_valid, ncol0, p, reinterpret_cast<uint4*>(out_buf));

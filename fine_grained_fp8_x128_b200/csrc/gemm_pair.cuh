@@ -351,6 +351,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
               const int64_t base = static_cast<int64_t>(r) * p.ldd + ncol0 + 2 * (lane & 3);
 #pragma unroll
               for (int k = 0; k < 16; ++k) {   // k < 8: first 64 columns, k >= 8: second
+                if (!chk(ncol0 + 8 * k + 2 * (lane & 3) + 1, p.N, CHK_GEMM_D)) continue;
                 const int x = 64 * (k >> 3) + 32 * g + 4 * (k & 7) + 2 * i;
                 const float x0 = acc[x / 2].x, x1 = acc[x / 2].y;
                 if (kOut == kOutF32) {
@@ -363,7 +364,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             }
           }
         }
-      } else if (vcol && row0 < p.M) {
+      } else if (vcol && row0 < p.M && chk(ncol0 + 127, p.N, CHK_GEMM_D)) {
         if (kOut == kOutE4m3)
           store_rows128_staged<kOut>(acc, lane, row0, min(32, p.M - row0), ncol0, p,
                                      reinterpret_cast<uint4*>(out_buf));

@@ -120,7 +120,7 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     const float s = tile_scale_fmt<kFmt>(m);
     const float nr = -__frcp_rn(s);
-    if (row < M) {
+    if (row < M && chk(kb * 128 + sub * 8 + 32 * 3 + 7, ldq, CHK_Q1)) {
       uint8_t* dst = q + row * ldq + kb * 128 + sub * 8;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -133,10 +133,12 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
           *reinterpret_cast<uint2*>(dst + 32 * i) = o;
       }
       if (sub == 0) {
-        if (kRowScales)
-          sf[row * ld_sf + kb] = s;      // row-major [M][ld_sf >= K/128]: a row's scales travel with it
-        else
+        if (kRowScales) {
+          if (chk(kb, ld_sf, CHK_Q1_SF))
+            sf[row * ld_sf + kb] = s;    // row-major [M][ld_sf >= K/128]: a row's scales travel with it
+        } else if (chk(row, ld_sf, CHK_Q1_SF)) {
           sf[kb * ld_sf + row] = s;
+        }
       }
     }
     cur = nxt;
@@ -198,14 +200,16 @@ quant_act_1x128_scatter_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, i
           if (sub == 0 && kb == 0) report_status(FP8Q_ERR_INVALID_ARG, BAD_ROW_INDEX);
           continue;
         }
+        if (!chk(kb * 128 + sub * 8 + 32 * 3 + 7, ldq, CHK_SCATTER)) continue;
         uint8_t* d = q + dst * ldq + kb * 128 + sub * 8;
 #pragma unroll
         for (int i = 0; i < 4; ++i) __stcs(reinterpret_cast<uint2*>(d + 32 * i), o[i]);
         if (sub == 0) {
-          if (kRowScales)
-            sf[dst * ld_sf + kb] = s;
-          else
+          if (kRowScales) {
+            if (chk(kb, ld_sf, CHK_SCATTER)) sf[dst * ld_sf + kb] = s;
+          } else if (chk(dst, ld_sf, CHK_SCATTER)) {
             sf[kb * ld_sf + dst] = s;
+          }
         }
       }
     }
@@ -460,7 +464,7 @@ __device__ __forceinline__ void qt_stage(uint32_t* tile, const __nv_bfloat16* __
 // warp store instruction then writes 4 whole 128-byte rows of qt.
 __device__ __forceinline__ void qt_store_transposed(uint8_t* smem16k, const uint4 (&codes)[4], bool active,
                                                     int64_t tb, int64_t c0, int64_t ncols,
-                                                    uint8_t* __restrict__ qt, int64_t ldqt, int tid) {
+                                                    uint8_t* __restrict__ qt, int64_t ldqt, int64_t qt_rows, int tid) {
   const int p = tid & 63;
   const int r = tid >> 6;
   __syncthreads();
@@ -477,7 +481,8 @@ __device__ __forceinline__ void qt_store_transposed(uint8_t* smem16k, const uint
   const int warp = tid >> 5, lane = tid & 31;
   for (int row = 4 * warp + (lane >> 3); row < ncols; row += 4 * (kQTThreads / 32)) {
     const int j = lane & 7;
-    *reinterpret_cast<uint4*>(qt + (c0 + row) * ldqt + tb * 128 + 16 * j) = crows[row * 8 + (j ^ ((row >> 1) & 7))];
+    if (chk(c0 + row, qt_rows, CHK_QT) && chk(tb * 128 + 16 * j + 15, ldqt, CHK_QT))
+      *reinterpret_cast<uint4*>(qt + (c0 + row) * ldqt + tb * 128 + 16 * j) = crows[row * 8 + (j ^ ((row >> 1) & 7))];
   }
 }
 
@@ -490,7 +495,7 @@ __device__ __forceinline__ void qt_store_transposed(uint8_t* smem16k, const uint
 template <int kFmt = kFmtE4M3>
 __device__ __forceinline__ void qt_cast_staged(uint8_t* tile_bytes, float* qmax, int64_t tb, int64_t c0,
                                                int64_t ncols, uint8_t* __restrict__ qt, int64_t ldqt,
-                                               float* __restrict__ sf, int64_t ld_sf, int tid) {
+                                               float* __restrict__ sf, int64_t ld_sf, int64_t C, int tid) {
   const int p = tid & 63;          // channel pair
   const int r = tid >> 6;          // token quarter
   constexpr int kWords = kQTCols / 2;   // 64 words per staged row
@@ -535,12 +540,12 @@ __device__ __forceinline__ void qt_cast_staged(uint8_t* tile_bytes, float* qmax,
       codes[h] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
       codes[2 + h] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
     }
-    if (r == 0) {
+    if (r == 0 && chk(ca + 1, ld_sf, CHK_QT_SF)) {
       sf[tb * ld_sf + ca] = sa;
       sf[tb * ld_sf + ca + 1] = sb;
     }
   }
-  qt_store_transposed(tile_bytes, codes, active, tb, c0, ncols, qt, ldqt, tid);
+  qt_store_transposed(tile_bytes, codes, active, tb, c0, ncols, qt, ldqt, C, tid);
 }
 
 template <int kFmt = kFmtE4M3>
@@ -569,7 +574,7 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
     const int64_t tb = it / col_blocks;
     const int64_t c0 = (it - tb * col_blocks) * kQTCols;
     const int64_t ncols = (C - c0) < kQTCols ? (C - c0) : kQTCols;
-    qt_cast_staged<kFmt>(q2_smem + buf * kQTTileBytes, qmax, tb, c0, ncols, qt, ldqt, sf, ld_sf, tid);
+    qt_cast_staged<kFmt>(q2_smem + buf * kQTTileBytes, qmax, tb, c0, ncols, qt, ldqt, sf, ld_sf, C, tid);
     __syncthreads();   // this buffer is refilled two items later; the maxima are reused next item
   }
 }
@@ -658,14 +663,16 @@ quant_act_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C,
         const float nr = -__frcp_rn(s);
         const int64_t row = tb * 128 + r;
         uint8_t* dst = q + row * ldq + cb * 128 + sub * 8;
+        if (chk(row, T, CHK_Q1) && chk(cb * 128 + sub * 8 + 32 * 3 + 7, ldq, CHK_Q1)) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint2 o;
-          o.x = quant_words<kFmt>(v[i].x, v[i].y, nr, s);
-          o.y = quant_words<kFmt>(v[i].z, v[i].w, nr, s);
-          *reinterpret_cast<uint2*>(dst + 32 * i) = o;
+          for (int i = 0; i < 4; ++i) {
+            uint2 o;
+            o.x = quant_words<kFmt>(v[i].x, v[i].y, nr, s);
+            o.y = quant_words<kFmt>(v[i].z, v[i].w, nr, s);
+            *reinterpret_cast<uint2*>(dst + 32 * i) = o;
+          }
         }
-        if (sub == 0) sf[cb * ld_sf + row] = s;
+        if (sub == 0 && chk(row, ld_sf, CHK_Q1_SF)) sf[cb * ld_sf + row] = s;
       }
     }
 
@@ -705,13 +712,13 @@ quant_act_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C,
         codes[h] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
         codes[2 + h] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
       }
-      if (r == 0) {
+      if (r == 0 && chk(cb * 128 + 2 * p + 1, ld_sft, CHK_QT_SF)) {
         sft[tb * ld_sft + cb * 128 + 2 * p] = sa;
         sft[tb * ld_sft + cb * 128 + 2 * p + 1] = sb;
       }
       // the transposed codes leave through the tile's first 16 KB once every
       // thread has finished reading it (both passes)
-      qt_store_transposed(tile_bytes, codes, true, tb, cb * 128, 128, qt, ldqt, tid);
+      qt_store_transposed(tile_bytes, codes, true, tb, cb * 128, 128, qt, ldqt, C, tid);
     }
     __syncthreads();   // this buffer is refilled two items later; the maxima are reused next item
   }
@@ -854,7 +861,7 @@ requant_1x128_to_128x1_kernel(const uint8_t* __restrict__ q, int64_t T, int64_t 
       sf[tb * ld_sf + c0 + 2 * p] = sa;
       sf[tb * ld_sf + c0 + 2 * p + 1] = sb;
     }
-    qt_store_transposed(st, codes, true, tb, c0, kQTCols, qt, ldqt, tid);
+    qt_store_transposed(st, codes, true, tb, c0, kQTCols, qt, ldqt, C, tid);
     __syncthreads();   // this stage buffer is refilled next item; the maxima are reused
   }
 }
@@ -922,7 +929,8 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
     for (int i = 0; i < 8; ++i) {
       lo[i] = quant_words(v[i].x, v[i].y, nr, s);
       hi[i] = quant_words(v[i].z, v[i].w, nr, s);
-      *reinterpret_cast<uint2*>(q + (n0 + 8 * a + i) * ldq + k0 + 8 * b) = make_uint2(lo[i], hi[i]);
+      if (chk(n0 + 8 * a + i, NB * 128, CHK_QW) && chk(k0 + 8 * b + 7, ldq, CHK_QW))
+        *reinterpret_cast<uint2*>(q + (n0 + 8 * a + i) * ldq + k0 + 8 * b) = make_uint2(lo[i], hi[i]);
     }
     if (qt != nullptr) {
       uint32_t c00[4], c01[4], c10[4], c11[4];   // c<rowhalf><colhalf>
@@ -944,12 +952,13 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
       for (int i = 0; i < 8; ++i) {
         const int kk = 16 * i + (tid >> 4);   // 16 rows per pass over the block's 256 threads
         const int c = tid & 15;
-        *reinterpret_cast<uint2*>(qt + (k0 + kk) * ldqt + n0 + 8 * c) = tstage[kk * 16 + (c ^ ((kk >> 3) & 15))];
+        if (chk(k0 + kk, KB * 128, CHK_QW) && chk(n0 + 8 * c + 7, ldqt, CHK_QW))
+          *reinterpret_cast<uint2*>(qt + (k0 + kk) * ldqt + n0 + 8 * c) = tstage[kk * 16 + (c ^ ((kk >> 3) & 15))];
       }
     }
     if (tid == 0) {
-      sf[nb * ld_sf + kb] = s;
-      if (sft != nullptr) sft[kb * ld_sft + nb] = s;
+      if (chk(kb, ld_sf, CHK_QW)) sf[nb * ld_sf + kb] = s;
+      if (sft != nullptr && chk(nb, ld_sft, CHK_QW)) sft[kb * ld_sft + nb] = s;
     }
     __syncthreads();   // warp_max is reused by the next block
   }
@@ -1073,7 +1082,7 @@ moe_layout_scatter_kernel(const int32_t* __restrict__ ids, int64_t n, int k, int
     __syncwarp();
     if (i < hi) {
       pos[i] = p;
-      if (p >= 0) rows[p] = static_cast<int32_t>(i / k);
+      if (p >= 0 && chk(p, n, CHK_LAYOUT)) rows[p] = static_cast<int32_t>(i / k);
     }
   }
 }
@@ -1160,7 +1169,8 @@ moe_regroup_order_kernel(const int32_t* __restrict__ off, int world, int rank, i
       const int mid = (lo + hi) >> 1;
       if (out_start[mid] <= m) lo = mid; else hi = mid;
     }
-    rows[m] = recv_start[lo] + static_cast<int32_t>(m - out_start[lo]);
+    const int32_t src = recv_start[lo] + static_cast<int32_t>(m - out_start[lo]);
+    rows[m] = chk(src, M_recv, CHK_LAYOUT) ? src : -1;
   }
 }
 

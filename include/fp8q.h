@@ -48,7 +48,8 @@ enum {
   FP8Q_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement     */
   FP8Q_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed     */
   FP8Q_ERR_TIMEOUT = 5,      /* a kernel gave up a bounded wait (device status) */
-  FP8Q_ERR_SCRATCH_LIMIT = 6 /* request exceeds a fixed no-allocation scratch     */
+  FP8Q_ERR_SCRATCH_LIMIT = 6, /* request exceeds a fixed no-allocation scratch    */
+  FP8Q_ERR_BOUNDS = 7        /* checked build: a computed index left its buffer   */
 };
 
 /* Scale layouts for operand B of fp8q_gemm_blockscaled. */
@@ -89,11 +90,24 @@ const char* fp8q_status_string(fp8q_status s);
  * problem; otherwise bits 0-7 hold the FP8Q_ERR_* code of the first report and
  * bits 8-31 say where it happened (which wait gave up, or which input check
  * failed).  Returns FP8Q_OK for a clean word, else the code in bits 0-7:
- * FP8Q_ERR_TIMEOUT (a bounded wait gave up) or FP8Q_ERR_INVALID_ARG (a
+ * FP8Q_ERR_TIMEOUT (a bounded wait gave up), FP8Q_ERR_INVALID_ARG (a
  * device-side input check failed: group offsets, a row index, an expert id
- * or a dispatch count table out of range).  FP8Q_ERR_CUDA if reading the word failed.
+ * or a dispatch count table out of range) or, in a checked build only,
+ * FP8Q_ERR_BOUNDS.  FP8Q_ERR_CUDA if reading the word failed.
  */
 fp8q_status fp8q_device_status(void* stream, int* out_code);
+
+/*
+ * 1 if this library was built with device-side bounds checks (-DFP8Q_CHECKS,
+ * `python fine_grained_fp8_x128_b200/build.py --checks`, libfp8q_checks.so),
+ * else 0.  In a checked build the kernels compare each computed global index
+ * of their stores (and of the dispatch's row maps) with the extent their
+ * arguments give; an index outside it records FP8Q_ERR_BOUNDS and the site
+ * in the device status word instead of being written, so a bad index shows
+ * up as a status, not as a fault.  Results are otherwise bit-identical to
+ * the unchecked build.
+ */
+int fp8q_build_checks(void);
 
 /*
  * Online 1x128 activation quantization.

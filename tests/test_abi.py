@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(fp8q):
 
 def test_version_and_status_strings(fp8q):
     assert fp8q.fp8q_version() >= 100
-    for code in range(7):
+    for code in range(8):
         assert fp8q.fp8q_status_string(code) != "unknown status"
     assert fp8q.fp8q_status_string(99) == "unknown status"
 
@@ -243,3 +243,18 @@ def test_regroup_order_validation(fp8q):
     assert ro(M=-1) == INV and ro(M=1 << 31) == UNS
     assert ro(off=None) == INV and ro(eo=None) == INV and ro(rows=None) == INV
     assert ro(off=FAKE + 2) == ALN and ro(rows=FAKE + 1) == ALN and ro(eo=FAKE + 3) == ALN
+
+
+def test_checked_build_exports_the_same_symbols(fp8q):
+    """The checked build (-DFP8Q_CHECKS) is the same C ABI and says so; the
+    default build says it is not checked."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("fp8q_build", os.path.join(ROOT, "fine_grained_fp8_x128_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    checked = ctypes.CDLL(b.build(checks=True))
+    for name in declared_symbols():
+        assert hasattr(checked, name), name
+    assert checked.fp8q_build_checks() == 1
+    assert ctypes.CDLL(b.LIB).fp8q_build_checks() == 0
+    assert fp8q.fp8q_status_string(fp8q.FP8Q_ERR_BOUNDS) != "unknown status"
