@@ -250,8 +250,8 @@ __device__ __forceinline__ void store_rows128_tma64(const float2* acc, int lane,
     } else {
       uint32_t m2 = 0;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
-      const float s = tile_scale(amax2_value(m2));
+      for (int j = 0; j < 64; ++j) m2 = amax2_sx(m2, w[j]);
+      const float s = tile_scale(amax2_value(amax2_sx_bits(m2)));
       const float nr = -__frcp_rn(s);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -308,8 +308,8 @@ __device__ __forceinline__ void store_rows128_staged4(const float2* acc, int lan
     } else {
       uint32_t m2 = 0;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
-      const float s = tile_scale(amax2_value(m2));
+      for (int j = 0; j < 64; ++j) m2 = amax2_sx(m2, w[j]);
+      const float s = tile_scale(amax2_value(amax2_sx_bits(m2)));
       const float nr = -__frcp_rn(s);
       uint8_t* base = static_cast<uint8_t*>(p.d) + static_cast<int64_t>(row0) * p.ldd + ncol0;
 #pragma unroll
@@ -374,8 +374,8 @@ __device__ __forceinline__ void store_rows128_staged(const float2* acc, int lane
     } else {
       uint32_t m2 = 0;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) m2 = amax2(m2, w[j]);
-      const float s = tile_scale(amax2_value(m2));
+      for (int j = 0; j < 64; ++j) m2 = amax2_sx(m2, w[j]);
+      const float s = tile_scale(amax2_value(amax2_sx_bits(m2)));
       const float nr = -__frcp_rn(s);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {

@@ -25,6 +25,17 @@ __device__ __forceinline__ uint32_t amax2(uint32_t m, uint32_t w) {
 }
 __device__ __forceinline__ float amax2_value(uint32_t m) { return fmaxf(bf16lo(m), bf16hi(m)); }
 
+// The same running maximum in one instruction: max.xorsign.abs keeps the
+// larger magnitude of each lane (its sign bit is the XOR of the inputs' signs,
+// cleared by amax2_sx_bits at the end); .NaN keeps a NaN, as the integer form
+// does (NaN patterns compare above every finite value and infinity).
+__device__ __forceinline__ uint32_t amax2_sx(uint32_t m, uint32_t w) {
+  uint32_t r;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(w));
+  return r;
+}
+__device__ __forceinline__ uint32_t amax2_sx_bits(uint32_t m) { return m & 0x7FFF7FFFu; }
+
 // Four BF16 values (two words) -> four E4M3 codes, one byte each in element
 // order: q = e4m3(fl32(x / s)), with nr = -fl32(1/s) (see e4m3x2_neg_quot,
 // which returns the codes with inverted signs; one XOR flips all four back).
@@ -112,10 +123,10 @@ quant_act_1x128_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K
     uint32_t m2 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      m2 = amax2(m2, cur.v[i].x); m2 = amax2(m2, cur.v[i].y);
-      m2 = amax2(m2, cur.v[i].z); m2 = amax2(m2, cur.v[i].w);
+      m2 = amax2_sx(m2, cur.v[i].x); m2 = amax2_sx(m2, cur.v[i].y);
+      m2 = amax2_sx(m2, cur.v[i].z); m2 = amax2_sx(m2, cur.v[i].w);
     }
-    float m = amax2_value(m2);
+    float m = amax2_value(amax2_sx_bits(m2));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     const float s = tile_scale_fmt<kFmt>(m);
@@ -178,10 +189,10 @@ quant_act_1x128_scatter_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, i
     uint32_t m2 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      m2 = amax2(m2, cur.v[i].x); m2 = amax2(m2, cur.v[i].y);
-      m2 = amax2(m2, cur.v[i].z); m2 = amax2(m2, cur.v[i].w);
+      m2 = amax2_sx(m2, cur.v[i].x); m2 = amax2_sx(m2, cur.v[i].y);
+      m2 = amax2_sx(m2, cur.v[i].z); m2 = amax2_sx(m2, cur.v[i].w);
     }
-    float m = amax2_value(m2);
+    float m = amax2_value(amax2_sx_bits(m2));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     const float s = tile_scale(m);
@@ -506,7 +517,8 @@ __device__ __forceinline__ void qt_cast_staged(uint8_t* tile_bytes, float* qmax,
   if (active) {
     uint32_t m2 = 0;   // channel 2p in the low half, 2p+1 in the high half
 #pragma unroll 8
-    for (int t = 32 * r; t < 32 * r + 32; ++t) m2 = amax2(m2, tile[t * kWords + p]);
+    for (int t = 32 * r; t < 32 * r + 32; ++t) m2 = amax2_sx(m2, tile[t * kWords + p]);
+    m2 = amax2_sx_bits(m2);
     ma = bf16lo(m2);
     mb = bf16hi(m2);
   }
@@ -595,10 +607,6 @@ quant_act_128x1_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C
 // kernel), the 128x1 pass gives a warp 32 consecutive channel-pair words of one
 // row.  Requires C % 128 == 0 (whole tiles).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int dual_word(int t, int w) {   // 32-bit word w of staged row t
-  return t * 64 + (((w >> 2) ^ (t & 15)) << 2) + (w & 3);
-}
-
 __device__ __forceinline__ void dual_stage(uint32_t* tile, const __nv_bfloat16* __restrict__ x, int64_t ldx,
                                            int64_t col_blocks, int64_t it, int tid) {
   const int64_t tb = it / col_blocks;
@@ -653,10 +661,10 @@ quant_act_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C,
         uint32_t m2 = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          m2 = amax2(m2, v[i].x); m2 = amax2(m2, v[i].y);
-          m2 = amax2(m2, v[i].z); m2 = amax2(m2, v[i].w);
+          m2 = amax2_sx(m2, v[i].x); m2 = amax2_sx(m2, v[i].y);
+          m2 = amax2_sx(m2, v[i].z); m2 = amax2_sx(m2, v[i].w);
         }
-        float m = amax2_value(m2);
+        float m = amax2_value(amax2_sx_bits(m2));
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
         const float s = tile_scale_fmt<kFmt>(m);
@@ -681,9 +689,17 @@ quant_act_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C,
       const int p = tid & 63;          // channel pair
       const int r = tid >> 6;          // token quarter
       uint4 codes[4];
+      // word p of token row 32r + k sits at k * 64 + woff[k % 16] from row 32r
+      // (32r is a multiple of 16, so the swizzle depends on k alone): the 16
+      // offsets are formed once and every load below is a base plus a constant
+      const uint32_t* trow = tile + 32 * r * 64;
+      int woff[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) woff[c] = (((p >> 2) ^ c) << 2) + (p & 3);
       uint32_t m2 = 0;
-#pragma unroll 8
-      for (int t = 32 * r; t < 32 * r + 32; ++t) m2 = amax2(m2, tile[dual_word(t, p)]);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) m2 = amax2_sx(m2, trow[k * 64 + woff[k & 15]]);
+      m2 = amax2_sx_bits(m2);
       float ma = bf16lo(m2), mb = bf16hi(m2);
       qmax[r * 128 + 2 * p] = ma;
       qmax[r * 128 + 2 * p + 1] = mb;
@@ -700,9 +716,9 @@ quant_act_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t T, int64_t C,
           uint32_t a4 = 0, b4 = 0;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int t = 32 * r + 16 * h + 4 * j + 2 * e;
-            const uint32_t w0 = tile[dual_word(t, p)];
-            const uint32_t w1 = tile[dual_word(t + 1, p)];
+            const int k = 16 * h + 4 * j + 2 * e;   // token 32r + k
+            const uint32_t w0 = trow[k * 64 + woff[k & 15]];
+            const uint32_t w1 = trow[(k + 1) * 64 + woff[(k + 1) & 15]];
             a4 |= fp8x2_neg_quot<kFmt>(bf16lo(w0), bf16lo(w1), nra, nra, sa, sa) << (16 * e);
             b4 |= fp8x2_neg_quot<kFmt>(bf16hi(w0), bf16hi(w1), nrb, nrb, sb, sb) << (16 * e);
           }
@@ -911,10 +927,10 @@ quant_w_128x128_kernel(const __nv_bfloat16* __restrict__ w, int64_t NB, int64_t 
     uint32_t m2 = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      m2 = amax2(m2, v[i].x); m2 = amax2(m2, v[i].y);
-      m2 = amax2(m2, v[i].z); m2 = amax2(m2, v[i].w);
+      m2 = amax2_sx(m2, v[i].x); m2 = amax2_sx(m2, v[i].y);
+      m2 = amax2_sx(m2, v[i].z); m2 = amax2_sx(m2, v[i].w);
     }
-    float m = amax2_value(m2);
+    float m = amax2_value(amax2_sx_bits(m2));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((tid & 31) == 0) warp_max[tid >> 5] = m;
