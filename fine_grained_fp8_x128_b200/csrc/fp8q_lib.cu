@@ -293,13 +293,19 @@ int64_t layout_chunks(int64_t n) {
 // 256-row tile pairs, m fastest.  Keep whichever operand fits in about 40% of
 // the 126 MB L2 resident and stream the other once: A resident -> one group
 // over all of M; B resident -> groups of one tile pair (all of N sweeps past
-// each 256 rows of A).  Otherwise groups of 8 tile pairs (2048 rows), which
-// measured fewer DRAM bytes on B200 than smaller groups sized to the L2.
-int64_t pair_group_m(int64_t m_pairs, int64_t a_bytes, int64_t b_bytes) {
+// each 256 rows of A).  Otherwise groups of 16 tile pairs when their rows of A
+// take at most 32 MiB, else 8 (2048 rows): each group streams all of B once,
+// so fewer groups re-read B fewer times, as long as a wave's A rows and B
+// columns still fit the L2.  On B200 (same box, alternating) 16 took Fprop
+// (K = 7168, 29 MiB of A per group) from 936 to 921 us, left Wgrad (K = 8192)
+// as it was, and made Dgrad (K = 18432, 72 MiB) 1 % slower; smaller groups
+// sized to the L2 measured more DRAM bytes, not fewer.
+int64_t pair_group_m(int64_t m_pairs, int64_t a_bytes, int64_t b_bytes, int64_t K) {
   const int64_t kResident = 48ll << 20;
   if (a_bytes <= kResident) return m_pairs < 1 ? 1 : m_pairs;
   if (b_bytes <= kResident) return 1;
-  return m_pairs < 8 ? m_pairs : 8;
+  const int64_t g = 16 * 256 * K <= (32ll << 20) ? 16 : 8;
+  return m_pairs < g ? m_pairs : g;
 }
 
 // Dense kernel choice set by fp8q_debug_force_dense_kernel (a test hook):
@@ -408,7 +414,7 @@ fp8q_status gemm_dense(const void* a, int64_t lda, const float* sfa, int64_t ld_
   const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
   const int64_t m_pairs = (M + 2 * fp8q::BM - 1) / (2 * fp8q::BM);
   const int64_t pair_tiles = m_pairs * args.num_n_tiles;
-  args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
+  args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K, K));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return sfb_mode == FP8Q_SFB_BLOCK128
              ? dense_launch<FP8Q_SFB_BLOCK128>(dev, pair, out, ta, tb, tsa, tsb, td, args, pair_tiles, grid, s)
@@ -845,7 +851,7 @@ fp8q_status fp8q_gemm_pertensor(const void* a, int64_t lda, const float* scale_a
   const int64_t m_pairs = (M + 2 * fp8q::BM - 1) / (2 * fp8q::BM);
   const int64_t pair_tiles = m_pairs * args.num_n_tiles;
   if (pair_tiles > kIntMax) return FP8Q_ERR_UNSUPPORTED;
-  args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K));
+  args.group_m = static_cast<int>(pair_group_m(m_pairs, M * K, N * K, K));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d_dtype == FP8Q_OUT_F32
              ? launch_gemm_pertensor<fp8q::kOutF32>(dev, ta, tb, args, scale_a, scale_b, pair_tiles, s)
