@@ -144,8 +144,9 @@ _HOST = {}
 def _to_host(t):
     """Copies a small int32 device tensor to the host without waiting: returns
     (host tensor, wait), where wait() blocks until the copy is done.  The host
-    buffer is pinned and kept per device; each call reads it before the next
-    call writes it."""
+    buffer is pinned and kept per device; a dispatch reads it before it
+    returns, so calls from one thread never overlap on it (concurrent
+    dispatches from several host threads on one device would)."""
     import torch
     if t.device.type != "cuda":
         return t, lambda: None
