@@ -152,9 +152,9 @@ fp8q_status make_tmap_f32(CUtensorMap* map, const float* base, int64_t inner, in
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
-// Output matrix [rows][ld] of BF16 (esz 2) or FP32 (esz 4) for the pair
-// kernel's tile-end tensor stores: box {128 bytes, 32 rows}, 128-byte swizzle
-// (the layout of the epilogue's staging buffer).
+// Output matrix [rows][ld] of E4M3 codes (esz 1), BF16 (esz 2) or FP32 (esz 4)
+// for the GEMMs' tile-end tensor stores: box {128 bytes, 32 rows}, 128-byte
+// swizzle (the layout of the epilogues' staging buffers).
 fp8q_status make_tmap_out(CUtensorMap* map, void* base, int64_t cols, int64_t rows, int64_t ld, int esz) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   fp8q_status st = encoder(&enc);
@@ -163,27 +163,11 @@ fp8q_status make_tmap_out(CUtensorMap* map, void* base, int64_t cols, int64_t ro
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esz)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 32u};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(map, esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
-}
-
-// The same for the one-CTA kernel: box {64 bytes, 32 rows} with the 64-byte
-// swizzle of its 2 KB staging buffers; esz 1 (E4M3 codes), 2 (BF16) or 4 (FP32).
-fp8q_status make_tmap_out64(CUtensorMap* map, void* base, int64_t cols, int64_t rows, int64_t ld, int esz) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
-  fp8q_status st = encoder(&enc);
-  if (st != FP8Q_OK) return st;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esz)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / esz), 32u};
-  cuuint32_t estr[2] = {1u, 1u};
   const CUtensorMapDataType dt = esz == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                  : esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUresult r = enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_CUDA;
 }
 
@@ -193,7 +177,7 @@ fp8q_status launch_gemm(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMa
   // the output's tensor map for the tile-end stores of full 32-row boxes
   CUtensorMap td;
   const int esz = OUT == fp8q::kOutF32 ? 4 : (OUT == fp8q::kOutE4m3 ? 1 : 2);
-  fp8q_status st = make_tmap_out64(&td, args.d, args.N, args.M, args.ldd, esz);
+  fp8q_status st = make_tmap_out(&td, args.d, args.N, args.M, args.ldd, esz);
   if (st != FP8Q_OK) return st;
   const uint32_t smem = (G ? fp8q::GemmSmemLayout::bytes_grouped : fp8q::GemmSmemLayout::bytes_dense) + 1024;
   auto kern = fp8q::gemm_blockscaled_kernel<G, MODE, OUT>;

@@ -25,6 +25,7 @@
 //   warps 10-11: idle (they complete the third warpgroup for setmaxnreg).
 // Pipelines:
 //   smem ring  : kStages x (A 128x128 + B 256x128 E4M3).
+//   tile-end   : two 4 KB staging buffers per epilogue warp for the tensor stores.
 //   TMEM       : 2 chunk accumulators of 128 lanes x 256 FP32 columns (all 512
 //                columns): the MMAs of chunk c+1 overlap the promotion of c.
 //   row scales : (FP8Q_SFB_ROW only) a ring of per-chunk B scale vectors.
@@ -47,7 +48,7 @@ namespace fp8q {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 #ifndef FP8Q_SB_RING
 #define FP8Q_SB_RING 8
 #endif
@@ -58,6 +59,9 @@ constexpr uint32_t kABytes = BM * BK;               // 16 KB
 constexpr uint32_t kBBytes = BN * BK;               // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes; // 48 KB
 constexpr uint32_t kSbBytes = BN * 4;               // 1 KB
+// Tile-end staging per epilogue warp: two 4 KB buffers (32 rows x 128 bytes
+// each), so a tile's tensor stores leave without waiting for one another.
+constexpr uint32_t kOutStageBytes = 8192;
 constexpr int kMaxGroups = 1024;
 constexpr int kGroupM = 16;                          // L2 swizzle: m-tiles per group
 
@@ -65,8 +69,8 @@ struct GemmSmemLayout {
   // offsets from the 1024-aligned base
   static constexpr uint32_t stages = 0;
   static constexpr uint32_t sb_ring = stages + kStages * kStageBytes;
-  static constexpr uint32_t out_stage = sb_ring + kSbRing * kSbBytes;   // 8 epilogue warps x 2 KB, 1024-aligned
-  static constexpr uint32_t bars = out_stage + 8 * 2048;
+  static constexpr uint32_t out_stage = sb_ring + kSbRing * kSbBytes;   // 8 epilogue warps x 8 KB, 1024-aligned
+  static constexpr uint32_t bars = out_stage + 8 * kOutStageBytes;
   // barriers: go[S], done[S], sbfull[R], sbempty[R]
   static constexpr uint32_t nbars = 2 * kStages + 2 * kSbRing;
   static constexpr uint32_t misc = bars + nbars * 8;           // tmem base, abort flag
@@ -206,30 +210,43 @@ __device__ __forceinline__ void tma_store_pass(uint8_t* buf, const CUtensorMap* 
   __syncwarp();
 }
 
-// store_rows128_staged4 for a warp whose 32 rows are all valid, through
-// tensor stores: each pass's 32 rows x 64 bytes go into the 2 KB buffer in
-// the 64-byte-swizzled layout of stage_store_pass4 (chunk j of row r at
-// j ^ ((r / 2) % 4), the tensor map's SWIZZLE_64B pattern) and leave as one
-// box.  kOutE4m3 also writes the row's tile scale, as the staged version does.
+// The tile-end store of a warp whose 32 rows are all valid, through tensor
+// stores of 128-byte boxes from two 4 KB buffers (the output's tensor map:
+// SWIZZLE_128B, box 128 bytes x 32 rows; chunk j of row r at j ^ (r % 8)).  BF16: 64 columns per box, both boxes issued back to back;
+// E4M3: all 128 codes of a row in one box; FP32: 32 columns per box, the two
+// buffers used twice.  The warp waits only before it refills a buffer that a
+// store may still be reading -- at the start of the next tile's stores -- so a
+// tile's global writes overlap the next tile's chunks.
 template <int kOut>
-__device__ __forceinline__ void store_rows128_tma64(const float2* acc, int lane, int row0, int ncol0,
-                                                    const GemmArgs& p, const CUtensorMap* tmap_d, uint8_t* buf) {
-  uint4* stage = reinterpret_cast<uint4*>(buf);
-  auto put = [&](const uint4(&chunk)[4]) {
+__device__ __forceinline__ void store_rows128_tma128(const float2* acc, int lane, int row0, int ncol0,
+                                                     const GemmArgs& p, const CUtensorMap* tmap_d, uint8_t* buf) {
+  auto put = [&](uint8_t* b, const uint4 (&chunk)[8]) {
+    uint4* stage = reinterpret_cast<uint4*>(b);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) stage[lane * 4 + (j ^ ((lane >> 1) & 3))] = chunk[j];
+    for (int j = 0; j < 8; ++j) stage[lane * 8 + (j ^ (lane & 7))] = chunk[j];
   };
-  uint4 chunk[4];
+  auto issue = [&](uint8_t* b, int x) {
+    fence_proxy_async_shared();   // the buffer's generic-proxy writes, before the async-proxy read
+    __syncwarp();
+    if (lane == 0) tma_store_2d(tmap_d, b, x, row0);
+  };
+  if (lane == 0) bulk_wait_group_read0();   // the previous tile's stores have read both buffers
+  __syncwarp();
+  uint4 chunk[8];
   if (kOut == kOutF32) {
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
+    for (int h = 0; h < 4; ++h) {
+      if (h == 2) {                  // the buffers come round again
+        if (lane == 0) { bulk_commit_group(); bulk_wait_group_read0(); }
+        __syncwarp();
+      }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 a = acc[8 * h + 2 * j], b = acc[8 * h + 2 * j + 1];
+      for (int j = 0; j < 8; ++j) {
+        const float2 a = acc[16 * h + 2 * j], b = acc[16 * h + 2 * j + 1];
         chunk[j] = make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
       }
-      put(chunk);
-      tma_store_pass(buf, tmap_d, ncol0 + 16 * h, row0, lane);
+      put(buf + 4096 * (h & 1), chunk);
+      issue(buf + 4096 * (h & 1), ncol0 + 32 * h);
     }
   } else {
     uint32_t w[64];   // BF16 pairs
@@ -240,12 +257,12 @@ __device__ __forceinline__ void store_rows128_tma64(const float2* acc, int lane,
     }
     if (kOut == kOutBf16) {
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          chunk[j] = make_uint4(w[16 * h + 4 * j], w[16 * h + 4 * j + 1], w[16 * h + 4 * j + 2], w[16 * h + 4 * j + 3]);
-        put(chunk);
-        tma_store_pass(buf, tmap_d, ncol0 + 32 * h, row0, lane);
+        for (int j = 0; j < 8; ++j)
+          chunk[j] = make_uint4(w[32 * h + 4 * j], w[32 * h + 4 * j + 1], w[32 * h + 4 * j + 2], w[32 * h + 4 * j + 3]);
+        put(buf + 4096 * h, chunk);
+        issue(buf + 4096 * h, ncol0 + 64 * h);
       }
     } else {
       uint32_t m2 = 0;
@@ -254,21 +271,19 @@ __device__ __forceinline__ void store_rows128_tma64(const float2* acc, int lane,
       const float s = tile_scale(amax2_value(amax2_sx_bits(m2)));
       const float nr = -__frcp_rn(s);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int j = 0; j < 8; ++j) {
+        uint32_t c[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t c[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            c[j] = quant_words(w[32 * h + 8 * i + 2 * j], w[32 * h + 8 * i + 2 * j + 1], nr, s);
-          chunk[i] = make_uint4(c[0], c[1], c[2], c[3]);
-        }
-        put(chunk);
-        tma_store_pass(buf, tmap_d, ncol0 + 64 * h, row0, lane);
+        for (int e = 0; e < 4; ++e) c[e] = quant_words(w[8 * j + 2 * e], w[8 * j + 2 * e + 1], nr, s);
+        chunk[j] = make_uint4(c[0], c[1], c[2], c[3]);
       }
+      put(buf, chunk);
+      issue(buf, ncol0);
       if (chk(row0 + lane, p.ld_sfd, CHK_GEMM_SFD)) p.sfd[static_cast<int64_t>(ncol0 / 128) * p.ld_sfd + row0 + lane] = s;
     }
   }
+  if (lane == 0) bulk_commit_group();
+  __syncwarp();
 }
 
 // store_rows128_staged through a 2 KB buffer: 8 passes of 16 FP32 columns, 4
@@ -644,17 +659,20 @@ gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid
       if (vcol) {   // warp-uniform
         const int row0 = c.a_row0 + quad * 32;
         const int rows_valid = min(32, c.row_end - row0);
-        uint8_t* out_buf = smem + GemmSmemLayout::out_stage + warp * 2048;
+        uint8_t* out_buf = smem + GemmSmemLayout::out_stage + warp * kOutStageBytes;
         // a box of 32 full rows leaves as tensor stores; a part-filled box (the
         // last rows of an expert or of M) keeps the per-row staged stores, so
         // nothing is written past the expert's rows
         const bool inside = rows_valid <= 0 || (chk(row0, p.M, CHK_GROUP) && chk(row0 + rows_valid - 1, p.M, CHK_GROUP) &&
                                                 chk(ncol0 + 127, p.N, CHK_GEMM_D));
         if (!inside) {
-        } else if (rows_valid == 32)
-          store_rows128_tma64<kOut>(acc, lane, row0, ncol0, p, &tmap_d, out_buf);
-        else if (rows_valid > 0)
+        } else if (rows_valid == 32) {
+          store_rows128_tma128<kOut>(acc, lane, row0, ncol0, p, &tmap_d, out_buf);
+        } else if (rows_valid > 0) {
+          if (lane == 0) bulk_wait_group_read0();   // earlier tensor stores have read the buffer
+          __syncwarp();
           store_rows128_staged4<kOut>(acc, lane, row0, rows_valid, ncol0, p, reinterpret_cast<uint4*>(out_buf));
+        }
       }
     }
     if (lane == 0) bulk_wait_group0();   // this warp's tensor stores are complete before the CTA exits
