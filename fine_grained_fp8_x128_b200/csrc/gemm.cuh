@@ -195,20 +195,6 @@ __device__ __forceinline__ void stage_store_pass4(uint4* stage, const uint4 (&ch
   __syncwarp();
 }
 
-// One pass of a tile-end tensor store: the warp's shared buffer (written in
-// the tensor map's swizzled layout) is stored as one box at (x, y) by lane 0,
-// which waits only until the buffer has been read; the global writes finish
-// in the background.
-__device__ __forceinline__ void tma_store_pass(uint8_t* buf, const CUtensorMap* tmap_d, int x, int y, int lane) {
-  fence_proxy_async_shared();   // the buffer's generic-proxy writes, before the async-proxy read
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(tmap_d, buf, x, y);
-    bulk_commit_group();
-    bulk_wait_group_read0();
-  }
-  __syncwarp();
-}
 
 // The tile-end store of a warp whose 32 rows are all valid, through tensor
 // stores of 128-byte boxes from two 4 KB buffers (the output's tensor map:

@@ -31,7 +31,7 @@
 // slot c; a proxy fence before each release orders those reads before the
 // refill.
 // At the end of a tile each epilogue warp writes its 32 rows x 128 columns
-// through a 4 KB shared buffer with TMA tensor stores (store_rows128_tma), so
+// through two 4 KB shared buffers with TMA tensor stores (store_rows128_tma), so
 // the global writes complete in the background while the warp returns to the
 // next tile's chunks.  The FP8 output keeps the staged 16-byte stores of
 // stage_store_pass (with its scales), and the FP8Q_SFB_ROW mode's 16x256b
@@ -43,7 +43,7 @@
 namespace fp8q {
 
 #ifndef FP8Q_PAIR_STAGES
-#define FP8Q_PAIR_STAGES 5
+#define FP8Q_PAIR_STAGES 4
 #endif
 constexpr int kPairStages = FP8Q_PAIR_STAGES;
 constexpr uint32_t kPairABytes = 128 * BK;                    // 16 KB
@@ -60,7 +60,7 @@ constexpr uint32_t kPairSaBytes = 128 * 4;
 template <int kSfbMode>
 __host__ __device__ constexpr uint32_t pair_sb_bytes() { return kSfbMode == FP8Q_SFB_ROW ? BN * 4 : 4 * 2 * 4; }
 
-constexpr uint32_t kPairOutStageBytes = 4096;                 // per epilogue warp: 32 rows x 128 bytes
+constexpr uint32_t kPairOutStageBytes = 8192;                 // per epilogue warp: two buffers of 32 rows x 128 bytes
 struct PairSmemLayout {
   static constexpr uint32_t stages = 0;
   static constexpr uint32_t scales = stages + kPairStages * kPairStageBytes;
@@ -107,34 +107,47 @@ __device__ __forceinline__ void promote_rows16(float2* acc, const uint32_t (&v)[
 
 // ---------------------------------------------------------------------------
 // Tile-end stores through TMA.  A warp's 32 rows x 128 columns leave in passes
-// of 32 rows x 128 bytes: the warp writes the pass into its 4 KB shared buffer
-// in the TMA's 128-byte-swizzled layout (16-byte chunk j of row r at chunk
-// j ^ (r % 8)), one lane issues a tensor store of the box and waits only
-// until the buffer has been read; the global writes complete in the
-// background while the warp goes on (to the next pass, then to the next
-// tile's chunks).  Rows past M are clipped by the tensor map.  (tma_store_pass
-// is in gemm.cuh.)
+// of 32 rows x 128 bytes: the warp writes each pass into one of its two 4 KB
+// shared buffers in the TMA's 128-byte-swizzled layout (16-byte chunk j of row
+// r at chunk j ^ (r % 8)) and one lane issues a tensor store of the box.  The
+// passes go out back to back; the warp waits for the TMA to have read the
+// buffers only when it next refills them (the FP32 output's third pass, or the
+// next tile's stores), so the global writes complete in the background while
+// the warp returns to the next tile's chunks.  Rows past M are clipped by the
+// tensor map.
 // ---------------------------------------------------------------------------
 // 32x32b fragments (thread = row `lane`, acc[j] = columns 2j, 2j+1 of the
 // warp's 128): BF16 in 2 passes of 64 columns, FP32 in 4 passes of 32.
 template <int kOut>
 __device__ __forceinline__ void store_rows128_tma(const float2* acc, int lane, int row0, int ncol0,
                                                   const CUtensorMap* tmap_d, uint8_t* buf) {
-  uint4* stage = reinterpret_cast<uint4*>(buf);
+  auto issue = [&](uint8_t* b, int x) {
+    fence_proxy_async_shared();
+    __syncwarp();
+    if (lane == 0) tma_store_2d(tmap_d, b, x, row0);
+  };
+  if (lane == 0) bulk_wait_group_read0();   // the previous tile's stores have read both buffers
+  __syncwarp();
   if (kOut == kOutF32) {
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
+      if (h == 2) {
+        if (lane == 0) { bulk_commit_group(); bulk_wait_group_read0(); }
+        __syncwarp();
+      }
+      uint4* stage = reinterpret_cast<uint4*>(buf + 4096 * (h & 1));
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float2 a = acc[16 * h + 2 * j], b = acc[16 * h + 2 * j + 1];
         stage[lane * 8 + (j ^ (lane & 7))] =
             make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y));
       }
-      tma_store_pass(buf, tmap_d, ncol0 + 32 * h, row0, lane);
+      issue(buf + 4096 * (h & 1), ncol0 + 32 * h);
     }
   } else {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      uint4* stage = reinterpret_cast<uint4*>(buf + 4096 * h);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         uint32_t w[4];
@@ -145,9 +158,11 @@ __device__ __forceinline__ void store_rows128_tma(const float2* acc, int lane, i
         }
         stage[lane * 8 + (j ^ (lane & 7))] = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      tma_store_pass(buf, tmap_d, ncol0 + 64 * h, row0, lane);
+      issue(buf + 4096 * h, ncol0 + 64 * h);
     }
   }
+  if (lane == 0) bulk_commit_group();
+  __syncwarp();
 }
 
 template <int kSfbMode, int kOut>
