@@ -157,3 +157,23 @@ def test_dispatch_gloo_ranks(T_list):
     # every routed entry was sent and received exactly once
     total_sent = sum(sum(s) for _, _, _, s in results)
     assert total_sent == sum(T_list) * k == sum(m for _, _, m, _ in results)
+
+
+def test_send_row_layout():
+    """A packed exchange row holds K codes then K/128 FP32 scales, padded to a
+    multiple of 16 bytes (the exchange and the GPU copies move 16-byte units),
+    and the two views read back what was written."""
+    import torch
+    from fine_grained_fp8_x128_b200.moe_dispatch import split_send_rows
+    for K in (128, 256, 384, 512, 2048, 4224, 7168):
+        w = send_row_bytes(K)
+        assert w % 16 == 0 and K + 4 * (K // 128) <= w < K + 4 * (K // 128) + 16
+        buf = torch.zeros((5, w), dtype=torch.uint8)
+        q, sf = split_send_rows(buf, K)
+        assert q.shape == (5, K) and sf.shape == (5, K // 128) and sf.dtype == torch.float32
+        assert q.stride(0) == w and sf.stride(0) * 4 == w
+        q[3] = 7
+        sf[3] = 2.5
+        row = buf[3].numpy()
+        assert np.all(row[:K] == 7) and np.all(row[K:K + 4 * (K // 128)].view(np.float32) == 2.5)
+        assert np.all(row[K + 4 * (K // 128):] == 0)
